@@ -1,0 +1,24 @@
+"""SVDQuant W4A4 (NVFP4) and AWQ W4A16 linear layers for NVIDIA B200 (sm_100a).
+
+The compute path is libsvdq.so (hand-written CUDA for sm_100a behind a C ABI,
+``include/svdq.h``); this package is its ctypes binding.  Importing fails if
+the library has not been built (``python -m bit_diffusion_transformer_act_b200.build``).
+"""
+
+from .ops import (  # noqa: F401
+    RANK,
+    SvdqError,
+    EXPORTED,
+    LIB,
+    svdq_packed_weight_bytes,
+    svdq_act_scale_bytes,
+    svdq_pack_weights,
+    svdq_unswizzle_scales,
+    svdq_swizzle_scales,
+    svdq_device_status,
+    svdq_quantize_act_lowrank_down,
+    svdq_w4a4_nvfp4_linear,
+    awq_w4a16_linear,
+    SvdqW4A4Linear,
+    AwqW4A16Linear,
+)

@@ -1,0 +1,61 @@
+// Byte layouts shared by the host packer and the CUDA launchers.
+//
+// Packed weight blob (device-private; produced on the host by svdq_pack_weights):
+//   [0, 256)     header: "SVDQNVF4", abi version, N, K, rank, g_w
+//   l1t          bf16 [rank][K]   L1 transposed (K contiguous) -- read by the
+//                                 activation kernel, which knows K but not N,
+//                                 so it comes first
+//   codes        u8   [N][K/2]    E2M1 codes of R, element 2i in the low nibble
+//   scales       u8   swizzled E4M3 block scales of R (128-row x 64-K atoms)
+//   l2t          bf16 [N][rank]   L2 transposed (rank contiguous)
+//   bias         bf16 [N]         zeros when the layer has no bias
+// Every section starts on a 1024-byte boundary.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace svdq {
+
+constexpr int kAbiVersion = 1;
+constexpr int kRank = 32;
+constexpr size_t kBlobAlign = 1024;
+
+struct BlobLayout {
+  size_t l1t, codes, scales, l2t, bias, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bytes of the swizzled scale tensor for `rows` rows and K columns (rows padded to 128).
+inline size_t swizzled_scale_bytes(size_t rows, size_t K) {
+  return align_up(rows, 128) * (K / 16);
+}
+
+// Offset of the scale of (row, group) in a swizzled scale tensor with K columns.
+inline size_t swizzled_scale_offset(size_t row, size_t group, size_t K) {
+  const size_t rb = row / 128, r = row % 128;
+  const size_t atom = group / 4, j = group % 4;
+  return (rb * (K / 64) + atom) * 512 + (r % 32) * 16 + (r / 32) * 4 + j;
+}
+
+inline BlobLayout blob_layout(size_t N, size_t K, size_t rank) {
+  BlobLayout L;
+  size_t off = kBlobAlign;                      // header, padded
+  L.l1t = off;    off = align_up(off + rank * K * 2, kBlobAlign);
+  L.codes = off;  off = align_up(off + N * K / 2, kBlobAlign);
+  L.scales = off; off = align_up(off + swizzled_scale_bytes(N, K), kBlobAlign);
+  L.l2t = off;    off = align_up(off + N * rank * 2, kBlobAlign);
+  L.bias = off;   off = align_up(off + N * 2, kBlobAlign);
+  L.total = off;
+  return L;
+}
+
+struct BlobHeader {
+  char magic[8];        // "SVDQNVF4"
+  int32_t abi_version;
+  int32_t N, K, rank;
+  float w_global_scale;
+};
+
+}  // namespace svdq

@@ -1,0 +1,267 @@
+// GPU entry points of libsvdq (declared in include/svdq.h): argument checks,
+// device checks, TMA descriptor encoding and kernel launches.  One translation
+// unit so that the device status word is shared by all kernels.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/svdq.h"
+#include "layout.h"
+#include "ptx.cuh"
+#include "quant_act.cuh"
+#include "gemm_nvfp4.cuh"
+#include "awq_w4a16.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2_scale(float g) {
+  if (!(g > 0.f) || !std::isfinite(g)) return false;
+  int e;
+  return std::frexp(static_cast<double>(g), &e) == 0.5;
+}
+
+// Current device, checked to be compute capability 10.0 (cached per device).
+int current_device_ok(int* dev_out) {
+  static int cc_major[kMaxDevices], cc_minor[kMaxDevices];
+  static bool known[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;
+  if (!known[dev]) {
+    if (cudaDeviceGetAttribute(&cc_major[dev], cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&cc_minor[dev], cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    known[dev] = true;
+  }
+  if (cc_major[dev] != 10 || cc_minor[dev] != 0) return SVDQ_ERR_ARCH;
+  *dev_out = dev;
+  return SVDQ_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes per element; box {box_cols, box_rows}.
+bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem, uint64_t rows, uint64_t cols,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raises the dynamic shared-memory limit of one kernel, once per device.
+template <auto Kernel>
+bool set_smem_once(int bytes, int dev) {
+  static bool done[kMaxDevices];
+  if (done[dev]) return true;
+  if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done[dev] = true;
+  return true;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                   int rank, float act_global_scale, void* act_codes, void* act_scales,
+                                   void* lowrank_act, void* stream) {
+  if (!X || !smooth_inv || !packed_w || !act_codes || !act_scales || !lowrank_act) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (rank != svdq::kRank || K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(smooth_inv) || !aligned16(packed_w) || !aligned16(act_codes) ||
+      !aligned16(act_scales) || !aligned16(lowrank_act))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  if (M == 0) return SVDQ_OK;
+
+  namespace k1 = svdq::k1;
+  const svdq::BlobLayout L = svdq::blob_layout(0, K, rank);   // the L1 section does not depend on N
+  k1::Params p;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.smooth = static_cast<const __nv_bfloat16*>(smooth_inv);
+  p.l1t = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(packed_w) + L.l1t);
+  p.codes = static_cast<uint8_t*>(act_codes);
+  p.scales = static_cast<uint8_t*>(act_scales);
+  p.U = static_cast<float*>(lowrank_act);
+  p.M = M;
+  p.K = K;
+  p.g = act_global_scale;
+  p.inv_g = 1.0f / act_global_scale;   // exact: a power of two
+
+  const int rowblocks = 2 * ((M + 127) / 128);         // 64-row CTAs covering the scale padding
+  const int kgroups = K / 64;
+  // K slices per row block (a cluster): the largest of 8, 4, 2, 1 that keeps slices whole
+  // (multiples of 64) and the grid within about four CTAs per SM
+  int ks = 1;
+  for (int c : {8, 4, 2, 1}) {
+    if (kgroups % c != 0) continue;
+    ks = c;
+    if (rowblocks * c <= 4 * 148) break;
+  }
+  p.kslices = ks;
+
+  const int smem = static_cast<int>(sizeof(k1::Smem));
+  if (!set_smem_once<k1::quant_act_lowrank_kernel>(smem, dev)) return SVDQ_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rowblocks, ks, 1);
+  cfg.blockDim = dim3(k1::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = ks;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                           float act_global_scale, const void* packed_w, float w_global_scale, int M, int N, int K,
+                           int rank, void* Y, void* stream) {
+  if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_scale(act_global_scale) || !is_pow2_scale(w_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
+      !aligned16(Y))
+    return SVDQ_ERR_INVALID_ARG;
+  const double alpha = static_cast<double>(act_global_scale) * w_global_scale;
+  if (!(alpha >= 0x1p-126 && alpha <= 0x1p126)) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  if (M == 0) return SVDQ_OK;
+
+  namespace k2 = svdq::k2;
+  const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
+  const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
+  k2::Params p;
+  p.sfa = static_cast<const uint8_t*>(act_scales);
+  p.sfb = blob + L.scales;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.alpha = static_cast<float>(alpha);
+  p.inv_alpha = static_cast<float>(1.0 / alpha);
+
+  const bool wide = (N % 256 == 0);
+  const int BN = wide ? 256 : 128;
+  CUtensorMap tA, tB, tU, tL2;
+  if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, 128, k2::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, BN,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, rank, rank, k2::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN,
+                 CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ERR_CUDA;
+
+  const dim3 grid(N / BN, (M + k2::BM - 1) / k2::BM, 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (wide) {
+    const int smem = k2::Cfg<256>::SMEM_BYTES;
+    if (!set_smem_once<k2::nvfp4_gemm_kernel<256>>(smem, dev)) return SVDQ_ERR_CUDA;
+    k2::nvfp4_gemm_kernel<256><<<grid, k2::kThreads, smem, s>>>(tA, tB, tU, tL2, p);
+  } else {
+    const int smem = k2::Cfg<128>::SMEM_BYTES;
+    if (!set_smem_once<k2::nvfp4_gemm_kernel<128>>(smem, dev)) return SVDQ_ERR_CUDA;
+    k2::nvfp4_gemm_kernel<128><<<grid, k2::kThreads, smem, s>>>(tA, tB, tU, tL2, p);
+  }
+  return launch_status();
+}
+
+int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, const void* zeros, const void* bias,
+                     int M, int N, int K, void* Y, void* stream) {
+  if (!X || !qweight || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (M > 64 || N % 64 != 0 || K % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(qweight) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(scales) & 7u) ||
+      (reinterpret_cast<uintptr_t>(zeros) & 7u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  if (M == 0) return SVDQ_OK;
+
+  namespace k3 = svdq::k3;
+  k3::Params p;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.qw = static_cast<const uint8_t*>(qweight);
+  p.scales = static_cast<const __nv_bfloat16*>(scales);
+  p.zeros = static_cast<const __nv_bfloat16*>(zeros);
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  const dim3 grid(N / k3::kRows, 1, 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+#define SVDQ_AWQ_LAUNCH(NT_)                                                              \
+  do {                                                                                    \
+    const int smem = static_cast<int>(sizeof(k3::Smem<NT_>));                             \
+    if (!set_smem_once<k3::awq_gemm_kernel<NT_>>(smem, dev)) return SVDQ_ERR_CUDA;        \
+    k3::awq_gemm_kernel<NT_><<<grid, k3::kThreads, smem, s>>>(p);                          \
+  } while (0)
+
+  if (M <= 8) SVDQ_AWQ_LAUNCH(1);
+  else if (M <= 16) SVDQ_AWQ_LAUNCH(2);
+  else if (M <= 32) SVDQ_AWQ_LAUNCH(4);
+  else SVDQ_AWQ_LAUNCH(8);
+#undef SVDQ_AWQ_LAUNCH
+  return launch_status();
+}
+
+int svdq_device_status(int clear) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, svdq::g_device_status, sizeof(v)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(svdq::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  }
+  return (v & 1u) ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,236 @@
+"""Python binding of libsvdq (include/svdq.h): argument marshalling only.
+
+Every function keeps the C name and forwards raw pointers and the current CUDA
+stream of PyTorch; PyTorch only provides device memory and streams.  There is
+no fallback: if the library is missing the import fails, and on a device that
+is not sm_100 the calls raise.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from .build import LIB_PATH
+
+RANK = 32
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device is not sm_100 (B200)",
+           4: "CUDA error", 5: "kernel wait timed out"}
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {_STATUS.get(status, 'unknown')} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libsvdq.so not built at {LIB_PATH}; run `python -m bit_diffusion_transformer_act_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "svdq_status_string": ([i], ctypes.c_char_p),
+        "svdq_abi_version": ([], i),
+        "svdq_packed_weight_bytes": ([i, i, i], sz),
+        "svdq_pack_weights": ([vp, vp, vp, vp, i, i, i, vp, sz, ctypes.POINTER(ctypes.c_float)], i),
+        "svdq_act_scale_bytes": ([i, i], sz),
+        "svdq_quantize_act_lowrank_down": ([vp, vp, vp, i, i, i, f, vp, vp, vp, vp], i),
+        "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
+        "awq_w4a16_linear": ([vp, vp, vp, vp, vp, i, i, i, vp, vp], i),
+        "svdq_unswizzle_scales": ([vp, i, i, vp], i),
+        "svdq_swizzle_scales": ([vp, i, i, vp], i),
+        "svdq_device_status": ([i], i),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+LIB = _load()
+EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes", "svdq_pack_weights",
+            "svdq_act_scale_bytes", "svdq_quantize_act_lowrank_down", "svdq_w4a4_nvfp4_linear",
+            "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status")
+
+
+def _check(fn, st):
+    if st != 0:
+        raise SvdqError(fn, st)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _np_ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _require(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected {dtype} tensor of shape {tuple(shape)}, got "
+                         f"{getattr(t, 'dtype', type(t))} {tuple(getattr(t, 'shape', ()))}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---------------------------------------------------------------- host side
+
+def svdq_packed_weight_bytes(N, K, rank=RANK):
+    return int(LIB.svdq_packed_weight_bytes(N, K, rank))
+
+
+def svdq_act_scale_bytes(M, K):
+    return int(LIB.svdq_act_scale_bytes(M, K))
+
+
+def svdq_pack_weights(R, L1_bits, L2_bits, bias_bits=None):
+    """R float32 [N, K]; L1 bf16 bits uint16 [K, r]; L2 bits [r, N]; bias bits [N] or None.
+
+    Returns (blob uint8 numpy array, w_global_scale float)."""
+    R = np.ascontiguousarray(R, dtype=np.float32)
+    N, K = R.shape
+    L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    rank = L1_bits.shape[1]
+    if L1_bits.shape != (K, rank) or L2_bits.shape != (rank, N):
+        raise ValueError("L1 must be [K, r] and L2 [r, N]")
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        if bias_bits.shape != (N,):
+            raise ValueError("bias must be [N]")
+    nbytes = svdq_packed_weight_bytes(N, K, rank)
+    if nbytes == 0:
+        _check("svdq_pack_weights", 2)
+    out = np.empty(nbytes, dtype=np.uint8)
+    g = ctypes.c_float(0.0)
+    st = LIB.svdq_pack_weights(_np_ptr(R), _np_ptr(L1_bits), _np_ptr(L2_bits), _np_ptr(bias_bits),
+                               N, K, rank, _np_ptr(out), nbytes, ctypes.byref(g))
+    _check("svdq_pack_weights", st)
+    return out, float(g.value)
+
+
+def svdq_unswizzle_scales(swizzled, rows, K):
+    """Swizzled scale bytes (numpy uint8 or a torch tensor) -> numpy uint8 [rows, K/16]."""
+    if isinstance(swizzled, torch.Tensor):
+        swizzled = swizzled.detach().cpu().numpy()
+    sw = np.ascontiguousarray(swizzled, dtype=np.uint8)
+    out = np.empty((rows, K // 16), dtype=np.uint8)
+    _check("svdq_unswizzle_scales", LIB.svdq_unswizzle_scales(_np_ptr(sw), rows, K, _np_ptr(out)))
+    return out
+
+
+def svdq_swizzle_scales(plain, rows, K):
+    plain = np.ascontiguousarray(plain, dtype=np.uint8)
+    out = np.empty(svdq_act_scale_bytes(rows, K), dtype=np.uint8)
+    _check("svdq_swizzle_scales", LIB.svdq_swizzle_scales(_np_ptr(plain), rows, K, _np_ptr(out)))
+    return out
+
+
+def svdq_device_status(clear=True):
+    """Synchronizes the device and returns the library's status word (0 or 5)."""
+    return int(LIB.svdq_device_status(1 if clear else 0))
+
+
+# ---------------------------------------------------------------- device side
+
+def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, rank=RANK,
+                                   act_codes=None, act_scales=None, lowrank_act=None):
+    """X bf16 [M, K] cuda; smooth_inv bf16 [K]; packed_w uint8 cuda (the blob).
+
+    Returns (act_codes uint8 [M, K/2], act_scales uint8 [svdq_act_scale_bytes], lowrank_act float32 [M, r])."""
+    M, K = X.shape
+    dev = X.device
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    if act_codes is None:
+        act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    if act_scales is None:
+        act_scales = torch.empty((svdq_act_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+    if lowrank_act is None:
+        lowrank_act = torch.empty((M, rank), dtype=torch.float32, device=dev)
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.float32, (M, rank), "lowrank_act")
+    st = LIB.svdq_quantize_act_lowrank_down(_ptr(X), _ptr(smooth_inv), _ptr(packed_w), M, K, rank,
+                                            float(act_global_scale), _ptr(act_codes), _ptr(act_scales),
+                                            _ptr(lowrank_act), _stream())
+    _check("svdq_quantize_act_lowrank_down", st)
+    return act_codes, act_scales, lowrank_act
+
+
+def svdq_w4a4_nvfp4_linear(act_codes, act_scales, lowrank_act, act_global_scale, packed_w, w_global_scale,
+                           M, N, K, rank=RANK, Y=None):
+    """Returns Y bf16 [M, N] = bf16(g_a g_w Q(X_hat) Q(R)^T + lowrank_act L2 + b)."""
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    st = LIB.svdq_w4a4_nvfp4_linear(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act),
+                                    float(act_global_scale), _ptr(packed_w), float(w_global_scale),
+                                    M, N, K, rank, _ptr(Y), _stream())
+    _check("svdq_w4a4_nvfp4_linear", st)
+    return Y
+
+
+def awq_w4a16_linear(X, qweight, scales, zeros, bias=None, Y=None):
+    """X bf16 [M, K]; qweight uint8 [N, K/2]; scales, zeros bf16 [N, K/64]; bias bf16 [N] or None."""
+    M, K = X.shape
+    N = qweight.shape[0]
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(qweight, torch.uint8, (N, K // 2), "qweight")
+    _require(scales, torch.bfloat16, (N, K // 64), "scales")
+    _require(zeros, torch.bfloat16, (N, K // 64), "zeros")
+    if bias is not None:
+        _require(bias, torch.bfloat16, (N,), "bias")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    st = LIB.awq_w4a16_linear(_ptr(X), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(bias), M, N, K,
+                              _ptr(Y), _stream())
+    _check("awq_w4a16_linear", st)
+    return Y
+
+
+# ---------------------------------------------------------------- layers
+
+class SvdqW4A4Linear:
+    """An SVDQuant W4A4 NVFP4 linear layer held on one GPU.
+
+    Built from the exporter's parameters: residual R [N, K] (float32), L1 [K, r],
+    L2 [r, N], bias [N] (bf16 bit patterns as uint16, or None), smooth_inv [K]
+    (bf16 bits) and the static activation scale g_a (a power of two)."""
+
+    def __init__(self, R, L1_bits, L2_bits, bias_bits, smooth_inv_bits, act_global_scale, device="cuda"):
+        blob, g_w = svdq_pack_weights(R, L1_bits, L2_bits, bias_bits)
+        self.N, self.K = R.shape
+        self.rank = L1_bits.shape[1]
+        self.packed = torch.from_numpy(blob).to(device)
+        self.w_global_scale = g_w
+        self.act_global_scale = float(act_global_scale)
+        self.smooth_inv = torch.from_numpy(np.ascontiguousarray(smooth_inv_bits, np.uint16).view(np.int16)) \
+            .view(torch.bfloat16).to(device)
+
+    def __call__(self, X, Y=None):
+        M = X.shape[0]
+        codes, scales, U = svdq_quantize_act_lowrank_down(X, self.smooth_inv, self.packed, self.act_global_scale,
+                                                          self.rank)
+        return svdq_w4a4_nvfp4_linear(codes, scales, U, self.act_global_scale, self.packed, self.w_global_scale,
+                                      M, self.N, self.K, self.rank, Y)
+
+
+class AwqW4A16Linear:
+    """An AWQ-style W4A16 int4 (group 64) linear layer held on one GPU."""
+
+    def __init__(self, qweight, scales, zeros, bias=None):
+        self.qweight, self.scales, self.zeros, self.bias = qweight, scales, zeros, bias
+
+    def __call__(self, X, Y=None):
+        return awq_w4a16_linear(X, self.qweight, self.scales, self.zeros, self.bias, Y)

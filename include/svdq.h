@@ -1,0 +1,178 @@
+/*
+ * svdq.h -- C ABI of libsvdq: the SVDQuant W4A4 (NVFP4) linear layer and the
+ * AWQ-style W4A16 (int4, group 64) linear layer on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  "Nunchaku Lite" (Hugging Face Diffusers docs), section
+ * "Supported quantization types": svdq_w4a4 with nvfp4 precision and group
+ * size 16 runs an NVFP4 runtime kernel with an SVDQ low-rank correction;
+ * awq_w4a16 with int4 precision and group size 64 runs an AWQ-style INT4
+ * weight-only kernel.  Section "NunchakuLiteQuantizationConfig": rank 32.  The
+ * Indonesian article on Nunchaku Lite (section on what happens when a
+ * diffusion model is quantized) describes the split: activation outliers go to
+ * a 16-bit low-rank branch, the rest runs with 4-bit weights and 4-bit
+ * activations.  The layer is
+ *
+ *     X_hat = X * smooth_inv                (smooth_inv[k] = 1/lambda_k)
+ *     y     = g_a g_w (Q(X_hat) Q(R)^T) + (X_hat L1) L2 + b
+ *
+ * with Q the NVFP4 quantizer: one E4M3 scale per 16 contiguous K elements,
+ * E2M1 codes, and a power-of-two per-tensor scale g (g_a for activations,
+ * supplied by the caller from calibration; g_w for the weight residual R,
+ * computed by svdq_pack_weights).  Block scale S = RNE_E4M3(amax/(6 g)),
+ * saturating at 448; code = RNE_E2M1(clamp(x/(S g), -6, 6)) with the IEEE sign
+ * kept; a block whose scale rounds to 0 gets all-zero codes.
+ *
+ * Conventions shared by every call.
+ *   - Matrices are row-major.  W, R are stored [N, K] (nn.Linear layout, K
+ *     contiguous); X, Y are [M, K] and [M, N].  bf16 tensors are passed as
+ *     uint16 bit patterns (host) or raw device pointers.
+ *   - Packed 4-bit codes: two per byte, element 2i in the low nibble.
+ *   - Scale-factor tensors ("swizzled scales") hold E4M3 codes in 512-byte
+ *     atoms of 128 rows x 4 scales (64 K elements): row blocks of 128 rows are
+ *     outermost, the K/64 atoms of a row block follow each other, and inside an
+ *     atom the scale of row i (0..127), group j (0..3) is at byte
+ *     (i % 32) * 16 + (i / 32) * 4 + j.  Row counts are padded up to 128.
+ *   - Ownership: the caller allocates and frees every buffer (host and
+ *     device).  The GPU entry points allocate nothing, never synchronize, and
+ *     enqueue their kernels on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) of the current device.
+ *   - Errors: every call checks its arguments first and returns a status
+ *     without launching anything when one is wrong.  Launch failures return
+ *     SVDQ_ERR_CUDA.  The kernels bound every wait on an mbarrier; a wait that
+ *     runs out (about one second) records SVDQ_ERR_TIMEOUT in a device-side
+ *     status word that svdq_device_status() reads, and the kernel releases its
+ *     tensor memory and returns instead of hanging.
+ *   - M == 0 is a valid empty call: it returns SVDQ_OK and launches nothing.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, bad count, misaligned pointer, non power-of-two scale */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* a dimension outside the supported tiling */
+  SVDQ_ERR_ARCH = 3,               /* current device is not compute capability 10.0 (B200) */
+  SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or a launch failed */
+  SVDQ_ERR_TIMEOUT = 5             /* a kernel gave up on a bounded wait (see svdq_device_status) */
+} svdq_status;
+
+/* Fixed parameters of the method table ("Supported quantization types"). */
+#define SVDQ_RANK 32
+#define SVDQ_NVFP4_GROUP 16
+#define SVDQ_AWQ_GROUP 64
+
+/* Human-readable name of a status code.  Never returns NULL. */
+const char* svdq_status_string(int status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+int svdq_abi_version(void);
+
+/* ------------------------------------------------------------------ weights */
+
+/* Bytes of the packed weight blob for an [N, K] residual with rank `rank`.
+ * Returns 0 for unsupported arguments (see svdq_pack_weights). */
+size_t svdq_packed_weight_bytes(int N, int K, int rank);
+
+/* Host-side weight preparation (no GPU work).
+ *   R     float32 [N, K]   residual weight W diag(lambda) - (L1 L2)^T.
+ *   L1    bf16   [K, rank] low-rank down factor (math orientation).
+ *   L2    bf16   [rank, N] low-rank up factor.
+ *   bias  bf16   [N] or NULL (then the bias is zero).
+ *   N % 128 == 0, K % 64 == 0, N, K > 0, rank == 32.
+ *   out   host buffer of out_bytes >= svdq_packed_weight_bytes(N, K, rank).
+ *   w_global_scale  receives g_w = 2^ceil(log2(amax(R) / 2688)) (1 if R == 0).
+ * The blob is device-private: copy it to the GPU as it is and pass that copy
+ * as `packed_w`.  It holds: a 256-byte header ("SVDQNVF4", N, K, rank, g_w),
+ * the NVFP4 codes of R [N, K/2], their swizzled E4M3 scales, L1 transposed to
+ * [rank, K], L2 transposed to [N, rank] and the bias [N] (bf16), each section
+ * aligned to 1024 bytes.  Codes and scales are bit-exact to the definition
+ * above (RNE on exact quotients).
+ * Returns SVDQ_ERR_INVALID_ARG for null pointers or a short buffer, and
+ * SVDQ_ERR_UNSUPPORTED_SHAPE for dimensions outside the rules above, or when R
+ * holds a NaN or infinity. */
+int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
+                      const uint16_t* bias, int N, int K, int rank,
+                      void* out, size_t out_bytes, float* w_global_scale);
+
+/* ------------------------------------------------------------- activations */
+
+/* Bytes of a swizzled activation-scale buffer for M rows and K columns:
+ * ceil(M/128)*128 * K/16.  Rows M..ceil(M/128)*128-1 are written as zero. */
+size_t svdq_act_scale_bytes(int M, int K);
+
+/* Kernel 1: smoothing, NVFP4 quantization and the rank-32 down-projection, in
+ * one pass over X (the article's "16-bit low-rank branch" is fed from the same
+ * smoothed values that are quantized).
+ *   X           device bf16 [M, K] (16-byte aligned rows: K % 64 == 0)
+ *   smooth_inv  device bf16 [K], the per-channel 1/lambda
+ *   packed_w    device copy of the blob from svdq_pack_weights (its L1 is used;
+ *               N is not needed here)
+ *   act_global_scale  g_a > 0, a power of two (static calibration)
+ *   act_codes   device u8 [M, K/2] out: E2M1 codes of X_hat
+ *   act_scales  device u8 [svdq_act_scale_bytes(M, K)] out: swizzled E4M3 scales
+ *   lowrank_act device float32 [M, rank] out: X_hat L1.  X_hat is split
+ *               exactly into two bf16 parts for the tensor cores, so the only
+ *               rounding is the fp32 accumulation.
+ * K % 64 == 0, rank == 32, M >= 0.  Asynchronous on `stream`. */
+int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv,
+                                   const void* packed_w, int M, int K, int rank,
+                                   float act_global_scale, void* act_codes,
+                                   void* act_scales, void* lowrank_act, void* stream);
+
+/* Kernel 2: the NVFP4 block-scaled GEMM on tcgen05 with the low-rank up
+ * projection, the bias and the bf16 cast fused in the epilogue:
+ *   Y = bf16( g_a g_w (Q(X_hat) Q(R)^T) + lowrank_act L2 + b ).
+ * The fp32 lowrank_act is split exactly into two bf16 parts for the tensor
+ * cores; all products are exact and accumulate in fp32.
+ *   act_codes, act_scales, lowrank_act  outputs of kernel 1 for the same M, K
+ *   act_global_scale  the g_a given to kernel 1 (power of two)
+ *   packed_w          device copy of the blob; w_global_scale its g_w
+ *   Y                 device bf16 [M, N] out
+ * N % 128 == 0, K % 64 == 0, rank == 32, M >= 0; all pointers 16-byte
+ * aligned.  Asynchronous on `stream`. */
+int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
+                           const void* lowrank_act, float act_global_scale,
+                           const void* packed_w, float w_global_scale,
+                           int M, int N, int K, int rank, void* Y, void* stream);
+
+/* ---------------------------------------------------------------- AWQ W4A16 */
+
+/* Kernel 3: y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.
+ *   X        device bf16 [M, K]
+ *   qweight  device u8 [N, K/2], element 2i of a row in the low nibble
+ *   scales   device bf16 [N, K/64]
+ *   zeros    device bf16 [N, K/64], integer zero points 0..15
+ *   bias     device bf16 [N] or NULL
+ *   Y        device bf16 [M, N] out
+ * 1 <= M <= 64 (or M == 0), N % 64 == 0, K % 256 == 0; pointers 16-byte
+ * aligned.  The products (q - z) x are exact and each group's partial sum is
+ * scaled by s in fp32.  Asynchronous on `stream`. */
+int awq_w4a16_linear(const void* X, const void* qweight, const void* scales,
+                     const void* zeros, const void* bias, int M, int N, int K,
+                     void* Y, void* stream);
+
+/* ----------------------------------------------------------------- helpers */
+
+/* Host: convert a swizzled scale buffer (rows rounded up to 128) into plain
+ * row-major [rows, K/16] E4M3 codes, and back. */
+int svdq_unswizzle_scales(const void* swizzled, int rows, int K, uint8_t* out);
+int svdq_swizzle_scales(const uint8_t* plain, int rows, int K, void* swizzled);
+
+/* Reads (and with clear != 0, resets) the device-side status word of the
+ * current device that kernels set when a bounded wait runs out.  Returns
+ * SVDQ_OK or SVDQ_ERR_TIMEOUT; SVDQ_ERR_CUDA if the read itself failed.
+ * This call synchronizes the device; it is meant for tests and diagnostics. */
+int svdq_device_status(int clear);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SVDQ_H_ */

@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every declared symbol, and checks its arguments
+(host-side logic only; no kernel runs here)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from bit_diffusion_transformer_act_b200 import build as _build
+
+_build.build()
+import bit_diffusion_transformer_act_b200 as P  # noqa: E402
+
+from parity_util import swizzled_offset, unswizzle  # noqa: E402
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "svdq.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)) - {"if"}
+
+
+def test_header_declares_the_expected_entry_points():
+    decl = _declared_functions()
+    for name in ("svdq_pack_weights", "svdq_quantize_act_lowrank_down", "svdq_w4a4_nvfp4_linear",
+                 "awq_w4a16_linear"):
+        assert name in decl
+    assert decl == set(P.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", P.ops.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in _declared_functions():
+        assert name in exported, name
+        assert getattr(P.LIB, name) is not None
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert P.LIB.svdq_status_string(s)
+    assert P.LIB.svdq_status_string(99) == b"unknown status"
+    assert P.LIB.svdq_abi_version() == 1
+
+
+def test_sizes():
+    assert P.svdq_packed_weight_bytes(3072, 3072) > 3072 * 1536
+    assert P.svdq_packed_weight_bytes(100, 3072) == 0          # N % 128
+    assert P.svdq_packed_weight_bytes(128, 100) == 0           # K % 64
+    assert P.svdq_packed_weight_bytes(128, 64, 16) == 0        # rank
+    assert P.svdq_act_scale_bytes(1, 64) == 128 * 4
+    assert P.svdq_act_scale_bytes(129, 128) == 256 * 8
+    assert P.svdq_act_scale_bytes(0, 64) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced: every case below fails its checks first
+
+
+def test_gpu_entry_points_reject_bad_arguments_before_any_device_work():
+    L = P.LIB
+    # null pointers
+    assert L.svdq_quantize_act_lowrank_down(None, FAKE, FAKE, 4, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, None, 1.0, FAKE, 1.0, 4, 128, 64, 32, FAKE, None) == 1
+    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 256, None, None) == 1
+    # scales that are not powers of two
+    assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 64, 32, 0.3, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, -2.0, 4, 128, 64, 32, FAKE, None) == 1
+    # unsupported shapes
+    assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 96, 32, 1.0, FAKE, FAKE, FAKE, None) == 2
+    assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 64, 16, 1.0, FAKE, FAKE, FAKE, None) == 2
+    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 192, 64, 32, FAKE, None) == 2
+    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 65, 64, 256, FAKE, None) == 2
+    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 320, FAKE, None) == 2
+    # misaligned pointers
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.svdq_quantize_act_lowrank_down(odd, FAKE, FAKE, 4, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 128, 64, 32, odd, None) == 1
+    # negative sizes
+    assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, -1, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_a_cuda_error():
+    assert P.LIB.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 4
+
+
+def test_swizzle_helpers_follow_the_documented_layout():
+    rng = np.random.default_rng(0)
+    for rows, K in [(1, 64), (130, 192), (256, 512)]:
+        plain = rng.integers(0, 256, size=(rows, K // 16)).astype(np.uint8)
+        sw = P.svdq_swizzle_scales(plain, rows, K)
+        assert sw.size == P.svdq_act_scale_bytes(rows, K)
+        assert np.array_equal(unswizzle(sw, rows, K), plain)
+        assert np.array_equal(P.svdq_unswizzle_scales(sw, rows, K), plain)
+    # one byte placed by hand: row 37 (lane 5 of quarter 1), group 6 (atom 1, slot 2), K = 128
+    assert swizzled_offset(37, 6, 128) == 512 + 5 * 16 + 1 * 4 + 2

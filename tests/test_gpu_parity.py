@@ -1,0 +1,212 @@
+"""GPU parity of the three kernels against the float64 oracle, through the C ABI.
+
+Bars: packed activation codes and scales bit-exact; the low-rank activations
+within fp32 accumulation error of the exact product; layer outputs within
+relative L2 5e-3 and, per element, max(1e-2 rms(y), 1 bf16 ulp) of the
+oracle rounded to bf16.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import awq as oawq
+from oracle import nvfp4, svdq
+from parity_util import check_output, unswizzle
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+
+
+def _pack(P, w, with_bias=True):
+    blob, gw = P.svdq_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2),
+                                   synth.bf16_bits(w.bias) if with_bias else None)
+    return torch.from_numpy(blob).cuda(), gw
+
+
+def _run_svdq(P, X, smooth, packed, g_a, g_w, N):
+    M, K = X.shape
+    Xd, sd = _bf16_dev(X), _bf16_dev(smooth)
+    codes, scales, U = P.svdq_quantize_act_lowrank_down(Xd, sd, packed, g_a)
+    Y = P.svdq_w4a4_nvfp4_linear(codes, scales, U, g_a, packed, g_w, M, N, K)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy(), U.cpu().numpy(), Y.float().cpu().numpy()
+
+
+def _check_act(codes, scales, U, X, smooth, L1, g_a):
+    M, K = X.shape
+    cx, sx = svdq.quantize_activations(X, smooth, g_a)
+    assert np.array_equal(codes, nvfp4.pack_nibbles(cx)), np.argwhere(codes != nvfp4.pack_nibbles(cx))[:5]
+    rows = (M + 127) // 128 * 128
+    sg = unswizzle(scales, rows, K)
+    assert np.array_equal(sg[:M], sx), np.argwhere(sg[:M] != sx)[:5]
+    assert np.all(sg[M:] == 0)
+    Xh = svdq.smooth(X, smooth)
+    U_ref = Xh @ L1.astype(np.float64)
+    bound = 1e-5 * (np.abs(Xh) @ np.abs(L1.astype(np.float64))) + 1e-30
+    assert np.all(np.abs(U - U_ref) <= bound), np.max(np.abs(U - U_ref) / bound)
+
+
+# ---------------------------------------------------------------- edge-case activations
+
+def _edge_activations(M, K, seed):
+    """bf16 activations with zero rows, negative zeros, exact E2M1 and E4M3 midpoints."""
+    rng = np.random.default_rng(seed)
+    smooth = np.exp2(rng.integers(-2, 3, size=K)).astype(np.float32)       # powers of two: x_hat exact
+    g_a = 2.0 ** -2
+    X = synth.to_bf16(rng.standard_normal((M, K)) * np.exp2(rng.integers(-3, 4, size=(M, 1))))
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 3.0, 6.0])
+    for m in range(M):
+        kind = m % 7
+        if kind == 1:
+            X[m] = 0.0
+        elif kind == 2:
+            X[m, ::3] = -0.0
+            X[m, 1::3] = -1e-30
+        elif kind in (3, 4):
+            S = nvfp4.E4M3_TABLE[rng.integers(1, 0x7F, size=K // 16)].repeat(16)
+            v = rng.choice(mids, size=K) * rng.choice([-1.0, 1.0], size=K) * S * g_a
+            v[::16] = 6.0 * S[::16] * g_a
+            if kind == 4:
+                v[5::16] = -6.375 * S[5::16] * g_a                        # scale tie: amax/6 on a midpoint
+            X[m] = (v / smooth).astype(np.float32)
+    assert np.array_equal(synth.to_bf16(X), X)
+    return X, smooth, g_a
+
+
+@pytest.fixture(scope="module")
+def P(cuda_lib):
+    return cuda_lib
+
+
+def test_tiny_layer(P):
+    w = synth.svdq_workload(256, 512, 512)
+    packed, gw = _pack(P, w)
+    codes, scales, U, Y = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, 512)
+    _check_act(codes, scales, U, w.X, w.smooth_inv, w.L1, w.g_a)
+    y_ref = svdq.forward(w.X, w.smooth_inv, w.R, w.L1, w.L2, w.bias, w.g_a)
+    check_output(Y, y_ref)
+    assert P.svdq_device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 64, 128), (63, 192, 256), (65, 320, 128), (127, 512, 384),
+                                   (129, 256, 640), (200, 1024, 256), (300, 448, 512)])
+def test_edge_shapes_and_values(P, M, K, N):
+    X, smooth, g_a = _edge_activations(M, K, seed=M * 7 + K)
+    rng = np.random.default_rng(K + N)
+    R = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    R[N // 2] = 0.0                                                        # a zero weight row
+    L1 = synth.to_bf16(rng.standard_normal((K, 32)) * 0.1)
+    L2 = synth.to_bf16(rng.standard_normal((32, N)) * 0.1)
+    b = synth.to_bf16(rng.standard_normal(N) * 0.01)
+    blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2), synth.bf16_bits(b))
+    packed = torch.from_numpy(blob).cuda()
+    codes, scales, U, Y = _run_svdq(P, X, smooth, packed, g_a, gw, N)
+    _check_act(codes, scales, U, X, smooth, L1, g_a)
+    check_output(Y, svdq.forward(X, smooth, R, L1, L2, b, g_a))
+
+
+def test_no_bias_and_empty_batch(P):
+    w = synth.svdq_workload(96, 256, 128, with_bias=False)
+    packed, gw = _pack(P, w, with_bias=False)
+    *_, Y = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, 128)
+    check_output(Y, svdq.forward(w.X, w.smooth_inv, w.R, w.L1, w.L2, None, w.g_a))
+    # M == 0: a valid empty call
+    Xd = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    codes, scales, U = P.svdq_quantize_act_lowrank_down(Xd, _bf16_dev(w.smooth_inv), packed, w.g_a)
+    Y0 = P.svdq_w4a4_nvfp4_linear(codes, scales, U, w.g_a, packed, gw, 0, 128, 256)
+    assert Y0.shape == (0, 128)
+
+
+def test_repeat_calls_are_deterministic(P):
+    w = synth.svdq_workload(384, 1024, 512)
+    packed, gw = _pack(P, w)
+    a = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, 512)
+    b = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, 512)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+# ---------------------------------------------------------------- full-size layers (sampled outputs)
+
+FULL = [
+    ("attention 4096x3072->3072", 4096, 3072, 3072, False),
+    ("mlp-up 4608x3072->12288", 4608, 3072, 12288, False),
+    ("mlp-down 4608x12288->3072 (gelu)", 4608, 12288, 3072, True),
+    ("qkv 64x3072->9216", 64, 3072, 9216, False),
+    ("qkv 18432x3072->9216", 18432, 3072, 9216, False),
+]
+
+
+@pytest.mark.parametrize("name,M,K,N,gelu", FULL, ids=[f[0] for f in FULL])
+def test_full_size_layer(P, name, M, K, N, gelu):
+    w = synth.svdq_workload(M, K, N, gelu_input=gelu)
+    packed, gw = _pack(P, w)
+    codes, scales, U, Y = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, N)
+    rng = np.random.default_rng(11)
+    rows = np.sort(rng.choice(M, size=min(M, 256), replace=False))
+    # activation codes and scales: every row (bit-exact), low-rank on the sampled rows
+    cx, sx = svdq.quantize_activations(w.X, w.smooth_inv, w.g_a)
+    assert np.array_equal(codes, nvfp4.pack_nibbles(cx))
+    assert np.array_equal(unswizzle(scales, (M + 127) // 128 * 128, K)[:M], sx)
+    Xh = svdq.smooth(w.X[rows], w.smooth_inv)
+    U_ref = Xh @ w.L1.astype(np.float64)
+    assert np.all(np.abs(U[rows] - U_ref) <= 1e-5 * (np.abs(Xh) @ np.abs(w.L1.astype(np.float64))) + 1e-30)
+    y_ref = svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, w.g_a)
+    check_output(Y[rows], y_ref)
+    assert P.svdq_device_status() == 0
+
+
+# ---------------------------------------------------------------- AWQ W4A16
+
+def _run_awq(P, a, bias=None):
+    X = _bf16_dev(a.X)
+    qw = torch.from_numpy(a.qweight).cuda()
+    s = _bf16_dev(a.scales)
+    z = _bf16_dev(a.zeros)
+    bd = _bf16_dev(bias) if bias is not None else None
+    Y = P.awq_w4a16_linear(X, qw, s, z, bd)
+    torch.cuda.synchronize()
+    return Y.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (9, 256, 64), (16, 1024, 256),
+                                   (33, 512, 320), (64, 256, 128), (64, 1536, 512)])
+def test_awq_shapes(P, M, K, N):
+    a = synth.awq_workload(M, K, N, seed=M + K)
+    b = synth.to_bf16(np.random.default_rng(N).standard_normal(N) * 0.1) if M % 2 else None
+    Y = _run_awq(P, a, b)
+    check_output(Y, oawq.forward(a.X, a.q, a.scales, a.zeros, b))
+
+
+def test_awq_integer_case_is_exact(P):
+    # s = 1, z = 8, small integer activations: every partial sum is an exact integer in fp32
+    rng = np.random.default_rng(3)
+    M, K, N = 5, 512, 128
+    a = synth.awq_workload(M, K, N)
+    a.X[:] = rng.integers(-4, 5, size=(M, K))
+    a.scales[:] = 1.0
+    a.zeros[:] = 8.0
+    Y = _run_awq(P, a)
+    ref = a.X.astype(np.int64) @ (a.q.astype(np.int64) - 8).T
+    assert np.array_equal(Y, synth.to_bf16(ref.astype(np.float64)))
+
+
+@pytest.fixture(scope="module")
+def awq_full():
+    a = synth.awq_workload(64, 3072, 18432)
+    deq = oawq.dequantize(a.q, a.scales, a.zeros)
+    return a, deq
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 64])
+def test_awq_adaln_full_size(P, awq_full, M):
+    a, deq = awq_full
+    sub = synth.AwqWorkload(M, a.K, a.N, a.X[:M].copy(), a.q, a.qweight, a.scales, a.zeros, a.W)
+    Y = _run_awq(P, sub)
+    check_output(Y, a.X[:M].astype(np.float64) @ deq.T)
+    assert P.svdq_device_status() == 0

@@ -1,0 +1,91 @@
+"""Host weight packing (C++) against the oracle: bit-exact codes, scales and g_w."""
+
+import numpy as np
+import pytest
+
+from bit_diffusion_transformer_act_b200 import build as _build
+
+_build.build()
+import bit_diffusion_transformer_act_b200 as P  # noqa: E402
+
+from oracle import nvfp4, svdq  # noqa: E402
+import synth  # noqa: E402
+from parity_util import unswizzle  # noqa: E402
+
+
+def _sections(blob, N, K, rank=32):
+    al = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
+    off = 1024
+    l1t = off; off = al(off + rank * K * 2)
+    codes = off; off = al(off + N * K // 2)
+    scales = off; off = al(off + ((N + 127) // 128 * 128) * (K // 16))
+    l2t = off; off = al(off + N * rank * 2)
+    bias = off; off = al(off + N * 2)
+    assert off == blob.size
+    return {
+        "l1t": blob[l1t:l1t + rank * K * 2].view(np.uint16).reshape(rank, K),
+        "codes": blob[codes:codes + N * K // 2].reshape(N, K // 2),
+        "scales": blob[scales:scales + ((N + 127) // 128 * 128) * (K // 16)],
+        "l2t": blob[l2t:l2t + N * rank * 2].view(np.uint16).reshape(N, rank),
+        "bias": blob[bias:bias + N * 2].view(np.uint16),
+    }
+
+
+def _check_pack(R, L1, L2, b):
+    N, K = R.shape
+    blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2),
+                                   None if b is None else synth.bf16_bits(b))
+    cw, sw, gw_ref = svdq.quantize_weights(R)
+    assert gw == gw_ref
+    s = _sections(blob, N, K)
+    assert np.array_equal(s["codes"], nvfp4.pack_nibbles(cw))
+    assert np.array_equal(unswizzle(s["scales"], N, K), sw)
+    assert np.array_equal(s["l1t"], synth.bf16_bits(L1).T)
+    assert np.array_equal(s["l2t"], synth.bf16_bits(L2).T)
+    assert np.array_equal(s["bias"], np.zeros(N, np.uint16) if b is None else synth.bf16_bits(b))
+    assert bytes(blob[:8]) == b"SVDQNVF4"
+    return blob
+
+
+def test_pack_synthetic_tiny_layer_is_bit_exact():
+    w = synth.svdq_workload(256, 512, 512)
+    _check_pack(w.R, w.L1, w.L2, w.bias)
+
+
+def test_pack_attention_layer_is_bit_exact():
+    w = synth.svdq_workload(64, 3072, 3072)
+    _check_pack(w.R, w.L1, w.L2, None)
+
+
+def test_pack_ties_zero_blocks_and_subnormal_scales():
+    rng = np.random.default_rng(5)
+    N, K = 128, 256
+    g = 2.0 ** -4
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0])
+    R = np.zeros((N, K))
+    for n in range(N):
+        kind = n % 5
+        if kind == 0:
+            continue                                        # zero row -> zero scales and codes
+        S = nvfp4.E4M3_TABLE[rng.integers(1, 0x7F)] if kind != 3 else 2.0 ** -9
+        blk = rng.choice(mids, size=K) * rng.choice([-1.0, 1.0], size=K) * S * g
+        blk[::16] = 6.0 * S * g                             # every block's amax is 6 S g
+        if kind == 4:
+            blk[1::16] = 6.375 * S * g                      # amax/6 lands between two E4M3 values
+        R[n] = blk
+    R[1, 0] = 6.0 * 448 * g                                 # pins g_w
+    R = R.astype(np.float32)
+    L1 = synth.to_bf16(rng.standard_normal((K, 32)))
+    L2 = synth.to_bf16(rng.standard_normal((32, N)))
+    _check_pack(R, L1, L2, synth.to_bf16(rng.standard_normal(N)))
+
+
+def test_pack_rejects_bad_shapes_and_values():
+    L1 = np.zeros((64, 32), np.float32)
+    L2 = np.zeros((32, 128), np.float32)
+    with pytest.raises(P.SvdqError):
+        P.svdq_pack_weights(np.zeros((100, 64), np.float32), L1, np.zeros((32, 100), np.float32))
+    R = np.zeros((128, 64), np.float32)
+    R[3, 5] = np.nan
+    with pytest.raises(P.SvdqError):
+        P.svdq_pack_weights(R, L1, L2)
