@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly (for profilers)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="one resident copy, eager launches of every kernel (for ncu captures); prints timings")
     return ap.parse_args()
 
 
@@ -508,8 +510,36 @@ def run_reference(args, world, rank):
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile_case(args):
+    """Each kernel launched eagerly `steps` times on one resident copy of the workload."""
+    import torch
+    import bit_diffusion_transformer_act_b200 as P
+    global NSETS
+    NSETS = 1
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = Workload(P, dev)
+    out = {}
+    jobs = [("k1", lambda: wl.k1(P, 0)), ("k2", lambda: wl.k2(P, 0))] + \
+           [("awq%d" % m, (lambda m=m: wl.awq(P, 0, m))) for m in AWQ_MS]
+    for name, fn in jobs:
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name + "_us"] = e0.elapsed_time(e1) * 1e3 / args.steps
+    out["device_status"] = P.svdq_device_status()
+    return out
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        print(json.dumps({"profile_case": run_profile_case(args)}))
+        return
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         out = run_reference(args, world, rank)

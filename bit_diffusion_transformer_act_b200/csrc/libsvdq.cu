@@ -96,16 +96,16 @@ extern "C" {
 int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
                                    int rank, float act_global_scale, void* act_codes, void* act_scales,
                                    void* lowrank_act, void* stream) {
-  if (!X || !smooth_inv || !packed_w || !act_codes || !act_scales || !lowrank_act) return SVDQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
   if (rank != svdq::kRank || K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;                       // empty batch: nothing to read or write
+  if (!X || !smooth_inv || !packed_w || !act_codes || !act_scales || !lowrank_act) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(smooth_inv) || !aligned16(packed_w) || !aligned16(act_codes) ||
       !aligned16(act_scales) || !aligned16(lowrank_act))
     return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
-  if (M == 0) return SVDQ_OK;
 
   namespace k1 = svdq::k1;
   const svdq::BlobLayout L = svdq::blob_layout(0, K, rank);   // the L1 section does not depend on N
@@ -158,10 +158,11 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
 int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act,
                            float act_global_scale, const void* packed_w, float w_global_scale, int M, int N, int K,
                            int rank, void* Y, void* stream) {
-  if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
   if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_scale(act_global_scale) || !is_pow2_scale(w_global_scale)) return SVDQ_ERR_INVALID_ARG;
   if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
       !aligned16(Y))
     return SVDQ_ERR_INVALID_ARG;
@@ -169,7 +170,6 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   if (!(alpha >= 0x1p-126 && alpha <= 0x1p126)) return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
-  if (M == 0) return SVDQ_OK;
 
   namespace k2 = svdq::k2;
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
@@ -214,15 +214,15 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
 
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, const void* zeros, const void* bias,
                      int M, int N, int K, void* Y, void* stream) {
-  if (!X || !qweight || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
   if (M < 0 || N <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
   if (M > 64 || N % 64 != 0 || K % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !qweight || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(qweight) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(scales) & 7u) ||
       (reinterpret_cast<uintptr_t>(zeros) & 7u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)))
     return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
-  if (M == 0) return SVDQ_OK;
 
   namespace k3 = svdq::k3;
   k3::Params p;

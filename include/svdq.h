@@ -42,7 +42,9 @@
  *     runs out (about one second) records SVDQ_ERR_TIMEOUT in a device-side
  *     status word that svdq_device_status() reads, and the kernel releases its
  *     tensor memory and returns instead of hanging.
- *   - M == 0 is a valid empty call: it returns SVDQ_OK and launches nothing.
+ *   - M == 0 is a valid empty call: once the sizes and scales pass their
+ *     checks it returns SVDQ_OK without touching the device (the M-sized
+ *     buffers may then be NULL).
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_

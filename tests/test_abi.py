@@ -84,6 +84,10 @@ def test_gpu_entry_points_reject_bad_arguments_before_any_device_work():
     assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 128, 64, 32, odd, None) == 1
     # negative sizes
     assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, -1, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
+    # an empty batch is valid even with null buffers, and needs no device
+    assert L.svdq_quantize_act_lowrank_down(None, None, None, 0, 64, 32, 1.0, None, None, None, None) == 0
+    assert L.svdq_w4a4_nvfp4_linear(None, None, None, 1.0, None, 1.0, 0, 128, 64, 32, None, None) == 0
+    assert L.awq_w4a16_linear(None, None, None, None, None, 0, 64, 256, None, None) == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")

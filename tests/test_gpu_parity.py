@@ -66,9 +66,12 @@ def _edge_activations(M, K, seed):
             X[m] = 0.0
         elif kind == 2:
             X[m, ::3] = -0.0
-            X[m, 1::3] = -1e-30
+            X[m, 1::3] = synth.to_bf16(np.full(len(X[m, 1::3]), -1e-30))
         elif kind in (3, 4):
-            S = nvfp4.E4M3_TABLE[rng.integers(1, 0x7F, size=K // 16)].repeat(16)
+            if kind == 3:
+                S = nvfp4.E4M3_TABLE[rng.integers(1, 0x7F, size=K // 16)].repeat(16)
+            else:                                                          # powers of two keep 6.375 S in bf16
+                S = np.exp2(rng.integers(-9, 9, size=K // 16)).repeat(16)
             v = rng.choice(mids, size=K) * rng.choice([-1.0, 1.0], size=K) * S * g_a
             v[::16] = 6.0 * S[::16] * g_a
             if kind == 4:
