@@ -180,7 +180,7 @@ class Workload:
         M, K, N = SVDQ_SHAPE
         w = synth.svdq_workload(M, K, N)
         blob, self.g_w = P.svdq_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2),
-                                             synth.bf16_bits(w.bias))
+                                             synth.bf16_bits(w.bias), synth.bf16_bits(w.smooth_inv))
         self.g_a = w.g_a
         self.M, self.K, self.N = M, K, N
         X = bf16_dev(w.X, dev)
@@ -193,7 +193,7 @@ class Workload:
                 "X": X.clone(), "W": blob_d.clone(),
                 "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
                 "scales": torch.empty((P.svdq_act_scale_bytes(M, K),), dtype=torch.uint8, device=dev),
-                "U": torch.empty((M, RANK), dtype=torch.float32, device=dev),
+                "U": torch.empty((M, 2 * RANK), dtype=torch.bfloat16, device=dev),
                 "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
             })
         a = synth.awq_workload(max(AWQ_MS), AWQ_K, AWQ_N)
@@ -229,7 +229,7 @@ def svdq_flops():
 
 def k1_bytes():
     M, K, N = SVDQ_SHAPE
-    return 2 * M * K + 2 * K + 2 * K * RANK + M * K / 2 + M * K / 16 + 4 * M * RANK
+    return 2 * M * K + 2 * K + 4 * K * RANK + M * K / 2 + M * K / 16 + 4 * M * RANK
 
 
 def k2_bytes():

@@ -10,20 +10,19 @@
 //   warp 0  TMA producer: E2M1 code tiles of A (activations) and B (weights)
 //           through a 3-stage ring of 128-byte-swizzled shared-memory tiles
 //           (256 K elements per stage), their E4M3 scale atoms by bulk copy,
-//           and once per tile the fp32 U tile [128 x 32] and the bf16 L2^T tile [BN x 32].
+//           and once per tile the low-rank activation tile [128 x 64] (bf16 hi | lo of
+//           U / g_a) and the (L2 / g_w)^T tile [BN x 32].
 //   warp 1  allocates tensor memory and issues, from one thread, the scale
 //           copies (tcgen05.cp, shared -> tensor memory, 4 columns per 128 rows
 //           per MMA) and the block-scaled MMAs
 //           (kind::mxf4nvf4, block16 = one UE4M3 scale per 16 K, K = 64 per
 //           instruction, fp32 accumulator in tensor memory); after the K loop,
-//           four bf16 MMAs (K = 16 each) add [U'_hi | U'_lo] [L2 | L2]^T into the
-//           same accumulator.
-//   warps 2-5  epilogue: while the K loop runs they turn the fp32 U tile into
-//           U' = U / alpha (exact: alpha is a power of two) split exactly into
-//           bf16 hi + lo, laid out as a 128-byte-swizzled K-major tile, so the
-//           accumulator ends as Acc + U L2 / alpha; then they read it from
-//           tensor memory (32 columns per tcgen05.ld), apply alpha and the
-//           bias with one fma, round to bf16 and store.
+//           four bf16 MMAs (K = 16 each) add [U_hi | U_lo] [L2 | L2]^T / (g_a g_w)
+//           into the same accumulator (both operands were pre-scaled by powers of
+//           two, so the accumulator ends as Acc + U L2 / alpha exactly).
+//   warps 2-5  epilogue: read the accumulator from tensor memory (32 columns
+//           per tcgen05.ld), apply alpha and the bias with one fma, round to
+//           bf16 and store.
 // Every mbarrier wait is bounded (about one second); a wait that runs out
 // records SVDQ_ERR_TIMEOUT in the device status word, makes the other roles
 // give up, drains the copies and MMAs in flight (bounded too), frees the
@@ -46,15 +45,13 @@ struct Cfg {
   static constexpr int B_BYTES = BN * BK / 2;
   static constexpr int SFA_BYTES = (BM / 128) * (BK / 64) * 512;
   static constexpr int SFB_BYTES = (BN / 128) * (BK / 64) * 512;
-  static constexpr int U_BYTES = BM * 32 * 4;          // fp32 U tile as loaded (rows of 128 B)
-  static constexpr int UCAT_BYTES = BM * 64 * 2;       // bf16 [hi | lo] of U / alpha (rows of 128 B)
+  static constexpr int UCAT_BYTES = BM * 64 * 2;       // bf16 [hi | lo] of U / g_a (rows of 128 B)
   static constexpr int L2_BYTES = BN * 32 * 2;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kStages * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + kStages * B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + kStages * SFA_BYTES;
-  static constexpr int OFF_U = OFF_SFB + kStages * SFB_BYTES;
-  static constexpr int OFF_UCAT = OFF_U + U_BYTES;
+  static constexpr int OFF_UCAT = OFF_SFB + kStages * SFB_BYTES;
   static constexpr int OFF_L2 = OFF_UCAT + UCAT_BYTES;
   static constexpr int OFF_BAR = OFF_L2 + L2_BYTES;
   static constexpr int NUM_BARS = 2 * kStages + 4;   // full, empty, lr_loaded, lr_ready, acc_full, drain
@@ -66,7 +63,7 @@ struct Cfg {
   static constexpr int TM_USED = BN + 4 * (BK / 64) + 4 * (BN / 128) * (BK / 64);
   static constexpr int TMEM_COLS = TM_USED <= 256 ? 256 : 512;
   static_assert(TM_USED <= 512, "tensor memory overflow");
-  static_assert(OFF_U % 1024 == 0 && OFF_UCAT % 1024 == 0 && OFF_L2 % 1024 == 0, "alignment");
+  static_assert(OFF_UCAT % 1024 == 0 && OFF_L2 % 1024 == 0, "alignment");
 };
 
 struct Params {
@@ -75,7 +72,7 @@ struct Params {
   const __nv_bfloat16* bias;       // [N]
   __nv_bfloat16* Y;                // [M, N]
   int M, N, K;
-  float alpha, inv_alpha;
+  float alpha;
 };
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
@@ -125,7 +122,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
     mbar_init(lr_loaded, 1);
-    mbar_init(lr_ready, 128);
+    mbar_init(lr_ready, 1);                         // unused
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -143,8 +140,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
-      mbar_arrive_expect_tx(lr_loaded, C::U_BYTES + C::L2_BYTES);
-      tma_load_2d(base + C::OFF_U, &tmU, 0, m0, lr_loaded);
+      mbar_arrive_expect_tx(lr_loaded, C::UCAT_BYTES + C::L2_BYTES);
+      tma_load_2d(base + C::OFF_UCAT, &tmU, 0, m0, lr_loaded);
       tma_load_2d(base + C::OFF_L2, &tmL2, 0, n0, lr_loaded);
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % kStages, it = kb / kStages;
@@ -197,7 +194,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         ++done;
       }
       *consumed_out = done;
-      if (done == nkb && mbar_wait_bounded(lr_ready, 0, abort_flag, 3)) {
+      if (done == nkb && mbar_wait_bounded(lr_loaded, 0, abort_flag, 3)) {
         tc_fence_after();
         const uint32_t idb = idesc_bf16<BN>();
 #pragma unroll
@@ -214,33 +211,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;                 // 0..127
-    if (mbar_wait_bounded(lr_loaded, 0, abort_flag, 4)) {
-      // row `et` of the tile: 8 pieces of 16 B, piece j stored at position j ^ (row & 7)
-      const int r = et, sw = r & 7;
-      const uint8_t* urow = gbase + C::OFF_U + r * 128;
-      uint8_t* crow = gbase + C::OFF_UCAT + r * 128;
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {                   // fp32 columns 4j .. 4j+7
-        const float4 a = *reinterpret_cast<const float4*>(urow + ((j ^ sw) << 4));
-        const float4 b = *reinterpret_cast<const float4*>(urow + (((j + 1) ^ sw) << 4));
-        const float v[8] = {a.x * p.inv_alpha, a.y * p.inv_alpha, a.z * p.inv_alpha, a.w * p.inv_alpha,
-                            b.x * p.inv_alpha, b.y * p.inv_alpha, b.z * p.inv_alpha, b.w * p.inv_alpha};
-        uint4 hi, lo;
-        uint32_t* h = reinterpret_cast<uint32_t*>(&hi);
-        uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          h[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
-          l[t] = pack_bf16x2(v[2 * t] - bf16lo_to_f32(h[t]), v[2 * t + 1] - bf16hi_to_f32(h[t]));
-        }
-        // bf16 columns 4j..4j+7 are piece j/2 (hi) and 4 + j/2 (lo) of the 128-byte row
-        *reinterpret_cast<uint4*>(crow + (((j >> 1) ^ sw) << 4)) = hi;
-        *reinterpret_cast<uint4*>(crow + (((4 + (j >> 1)) ^ sw) << 4)) = lo;
-      }
-      fence_proxy_async_smem();
-    }
-    mbar_arrive(lr_ready);
 
     const int quarter = warp & 3;                    // tensor-memory lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;

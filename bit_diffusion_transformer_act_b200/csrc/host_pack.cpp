@@ -72,7 +72,19 @@ double pow2_global_scale(double amax) {
   return g;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+float bf16_to_float(uint16_t b) {
+  const uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+uint16_t float_to_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);   // finite inputs only
+  return static_cast<uint16_t>(u >> 16);
+}
 
 }  // namespace
 
@@ -103,9 +115,9 @@ size_t svdq_act_scale_bytes(int M, int K) {
 }
 
 int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
-                      const uint16_t* bias, int N, int K, int rank,
+                      const uint16_t* bias, const uint16_t* smooth_inv, int N, int K, int rank,
                       void* out, size_t out_bytes, float* w_global_scale) {
-  if (!R || !L1 || !L2 || !out || !w_global_scale) return SVDQ_ERR_INVALID_ARG;
+  if (!R || !L1 || !L2 || !smooth_inv || !out || !w_global_scale) return SVDQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || rank != svdq::kRank)
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
@@ -145,12 +157,22 @@ int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
     }
   }
 
-  uint16_t* l1t = reinterpret_cast<uint16_t*>(blob + L.l1t);
+  // smooth_inv[k] * L1[k][j] is a product of two bf16 values (at most 16 significant
+  // bits, exact in float); it splits exactly into hi = RN_bf16(p) and lo = p - hi.
+  uint16_t* l1s_hi = reinterpret_cast<uint16_t*>(blob + L.l1s);
+  uint16_t* l1s_lo = l1s_hi + static_cast<size_t>(rank) * k;
   for (size_t j = 0; j < static_cast<size_t>(rank); ++j)
-    for (size_t kk = 0; kk < k; ++kk) l1t[j * k + kk] = L1[kk * rank + j];
+    for (size_t kk = 0; kk < k; ++kk) {
+      const float prod = bf16_to_float(smooth_inv[kk]) * bf16_to_float(L1[kk * rank + j]);
+      const uint16_t hi = float_to_bf16_rne(prod);
+      l1s_hi[j * k + kk] = hi;
+      l1s_lo[j * k + kk] = float_to_bf16_rne(prod - bf16_to_float(hi));
+    }
+  // L2 / g_w: g_w is a power of two, so the division only moves the exponent.
   uint16_t* l2t = reinterpret_cast<uint16_t*>(blob + L.l2t);
   for (size_t row = 0; row < n; ++row)
-    for (size_t j = 0; j < static_cast<size_t>(rank); ++j) l2t[row * rank + j] = L2[j * n + row];
+    for (size_t j = 0; j < static_cast<size_t>(rank); ++j)
+      l2t[row * rank + j] = float_to_bf16_rne(static_cast<float>(bf16_to_float(L2[j * n + row]) / g));
   if (bias) std::memcpy(blob + L.bias, bias, n * 2);
 
   svdq::BlobHeader h;

@@ -2,12 +2,13 @@
 //
 // Packed weight blob (device-private; produced on the host by svdq_pack_weights):
 //   [0, 256)     header: "SVDQNVF4", abi version, N, K, rank, g_w
-//   l1t          bf16 [rank][K]   L1 transposed (K contiguous) -- read by the
-//                                 activation kernel, which knows K but not N,
-//                                 so it comes first
+//   l1s          bf16 [2][rank][K] (diag(smooth_inv) L1)^T split exactly into a
+//                                 high and a low bf16 part (K contiguous) -- read
+//                                 by the activation kernel, which knows K but not
+//                                 N, so it comes first
 //   codes        u8   [N][K/2]    E2M1 codes of R, element 2i in the low nibble
 //   scales       u8   swizzled E4M3 block scales of R (128-row x 64-K atoms)
-//   l2t          bf16 [N][rank]   L2 transposed (rank contiguous)
+//   l2t          bf16 [N][rank]   (L2 / g_w) transposed (rank contiguous)
 //   bias         bf16 [N]         zeros when the layer has no bias
 // Every section starts on a 1024-byte boundary.
 #pragma once
@@ -17,12 +18,12 @@
 
 namespace svdq {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int kRank = 32;
 constexpr size_t kBlobAlign = 1024;
 
 struct BlobLayout {
-  size_t l1t, codes, scales, l2t, bias, total;
+  size_t l1s, codes, scales, l2t, bias, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -42,7 +43,7 @@ inline size_t swizzled_scale_offset(size_t row, size_t group, size_t K) {
 inline BlobLayout blob_layout(size_t N, size_t K, size_t rank) {
   BlobLayout L;
   size_t off = kBlobAlign;                      // header, padded
-  L.l1t = off;    off = align_up(off + rank * K * 2, kBlobAlign);
+  L.l1s = off;    off = align_up(off + 2 * rank * K * 2, kBlobAlign);
   L.codes = off;  off = align_up(off + N * K / 2, kBlobAlign);
   L.scales = off; off = align_up(off + swizzled_scale_bytes(N, K), kBlobAlign);
   L.l2t = off;    off = align_up(off + N * rank * 2, kBlobAlign);

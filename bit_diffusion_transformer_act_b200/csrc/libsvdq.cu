@@ -112,25 +112,26 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   k1::Params p;
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.smooth = static_cast<const __nv_bfloat16*>(smooth_inv);
-  p.l1t = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(packed_w) + L.l1t);
+  p.l1s = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(packed_w) + L.l1s);
   p.codes = static_cast<uint8_t*>(act_codes);
   p.scales = static_cast<uint8_t*>(act_scales);
-  p.U = static_cast<float*>(lowrank_act);
+  p.ucat = static_cast<__nv_bfloat16*>(lowrank_act);
   p.M = M;
   p.K = K;
   p.g = act_global_scale;
   p.inv_g = 1.0f / act_global_scale;   // exact: a power of two
 
-  const int rowblocks = 2 * ((M + 127) / 128);         // 64-row CTAs covering the scale padding
+  const int rowblocks = (M + 127) / 128;               // 128-row CTAs covering the scale padding
   const int kgroups = K / 64;
-  // K slices per row block (a cluster): the largest of 8, 4, 2, 1 that keeps slices whole
-  // (multiples of 64) and the grid within about four CTAs per SM
-  int ks = 1;
-  for (int c : {8, 4, 2, 1}) {
-    if (kgroups % c != 0) continue;
-    ks = c;
-    if (rowblocks * c <= 4 * 148) break;
+  // K slices per row block (one cluster): the fewest of 1, 2, 4, 8 that keep every slice
+  // whole (a multiple of 64) and within the kernel's smoothing buffer, then more while
+  // the grid has fewer CTAs than two per SM
+  int ks = 0;
+  for (int c : {1, 2, 4, 8}) {
+    if (kgroups % c == 0 && K / c <= k1::kMaxSlice) { ks = c; break; }
   }
+  if (ks == 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  while (ks < 8 && kgroups % (2 * ks) == 0 && rowblocks * ks < 2 * 148) ks *= 2;
   p.kslices = ks;
 
   const int smem = static_cast<int>(sizeof(k1::Smem));
@@ -183,7 +184,6 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   p.N = N;
   p.K = K;
   p.alpha = static_cast<float>(alpha);
-  p.inv_alpha = static_cast<float>(1.0 / alpha);
 
   const bool wide = (N % 256 == 0);
   const int BN = wide ? 256 : 128;
@@ -192,7 +192,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, BN,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, rank, rank, k2::BM,
+      !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, 2 * rank, 2 * rank, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN,
                  CU_TENSOR_MAP_SWIZZLE_64B))

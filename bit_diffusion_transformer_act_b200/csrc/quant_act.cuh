@@ -5,28 +5,34 @@
 // nvfp4 / group 16; the Nunchaku Lite article: outliers go to a 16-bit
 // low-rank branch): X_hat = X * smooth_inv; per 16 K elements one E4M3 scale
 // S = RNE(amax / (6 g_a)) and E2M1 codes RNE(clamp(X_hat / (S g_a))); and
-// U = X_hat L1 (rank 32, fp32) from the same smoothed values.
+// U = X_hat L1 (rank 32) from the same smoothed activations.
 //
-// Design (sm_100a).  A CTA owns 64 rows and one K slice; the K slices of a row
-// block form a thread-block cluster (1..8 CTAs) so the grid fills the 148 SMs
-// even for a few thousand rows, and the partial U of the slices is summed over
-// distributed shared memory -- no global scratch, no atomics.  X and L1 chunks
-// of 128 columns are double-buffered in shared memory with cp.async (rows past
-// M are zero-filled), the four warps each read their 16 x 16 tiles with
-// ldmatrix straight into the mma.sync A-fragment layout, and all the per-element
-// work happens on those registers: smoothing in fp32 (the product of two bf16
-// values is exact), the group amax with two xor-shuffles inside each lane
-// quad, the scale, the codes and the bf16 A operand of the low-rank mma.
+// Design (sm_100a).  A CTA (8 warps) owns 128 rows and one K slice; the K
+// slices of a row block form a thread-block cluster (1..8 CTAs) so the grid
+// fills the 148 SMs, and the partial U of the slices is summed over
+// distributed shared memory -- no global scratch, no atomics.  X and the L1
+// operand arrive in 128-column chunks, double-buffered in shared memory with
+// cp.async (rows past M zero-filled) and XOR-swizzled against bank conflicts.
+//   * Quantization: each thread owns one row and 64 consecutive columns (four
+//     16-element groups, i.e. one 32-bit word of the scale layout and 32
+//     contiguous code bytes, stored directly).
+//   * Low-rank: X_hat L1 = X (diag(smooth_inv) L1); the packed weights hold
+//     diag(smooth_inv) L1 split exactly into bf16 hi + lo, so ldmatrix feeds
+//     the raw bf16 X tile to mma.sync twice (hi, lo) with fp32 accumulation:
+//     every product is exact.  The result U / g_a is written split into bf16
+//     hi + lo, the operand layout of the GEMM's low-rank MMA.
 //
-// Rounding: the scale uses a correctly rounded quotient amax/6 (x 1/g_a, a
-// power of two), converted with cvt.rn.satfinite.e4m3x2.  Codes use
-// q = x_hat / (S g_a) correctly rounded by one Markstein correction step
-// (q0 = x r, e = fma(-q0, D, x), q = fma(e, r, q0) with r = RN(1/D)), then
-// cvt.rn.satfinite.e2m1x2.  A quotient that is not exactly a rounding
-// midpoint sits 2^-16 (relative) or more away from one, far above fp32
-// rounding, and an exact midpoint comes out exact, so the codes equal those of
-// exact arithmetic.  The sign of q is copied from x_hat (negative zero stays
-// negative).
+// Rounding.  amax/6 is formed by a Markstein-corrected multiplication by the
+// rounded reciprocal of 6 (P. Markstein's correction: with y = RN(1/b) and
+// q0 = RN(a y), q0 + RN(a - b q0) y rounds to RN(a/b)), then scaled by 1/g_a
+// (a power of two) and converted with cvt.rn.satfinite.e4m3x2.  A code
+// quotient x_hat / (S g_a) is q0 = x_hat * r with r = rcp.approx(S g_a)
+// followed by the same correction step; because x_hat has at most 16
+// significant bits and the E2M1 midpoints times S g_a at most 7, a quotient is
+// either exactly a midpoint -- and then the corrected value is that midpoint
+// exactly -- or at least 2^-16 (relative) away from one, far beyond the
+// few-ulp error of q.  cvt.rn.satfinite.e2m1x2 then rounds to nearest even.
+// The sign of q is copied from x_hat so that negative zero keeps its sign.
 #pragma once
 
 #include "ptx.cuh"
@@ -34,20 +40,21 @@
 namespace svdq {
 namespace k1 {
 
-constexpr int kRows = 64;                 // rows per CTA
-constexpr int kWarps = 4;                 // 16 rows each
+constexpr int kRows = 128;                // rows per CTA
+constexpr int kWarps = 8;                 // 16 rows each for the low-rank MMA
 constexpr int kThreads = kWarps * 32;
 constexpr int kChunk = 128;               // K columns per pipeline chunk
 constexpr int kRank = 32;
-constexpr int kCodeStride = 80;          // bytes per staged code row (64 used; 80 spreads banks)
+constexpr int kMaxSlice = 2048;           // longest K slice (columns) held as fp32 smoothing factors
 
 struct __align__(128) Smem {
   __nv_bfloat16 x[2][kRows * kChunk];     // rows of 256 B, 16-B pieces XOR-swizzled by (row & 7)
-  __nv_bfloat16 l1[2][kRank * kChunk];    // L1^T chunk, same swizzle
-  __nv_bfloat16 smooth[2][kChunk];
-  uint8_t codes[kWarps][16 * kCodeStride];
-  float upart[kRows * kRank];             // this CTA's partial U (fp32)
+  __nv_bfloat16 lh[2][kRank * kChunk];    // (diag(s) L1)^T high part, same swizzle
+  __nv_bfloat16 ll[2][kRank * kChunk];    // low part
+  float smooth[kMaxSlice];                // this CTA's slice of smooth_inv, as floats
 };
+// The partial U of the CTA (128 x 32 fp32) reuses the X buffers once the K loop is done.
+static_assert(sizeof(__nv_bfloat16) * 2 * kRows * kChunk >= sizeof(float) * kRows * kRank, "upart alias");
 
 // Byte offset of element (row, col) in a swizzled [rows][128] bf16 chunk.
 __device__ __forceinline__ uint32_t swz(int row, int col) {
@@ -57,10 +64,10 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 struct Params {
   const __nv_bfloat16* X;          // [M, K]
   const __nv_bfloat16* smooth;     // [K]
-  const __nv_bfloat16* l1t;        // [32, K]
+  const __nv_bfloat16* l1s;        // [2][32][K]: (diag(smooth) L1)^T hi, then lo
   uint8_t* codes;                  // [M, K/2]
-  uint8_t* scales;                 // swizzled
-  float* U;                        // [M, 32]
+  uint8_t* scales;                 // swizzled, rows padded to 128
+  __nv_bfloat16* ucat;             // [M, 64]: U / g_a as bf16 hi (0..31) and lo (32..63)
   int M, K;
   int kslices;                     // cluster size along K
   float g;                         // per-tensor scale (power of two)
@@ -78,27 +85,23 @@ __device__ __forceinline__ void load_chunk(Smem& s, int buf, const Params& p, in
     const __nv_bfloat16* src = p.X + (ok ? (static_cast<size_t>(m) * p.K + kc + c) : 0);
     cp_async_16(xbase + swz(r, c), src, ok ? 16u : 0u);
   }
-  const uint32_t lbase = smem_addr(s.l1[buf]);
+  const uint32_t hbase = smem_addr(s.lh[buf]), lbase = smem_addr(s.ll[buf]);
+  const __nv_bfloat16* lo_src = p.l1s + static_cast<size_t>(kRank) * p.K;
   for (int i = tid; i < kRank * pieces; i += kThreads) {
     const int r = i / pieces, c = (i % pieces) * 8;
-    cp_async_16(lbase + swz(r, c), p.l1t + static_cast<size_t>(r) * p.K + kc + c, 16u);
+    cp_async_16(hbase + swz(r, c), p.l1s + static_cast<size_t>(r) * p.K + kc + c, 16u);
+    cp_async_16(lbase + swz(r, c), lo_src + static_cast<size_t>(r) * p.K + kc + c, 16u);
   }
-  if (tid < pieces) cp_async_16(smem_addr(&s.smooth[buf][tid * 8]), p.smooth + kc + tid * 8, 16u);
   cp_async_commit();
 }
 
-// Scale code for one group given its amax (fp32).
-__device__ __forceinline__ float group_scale_arg(float amax, float inv_g) {
-  return __fdiv_rn(amax, 6.0f) * inv_g;
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
-// a = hi + lo exactly for each of the two values (hi = RN_bf16(a), lo = RN_bf16(a - hi), and
-// a - hi fits in bf16 whenever a has at most 16 significant bits).
-__device__ __forceinline__ void split_bf16x2(float a0, float a1, uint32_t& hi, uint32_t& lo) {
-  hi = pack_bf16x2(a0, a1);
-  lo = pack_bf16x2(a0 - bf16lo_to_f32(hi), a1 - bf16hi_to_f32(hi));
-}
-
+// Quotient x / D for the E2M1 decision (see the rounding note above); r ~ 1/D.
 __device__ __forceinline__ float quotient(float x, float D, float r) {
   const float q0 = x * r;
   const float e = fmaf(-q0, D, x);
@@ -106,19 +109,51 @@ __device__ __forceinline__ float quotient(float x, float D, float r) {
   return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
 }
 
-__global__ void __launch_bounds__(kThreads)
+// RN(a / 6) for a >= 0 (Markstein correction of a * RN(1/6)).
+__device__ __forceinline__ float div6(float a) {
+  const float y = 0.16666667163372039794921875f;      // RN(1/6) in binary32
+  const float q0 = a * y;
+  const float e = fmaf(-q0, 6.0f, a);
+  return fmaf(e, y, q0);
+}
+
+// Quantizes 16 smoothed values (one group): returns the E4M3 scale code, writes 8 code bytes.
+__device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], const Params& p, uint2& out) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sc = cvt_e4m3x2(div6(amax) * p.inv_g, 0.f) & 0xFFu;
+  float S, unused;
+  e4m3x2_to_f32(sc, S, unused);
+  const float D = S * p.g;
+  if (D == 0.f) {
+    out = make_uint2(0u, 0u);
+    return 0u;
+  }
+  const float r = rcp_approx(D);
+  out.x = cvt_e2m1x8(quotient(v[0], D, r), quotient(v[1], D, r), quotient(v[2], D, r), quotient(v[3], D, r),
+                     quotient(v[4], D, r), quotient(v[5], D, r), quotient(v[6], D, r), quotient(v[7], D, r));
+  out.y = cvt_e2m1x8(quotient(v[8], D, r), quotient(v[9], D, r), quotient(v[10], D, r), quotient(v[11], D, r),
+                     quotient(v[12], D, r), quotient(v[13], D, r), quotient(v[14], D, r), quotient(v[15], D, r));
+  return sc;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 quant_act_lowrank_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
 
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  const int g = lane / 4, q = lane % 4;
+  const int tid = threadIdx.x;
+  const int warp = tid / 32;
+  const int lane = tid % 32;
   const int m0 = blockIdx.x * kRows;
   const int slice = blockIdx.y;
   const int klen = p.K / p.kslices;
   const int kbeg = slice * klen;
   const int nchunks = (klen + kChunk - 1) / kChunk;
+
+  load_chunk(s, 0, p, m0, kbeg, min(kChunk, klen));
+  for (int i = tid; i < klen; i += kThreads) s.smooth[i] = __bfloat162float(p.smooth[kbeg + i]);
 
   float acc[4][4];
 #pragma unroll
@@ -126,7 +161,9 @@ quant_act_lowrank_kernel(const Params p) {
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[j][t] = 0.f;
 
-  load_chunk(s, 0, p, m0, kbeg, min(kChunk, klen));
+  // quantization role of this thread: row qr, columns [64 qh, 64 qh + 64) of each chunk
+  const int qr = tid >> 1, qh = tid & 1;
+  const int qm = m0 + qr;
 
   for (int ci = 0; ci < nchunks; ++ci) {
     const int buf = ci & 1;
@@ -141,120 +178,84 @@ quant_act_lowrank_kernel(const Params p) {
     }
     __syncthreads();
 
-    const uint32_t xbase = smem_addr(s.x[buf]);
-    const uint32_t lbase = smem_addr(s.l1[buf]);
-    const uint32_t* sm32 = reinterpret_cast<const uint32_t*>(s.smooth[buf]);
-    uint8_t* cst = s.codes[warp];
-    uint32_t sc_g = 0, sc_h = 0;                     // scale bytes of rows g and g+8 for the current 64-K atom
+    const uint8_t* xs = reinterpret_cast<const uint8_t*>(s.x[buf]);
 
-    const int steps = ncols / 16;
-    for (int st = 0; st < steps; ++st) {
-      // A fragment: rows 16w + {g, g+8}, columns 16 st + {2q, 2q+1, 2q+8, 2q+9}
-      uint32_t a0, a1, a2, a3;
-      {
-        const int mi = lane >> 3;
-        const int row = warp * 16 + (lane & 7) + ((mi & 1) << 3);
-        const int col = st * 16 + ((mi >> 1) << 3);
-        ldmatrix_x4(xbase + swz(row, col), a0, a1, a2, a3);
-      }
-      const uint32_t sp0 = sm32[(st * 16 + 2 * q) >> 1];
-      const uint32_t sp1 = sm32[(st * 16 + 8 + 2 * q) >> 1];
-      const float s0 = bf16lo_to_f32(sp0), s1 = bf16hi_to_f32(sp0);
-      const float s8 = bf16lo_to_f32(sp1), s9 = bf16hi_to_f32(sp1);
-      // row g: a0 (k 2q, 2q+1), a2 (k 2q+8, 2q+9); row g+8: a1, a3
-      const float x0 = bf16lo_to_f32(a0) * s0, x1 = bf16hi_to_f32(a0) * s1;
-      const float x2 = bf16lo_to_f32(a2) * s8, x3 = bf16hi_to_f32(a2) * s9;
-      const float y0 = bf16lo_to_f32(a1) * s0, y1 = bf16hi_to_f32(a1) * s1;
-      const float y2 = bf16lo_to_f32(a3) * s8, y3 = bf16hi_to_f32(a3) * s9;
-
-      float mx = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
-      float my = fmaxf(fmaxf(fabsf(y0), fabsf(y1)), fmaxf(fabsf(y2), fabsf(y3)));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-      my = fmaxf(my, __shfl_xor_sync(0xFFFFFFFFu, my, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-      my = fmaxf(my, __shfl_xor_sync(0xFFFFFFFFu, my, 2));
-
-      const uint32_t sc2 = cvt_e4m3x2(group_scale_arg(mx, p.inv_g), group_scale_arg(my, p.inv_g));
-      float Sx, Sy;
-      e4m3x2_to_f32(sc2, Sx, Sy);
-      const float Dx = Sx * p.g, Dy = Sy * p.g;
-      const float rx = Dx > 0.f ? __frcp_rn(Dx) : 0.f;
-      const float ry = Dy > 0.f ? __frcp_rn(Dy) : 0.f;
-
-      uint32_t cw = cvt_e2m1x8(quotient(x0, Dx, rx), quotient(x1, Dx, rx), quotient(x2, Dx, rx),
-                               quotient(x3, Dx, rx), quotient(y0, Dy, ry), quotient(y1, Dy, ry),
-                               quotient(y2, Dy, ry), quotient(y3, Dy, ry));
-      if (Dx == 0.f) cw &= 0xFFFF0000u;
-      if (Dy == 0.f) cw &= 0x0000FFFFu;
-      // byte 0: row g, elements 2q..2q+1 -> code byte 8 st + q; byte 1: elements 2q+8.. -> 8 st + 4 + q
-      cst[g * kCodeStride + st * 8 + q] = static_cast<uint8_t>(cw);
-      cst[g * kCodeStride + st * 8 + 4 + q] = static_cast<uint8_t>(cw >> 8);
-      cst[(g + 8) * kCodeStride + st * 8 + q] = static_cast<uint8_t>(cw >> 16);
-      cst[(g + 8) * kCodeStride + st * 8 + 4 + q] = static_cast<uint8_t>(cw >> 24);
-
-      const int sh = 8 * (st & 3);
-      sc_g |= (sc2 & 0xFFu) << sh;
-      sc_h |= ((sc2 >> 8) & 0xFFu) << sh;
-      if ((st & 3) == 3) {
-        const int atom = (kc + st * 16) / 64;        // 64-K atom index
-        if (q < 2) {
-          const int r = warp * 16 + g + 8 * q;       // lane q=0 stores row g, q=1 row g+8
-          const int m = m0 + r;
-          const size_t off = (static_cast<size_t>(m / 128) * (p.K / 64) + atom) * 512 +
-                             (m % 32) * 16 + ((m % 128) / 32) * 4;
-          *reinterpret_cast<uint32_t*>(p.scales + off) = q == 0 ? sc_g : sc_h;
-        }
-        sc_g = 0; sc_h = 0;
-      }
-
-      // low-rank down projection on the smoothed values.  X_hat (at most 16 significant
-      // bits) is split exactly into bf16 hi + lo, so two bf16 MMAs with fp32
-      // accumulation give X_hat L1 without rounding the operand.
-      uint32_t H0, H1, H2, H3, L0, L1, L2, L3;
-      split_bf16x2(x0, x1, H0, L0);
-      split_bf16x2(y0, y1, H1, L1);
-      split_bf16x2(x2, x3, H2, L2);
-      split_bf16x2(y2, y3, H3, L3);
+    // ---------------------------------------------------------------- quantization
+    if (qh * 64 < ncols) {
+      const float* sm = s.smooth + (kc - kbeg) + qh * 64;
+      uint32_t scw = 0;
+      uint2 cb[4];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t b00, b01, b10, b11;
-        const int mi = lane >> 3;
-        const int n = half * 16 + ((mi >> 1) << 3) + (lane & 7);
-        const int col = st * 16 + ((mi & 1) << 3);
-        ldmatrix_x4(lbase + swz(n, col), b00, b01, b10, b11);
-        mma_bf16_16816(acc[half * 2 + 0], H0, H1, H2, H3, b00, b01);
-        mma_bf16_16816(acc[half * 2 + 1], H0, H1, H2, H3, b10, b11);
-        mma_bf16_16816(acc[half * 2 + 0], L0, L1, L2, L3, b00, b01);
-        mma_bf16_16816(acc[half * 2 + 1], L0, L1, L2, L3, b10, b11);
+      for (int gq = 0; gq < 4; ++gq) {
+        float v[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col = qh * 64 + gq * 16 + h * 8;
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + swz(qr, col));
+          const float4 s0 = *reinterpret_cast<const float4*>(sm + gq * 16 + h * 8);
+          const float4 s1 = *reinterpret_cast<const float4*>(sm + gq * 16 + h * 8 + 4);
+          v[h * 8 + 0] = bf16lo_to_f32(xv.x) * s0.x;
+          v[h * 8 + 1] = bf16hi_to_f32(xv.x) * s0.y;
+          v[h * 8 + 2] = bf16lo_to_f32(xv.y) * s0.z;
+          v[h * 8 + 3] = bf16hi_to_f32(xv.y) * s0.w;
+          v[h * 8 + 4] = bf16lo_to_f32(xv.z) * s1.x;
+          v[h * 8 + 5] = bf16hi_to_f32(xv.z) * s1.y;
+          v[h * 8 + 6] = bf16lo_to_f32(xv.w) * s1.z;
+          v[h * 8 + 7] = bf16hi_to_f32(xv.w) * s1.w;
+        }
+        scw |= quantize_group(v, p, cb[gq]) << (8 * gq);
+      }
+      const int atom = (kc + qh * 64) / 64;
+      const size_t soff = (static_cast<size_t>(qm / 128) * (p.K / 64) + atom) * 512 + (qm % 32) * 16 +
+                          ((qm % 128) / 32) * 4;
+      *reinterpret_cast<uint32_t*>(p.scales + soff) = scw;      // rows past M get zero scales
+      if (qm < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(qm) * (p.K / 2) + (kc + qh * 64) / 2);
+        dst[0] = make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y);
+        dst[1] = make_uint4(cb[2].x, cb[2].y, cb[3].x, cb[3].y);
       }
     }
 
-    // codes of this warp's 16 rows for the chunk -> global, 16 bytes per store
-    __syncwarp();
+    // ---------------------------------------------------------------- low-rank down projection
     {
-      const int rowbytes = ncols / 2;
-      const int per_row = rowbytes / 16;
-      for (int i = lane; i < 16 * per_row; i += 32) {
-        const int r = i / per_row, seg = i % per_row;
-        const int m = m0 + warp * 16 + r;
-        if (m < p.M) {
-          const uint4 v = *reinterpret_cast<const uint4*>(cst + r * kCodeStride + seg * 16);
-          *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc / 2 + seg * 16) = v;
+      const uint32_t xbase = smem_addr(s.x[buf]);
+      const uint32_t hbase = smem_addr(s.lh[buf]), lbase = smem_addr(s.ll[buf]);
+      const int mi = lane >> 3;
+      const int steps = ncols / 16;
+      for (int st = 0; st < steps; ++st) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(xbase + swz(warp * 16 + (lane & 7) + ((mi & 1) << 3), st * 16 + ((mi >> 1) << 3)),
+                    a0, a1, a2, a3);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int n = half * 16 + ((mi >> 1) << 3) + (lane & 7);
+          const int col = st * 16 + ((mi & 1) << 3);
+          uint32_t h00, h01, h10, h11, l00, l01, l10, l11;
+          ldmatrix_x4(hbase + swz(n, col), h00, h01, h10, h11);
+          ldmatrix_x4(lbase + swz(n, col), l00, l01, l10, l11);
+          mma_bf16_16816(acc[half * 2 + 0], a0, a1, a2, a3, h00, h01);
+          mma_bf16_16816(acc[half * 2 + 1], a0, a1, a2, a3, h10, h11);
+          mma_bf16_16816(acc[half * 2 + 0], a0, a1, a2, a3, l00, l01);
+          mma_bf16_16816(acc[half * 2 + 1], a0, a1, a2, a3, l10, l11);
         }
       }
     }
-    __syncthreads();          // buffer `buf` and the code staging are free again
+    __syncthreads();          // buffer `buf` is free again
   }
 
-  // partial U of this slice -> shared memory
+  // partial U of this slice -> shared memory (reusing the X buffers)
+  float* upart = reinterpret_cast<float*>(s.x[0]);
+  {
+    const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int col = 8 * j + 2 * q;
-    const int r0 = warp * 16 + g;
-    s.upart[r0 * kRank + col] = acc[j][0];
-    s.upart[r0 * kRank + col + 1] = acc[j][1];
-    s.upart[(r0 + 8) * kRank + col] = acc[j][2];
-    s.upart[(r0 + 8) * kRank + col + 1] = acc[j][3];
+    for (int j = 0; j < 4; ++j) {
+      const int col = 8 * j + 2 * q;
+      const int r0 = warp * 16 + g;
+      upart[r0 * kRank + col] = acc[j][0];
+      upart[r0 * kRank + col + 1] = acc[j][1];
+      upart[(r0 + 8) * kRank + col] = acc[j][2];
+      upart[(r0 + 8) * kRank + col + 1] = acc[j][3];
+    }
   }
 
   // sum the slices' partials across the cluster; CTA `rank` finishes rows [rank*rpc, (rank+1)*rpc)
@@ -262,17 +263,23 @@ quant_act_lowrank_kernel(const Params p) {
   if (ks > 1) cluster_sync_all(); else __syncthreads();
   const uint32_t rank = ks > 1 ? cluster_ctarank() : 0u;
   const int rpc = kRows / ks;
-  for (int i = threadIdx.x; i < rpc * kRank; i += kThreads) {
+  for (int i = tid; i < rpc * kRank; i += kThreads) {
     const int r = static_cast<int>(rank) * rpc + i / kRank;
     const int c = i % kRank;
     float sum = 0.f;
     if (ks > 1) {
-      for (int src = 0; src < ks; ++src) sum += ld_dsmem_f32(&s.upart[r * kRank + c], static_cast<uint32_t>(src));
+      for (int src = 0; src < ks; ++src) sum += ld_dsmem_f32(&upart[r * kRank + c], static_cast<uint32_t>(src));
     } else {
-      sum = s.upart[r * kRank + c];
+      sum = upart[r * kRank + c];
     }
     const int m = m0 + r;
-    if (m < p.M) p.U[static_cast<size_t>(m) * kRank + c] = sum;
+    if (m < p.M) {
+      const float u = sum * p.inv_g;                   // exact: a power of two
+      const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
+      p.ucat[static_cast<size_t>(m) * (2 * kRank) + c] = hi;
+      p.ucat[static_cast<size_t>(m) * (2 * kRank) + kRank + c] = lo;
+    }
   }
   if (ks > 1) cluster_sync_all();   // keep this CTA's shared memory alive until the others have read it
 }

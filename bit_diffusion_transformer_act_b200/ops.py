@@ -35,7 +35,7 @@ def _load():
         "svdq_status_string": ([i], ctypes.c_char_p),
         "svdq_abi_version": ([], i),
         "svdq_packed_weight_bytes": ([i, i, i], sz),
-        "svdq_pack_weights": ([vp, vp, vp, vp, i, i, i, vp, sz, ctypes.POINTER(ctypes.c_float)], i),
+        "svdq_pack_weights": ([vp, vp, vp, vp, vp, i, i, i, vp, sz, ctypes.POINTER(ctypes.c_float)], i),
         "svdq_act_scale_bytes": ([i, i], sz),
         "svdq_quantize_act_lowrank_down": ([vp, vp, vp, i, i, i, f, vp, vp, vp, vp], i),
         "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
@@ -92,8 +92,9 @@ def svdq_act_scale_bytes(M, K):
     return int(LIB.svdq_act_scale_bytes(M, K))
 
 
-def svdq_pack_weights(R, L1_bits, L2_bits, bias_bits=None):
-    """R float32 [N, K]; L1 bf16 bits uint16 [K, r]; L2 bits [r, N]; bias bits [N] or None.
+def svdq_pack_weights(R, L1_bits, L2_bits, bias_bits, smooth_bits):
+    """R float32 [N, K]; L1 bf16 bits uint16 [K, r]; L2 bits [r, N]; bias bits [N] or None;
+    smooth_inv bits [K] (the same vector later given to the activation kernel).
 
     Returns (blob uint8 numpy array, w_global_scale float)."""
     R = np.ascontiguousarray(R, dtype=np.float32)
@@ -107,13 +108,16 @@ def svdq_pack_weights(R, L1_bits, L2_bits, bias_bits=None):
         bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
         if bias_bits.shape != (N,):
             raise ValueError("bias must be [N]")
+    smooth_bits = np.ascontiguousarray(smooth_bits, dtype=np.uint16)
+    if smooth_bits.shape != (K,):
+        raise ValueError("smooth_inv must be [K]")
     nbytes = svdq_packed_weight_bytes(N, K, rank)
     if nbytes == 0:
         _check("svdq_pack_weights", 2)
     out = np.empty(nbytes, dtype=np.uint8)
     g = ctypes.c_float(0.0)
     st = LIB.svdq_pack_weights(_np_ptr(R), _np_ptr(L1_bits), _np_ptr(L2_bits), _np_ptr(bias_bits),
-                               N, K, rank, _np_ptr(out), nbytes, ctypes.byref(g))
+                               _np_ptr(smooth_bits), N, K, rank, _np_ptr(out), nbytes, ctypes.byref(g))
     _check("svdq_pack_weights", st)
     return out, float(g.value)
 
@@ -146,7 +150,8 @@ def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, ra
                                    act_codes=None, act_scales=None, lowrank_act=None):
     """X bf16 [M, K] cuda; smooth_inv bf16 [K]; packed_w uint8 cuda (the blob).
 
-    Returns (act_codes uint8 [M, K/2], act_scales uint8 [svdq_act_scale_bytes], lowrank_act float32 [M, r])."""
+    Returns (act_codes uint8 [M, K/2], act_scales uint8 [svdq_act_scale_bytes],
+    lowrank_act bf16 [M, 2r] holding U / g_a as a high part then a low part)."""
     M, K = X.shape
     dev = X.device
     _require(X, torch.bfloat16, (M, K), "X")
@@ -156,10 +161,10 @@ def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, ra
     if act_scales is None:
         act_scales = torch.empty((svdq_act_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
     if lowrank_act is None:
-        lowrank_act = torch.empty((M, rank), dtype=torch.float32, device=dev)
+        lowrank_act = torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev)
     _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
     _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
-    _require(lowrank_act, torch.float32, (M, rank), "lowrank_act")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
     st = LIB.svdq_quantize_act_lowrank_down(_ptr(X), _ptr(smooth_inv), _ptr(packed_w), M, K, rank,
                                             float(act_global_scale), _ptr(act_codes), _ptr(act_scales),
                                             _ptr(lowrank_act), _stream())
@@ -209,7 +214,7 @@ class SvdqW4A4Linear:
     (bf16 bits) and the static activation scale g_a (a power of two)."""
 
     def __init__(self, R, L1_bits, L2_bits, bias_bits, smooth_inv_bits, act_global_scale, device="cuda"):
-        blob, g_w = svdq_pack_weights(R, L1_bits, L2_bits, bias_bits)
+        blob, g_w = svdq_pack_weights(R, L1_bits, L2_bits, bias_bits, smooth_inv_bits)
         self.N, self.K = R.shape
         self.rank = L1_bits.shape[1]
         self.packed = torch.from_numpy(blob).to(device)

@@ -87,20 +87,24 @@ size_t svdq_packed_weight_bytes(int N, int K, int rank);
  *   L1    bf16   [K, rank] low-rank down factor (math orientation).
  *   L2    bf16   [rank, N] low-rank up factor.
  *   bias  bf16   [N] or NULL (then the bias is zero).
+ *   smooth_inv bf16 [K]    the layer's 1/lambda; the same vector must be passed
+ *                          to svdq_quantize_act_lowrank_down.
  *   N % 128 == 0, K % 64 == 0, N, K > 0, rank == 32.
  *   out   host buffer of out_bytes >= svdq_packed_weight_bytes(N, K, rank).
  *   w_global_scale  receives g_w = 2^ceil(log2(amax(R) / 2688)) (1 if R == 0).
  * The blob is device-private: copy it to the GPU as it is and pass that copy
- * as `packed_w`.  It holds: a 256-byte header ("SVDQNVF4", N, K, rank, g_w),
- * the NVFP4 codes of R [N, K/2], their swizzled E4M3 scales, L1 transposed to
- * [rank, K], L2 transposed to [N, rank] and the bias [N] (bf16), each section
- * aligned to 1024 bytes.  Codes and scales are bit-exact to the definition
- * above (RNE on exact quotients).
+ * as `packed_w`.  It holds: a 1 KB header ("SVDQNVF4", N, K, rank, g_w);
+ * (diag(smooth_inv) L1)^T [rank, K] split exactly into a high and a low bf16
+ * part (each product of two bf16 values has at most 16 significant bits); the
+ * NVFP4 codes of R [N, K/2] and their swizzled E4M3 scales; (L2 / g_w)
+ * transposed to [N, rank] (exact: g_w is a power of two); the bias [N] (bf16).
+ * Sections are aligned to 1024 bytes.  Codes and scales are bit-exact to the
+ * definition above (RNE on exact quotients).
  * Returns SVDQ_ERR_INVALID_ARG for null pointers or a short buffer, and
  * SVDQ_ERR_UNSUPPORTED_SHAPE for dimensions outside the rules above, or when R
  * holds a NaN or infinity. */
 int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
-                      const uint16_t* bias, int N, int K, int rank,
+                      const uint16_t* bias, const uint16_t* smooth_inv, int N, int K, int rank,
                       void* out, size_t out_bytes, float* w_global_scale);
 
 /* ------------------------------------------------------------- activations */
@@ -119,9 +123,11 @@ size_t svdq_act_scale_bytes(int M, int K);
  *   act_global_scale  g_a > 0, a power of two (static calibration)
  *   act_codes   device u8 [M, K/2] out: E2M1 codes of X_hat
  *   act_scales  device u8 [svdq_act_scale_bytes(M, K)] out: swizzled E4M3 scales
- *   lowrank_act device float32 [M, rank] out: X_hat L1.  X_hat is split
- *               exactly into two bf16 parts for the tensor cores, so the only
- *               rounding is the fp32 accumulation.
+ *   lowrank_act device bf16 [M, 2*rank] out: U / g_a with U = X_hat L1,
+ *               stored as a high part (columns 0..rank-1) and a low part
+ *               (columns rank..2*rank-1), U = g_a (hi + lo) to 2^-16 relative.
+ *               The product is formed exactly (X times the packed exact split
+ *               of diag(smooth_inv) L1) and accumulated in fp32.
  * K % 64 == 0, rank == 32, M >= 0.  Asynchronous on `stream`. */
 int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv,
                                    const void* packed_w, int M, int K, int rank,
@@ -131,8 +137,8 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv,
 /* Kernel 2: the NVFP4 block-scaled GEMM on tcgen05 with the low-rank up
  * projection, the bias and the bf16 cast fused in the epilogue:
  *   Y = bf16( g_a g_w (Q(X_hat) Q(R)^T) + lowrank_act L2 + b ).
- * The fp32 lowrank_act is split exactly into two bf16 parts for the tensor
- * cores; all products are exact and accumulate in fp32.
+ * The low-rank term is (hi + lo)(L2 / g_w) accumulated with the FP4 products
+ * in one fp32 accumulator and scaled by g_a g_w once, in the epilogue.
  *   act_codes, act_scales, lowrank_act  outputs of kernel 1 for the same M, K
  *   act_global_scale  the g_a given to kernel 1 (power of two)
  *   packed_w          device copy of the blob; w_global_scale its g_w

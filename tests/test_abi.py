@@ -47,7 +47,7 @@ def test_status_strings_and_version():
     for s in range(6):
         assert P.LIB.svdq_status_string(s)
     assert P.LIB.svdq_status_string(99) == b"unknown status"
-    assert P.LIB.svdq_abi_version() == 1
+    assert P.LIB.svdq_abi_version() == 2
 
 
 def test_sizes():

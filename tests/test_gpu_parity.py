@@ -24,7 +24,7 @@ def _bf16_dev(a):
 
 def _pack(P, w, with_bias=True):
     blob, gw = P.svdq_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2),
-                                   synth.bf16_bits(w.bias) if with_bias else None)
+                                   synth.bf16_bits(w.bias) if with_bias else None, synth.bf16_bits(w.smooth_inv))
     return torch.from_numpy(blob).cuda(), gw
 
 
@@ -34,7 +34,10 @@ def _run_svdq(P, X, smooth, packed, g_a, g_w, N):
     codes, scales, U = P.svdq_quantize_act_lowrank_down(Xd, sd, packed, g_a)
     Y = P.svdq_w4a4_nvfp4_linear(codes, scales, U, g_a, packed, g_w, M, N, K)
     torch.cuda.synchronize()
-    return codes.cpu().numpy(), scales.cpu().numpy(), U.cpu().numpy(), Y.float().cpu().numpy()
+    # the low-rank activations come back as bf16 hi and lo parts of U / g_a
+    Uc = U.float().cpu().numpy().astype(np.float64)
+    U_full = g_a * (Uc[:, :32] + Uc[:, 32:])
+    return codes.cpu().numpy(), scales.cpu().numpy(), U_full, Y.float().cpu().numpy()
 
 
 def _check_act(codes, scales, U, X, smooth, L1, g_a):
@@ -47,7 +50,8 @@ def _check_act(codes, scales, U, X, smooth, L1, g_a):
     assert np.all(sg[M:] == 0)
     Xh = svdq.smooth(X, smooth)
     U_ref = Xh @ L1.astype(np.float64)
-    bound = 1e-5 * (np.abs(Xh) @ np.abs(L1.astype(np.float64))) + 1e-30
+    # fp32 accumulation over K plus the bf16 hi/lo representation (2^-16 relative)
+    bound = 1e-5 * (np.abs(Xh) @ np.abs(L1.astype(np.float64))) + 2.0 ** -15 * np.abs(U_ref) + 1e-30
     assert np.all(np.abs(U - U_ref) <= bound), np.max(np.abs(U - U_ref) / bound)
 
 
@@ -106,7 +110,8 @@ def test_edge_shapes_and_values(P, M, K, N):
     L1 = synth.to_bf16(rng.standard_normal((K, 32)) * 0.1)
     L2 = synth.to_bf16(rng.standard_normal((32, N)) * 0.1)
     b = synth.to_bf16(rng.standard_normal(N) * 0.01)
-    blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2), synth.bf16_bits(b))
+    blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2), synth.bf16_bits(b),
+                                   synth.bf16_bits(smooth))
     packed = torch.from_numpy(blob).cuda()
     codes, scales, U, Y = _run_svdq(P, X, smooth, packed, g_a, gw, N)
     _check_act(codes, scales, U, X, smooth, L1, g_a)
@@ -158,7 +163,8 @@ def test_full_size_layer(P, name, M, K, N, gelu):
     assert np.array_equal(unswizzle(scales, (M + 127) // 128 * 128, K)[:M], sx)
     Xh = svdq.smooth(w.X[rows], w.smooth_inv)
     U_ref = Xh @ w.L1.astype(np.float64)
-    assert np.all(np.abs(U[rows] - U_ref) <= 1e-5 * (np.abs(Xh) @ np.abs(w.L1.astype(np.float64))) + 1e-30)
+    assert np.all(np.abs(U[rows] - U_ref) <= 1e-5 * (np.abs(Xh) @ np.abs(w.L1.astype(np.float64)))
+                  + 2.0 ** -15 * np.abs(U_ref) + 1e-30)
     y_ref = svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, w.g_a)
     check_output(Y[rows], y_ref)
     assert P.svdq_device_status() == 0

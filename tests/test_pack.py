@@ -16,14 +16,14 @@ from parity_util import unswizzle  # noqa: E402
 def _sections(blob, N, K, rank=32):
     al = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
     off = 1024
-    l1t = off; off = al(off + rank * K * 2)
+    l1s = off; off = al(off + 2 * rank * K * 2)
     codes = off; off = al(off + N * K // 2)
     scales = off; off = al(off + ((N + 127) // 128 * 128) * (K // 16))
     l2t = off; off = al(off + N * rank * 2)
     bias = off; off = al(off + N * 2)
     assert off == blob.size
     return {
-        "l1t": blob[l1t:l1t + rank * K * 2].view(np.uint16).reshape(rank, K),
+        "l1s": blob[l1s:l1s + 2 * rank * K * 2].view(np.uint16).reshape(2, rank, K),
         "codes": blob[codes:codes + N * K // 2].reshape(N, K // 2),
         "scales": blob[scales:scales + ((N + 127) // 128 * 128) * (K // 16)],
         "l2t": blob[l2t:l2t + N * rank * 2].view(np.uint16).reshape(N, rank),
@@ -31,17 +31,23 @@ def _sections(blob, N, K, rank=32):
     }
 
 
-def _check_pack(R, L1, L2, b):
+def _check_pack(R, L1, L2, b, smooth):
     N, K = R.shape
     blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2),
-                                   None if b is None else synth.bf16_bits(b))
+                                   None if b is None else synth.bf16_bits(b), synth.bf16_bits(smooth))
     cw, sw, gw_ref = svdq.quantize_weights(R)
     assert gw == gw_ref
     s = _sections(blob, N, K)
     assert np.array_equal(s["codes"], nvfp4.pack_nibbles(cw))
     assert np.array_equal(unswizzle(s["scales"], N, K), sw)
-    assert np.array_equal(s["l1t"], synth.bf16_bits(L1).T)
-    assert np.array_equal(s["l2t"], synth.bf16_bits(L2).T)
+    # (diag(smooth) L1)^T = hi + lo exactly, hi the nearest bf16
+    prod = (smooth.astype(np.float64)[:, None] * L1.astype(np.float64)).T
+    hi = synth.bf16_from_bits(s["l1s"][0]).astype(np.float64)
+    lo = synth.bf16_from_bits(s["l1s"][1]).astype(np.float64)
+    assert np.array_equal(hi + lo, prod)
+    assert np.array_equal(hi, synth.to_bf16(prod).astype(np.float64))
+    # L2 / g_w, transposed
+    assert np.array_equal(synth.bf16_from_bits(s["l2t"]).astype(np.float64), L2.astype(np.float64).T / gw)
     assert np.array_equal(s["bias"], np.zeros(N, np.uint16) if b is None else synth.bf16_bits(b))
     assert bytes(blob[:8]) == b"SVDQNVF4"
     return blob
@@ -49,12 +55,12 @@ def _check_pack(R, L1, L2, b):
 
 def test_pack_synthetic_tiny_layer_is_bit_exact():
     w = synth.svdq_workload(256, 512, 512)
-    _check_pack(w.R, w.L1, w.L2, w.bias)
+    _check_pack(w.R, w.L1, w.L2, w.bias, w.smooth_inv)
 
 
 def test_pack_attention_layer_is_bit_exact():
     w = synth.svdq_workload(64, 3072, 3072)
-    _check_pack(w.R, w.L1, w.L2, None)
+    _check_pack(w.R, w.L1, w.L2, None, w.smooth_inv)
 
 
 def test_pack_ties_zero_blocks_and_subnormal_scales():
@@ -77,15 +83,16 @@ def test_pack_ties_zero_blocks_and_subnormal_scales():
     R = R.astype(np.float32)
     L1 = synth.to_bf16(rng.standard_normal((K, 32)))
     L2 = synth.to_bf16(rng.standard_normal((32, N)))
-    _check_pack(R, L1, L2, synth.to_bf16(rng.standard_normal(N)))
+    _check_pack(R, L1, L2, synth.to_bf16(rng.standard_normal(N)), synth.to_bf16(np.exp2(rng.uniform(-3, 3, K))))
 
 
 def test_pack_rejects_bad_shapes_and_values():
-    L1 = np.zeros((64, 32), np.float32)
-    L2 = np.zeros((32, 128), np.float32)
+    L1 = np.zeros((64, 32), np.uint16)
+    L2 = np.zeros((32, 128), np.uint16)
+    sm = np.full(64, 0x3F80, np.uint16)
     with pytest.raises(P.SvdqError):
-        P.svdq_pack_weights(np.zeros((100, 64), np.float32), L1, np.zeros((32, 100), np.float32))
+        P.svdq_pack_weights(np.zeros((100, 64), np.float32), L1, np.zeros((32, 100), np.uint16), None, sm)
     R = np.zeros((128, 64), np.float32)
     R[3, 5] = np.nan
     with pytest.raises(P.SvdqError):
-        P.svdq_pack_weights(R, L1, L2)
+        P.svdq_pack_weights(R, L1, L2, None, sm)
