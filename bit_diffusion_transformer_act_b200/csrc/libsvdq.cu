@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "../../include/svdq.h"
@@ -82,6 +84,17 @@ bool set_smem_once(int bytes, int dev) {
   if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
   done[dev] = true;
   return true;
+}
+
+// Number of SMs of a device (cached).
+int sm_count(int dev) {
+  static int count[kMaxDevices];
+  if (count[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    count[dev] = c;
+  }
+  return count[dev];
 }
 
 int launch_status() {
@@ -175,40 +188,48 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   namespace k2 = svdq::k2;
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
+  const int BN = (N % 192 == 0) ? 192 : (N % 256 == 0 ? 256 : 128);
   k2::Params p;
-  p.sfa = static_cast<const uint8_t*>(act_scales);
-  p.sfb = blob + L.scales;
   p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.M = M;
   p.N = N;
   p.K = K;
+  p.tiles_n = N / BN;
+  p.tiles = ((M + 255) / 256) * p.tiles_n;
   p.alpha = static_cast<float>(alpha);
 
-  const bool wide = (N % 256 == 0);
-  const int BN = wide ? 256 : 128;
-  CUtensorMap tA, tB, tU, tL2;
+  const int natoms = K / 64;
+  const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
+  const uint64_t sfb_rows = static_cast<uint64_t>(N / 128) * natoms;
+  CUtensorMap tA, tB, tSFA, tSFB, tU, tL2;
   if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, 128, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, BN,
+      !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, BN / 2,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tSFA, act_scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, sfa_rows, 128, 128, k2::BK / 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap(&tSFB, blob + L.scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, sfb_rows, 128, 128, k2::BK / 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, 2 * rank, 2 * rank, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN,
+      !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN / 2,
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
 
-  const dim3 grid(N / BN, (M + k2::BM - 1) / k2::BM, 1);
+  const int pairs = std::min(p.tiles, sm_count(dev) / 2);
+  const dim3 grid(2 * pairs, 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (wide) {
-    const int smem = k2::Cfg<256>::SMEM_BYTES;
-    if (!set_smem_once<k2::nvfp4_gemm_kernel<256>>(smem, dev)) return SVDQ_ERR_CUDA;
-    k2::nvfp4_gemm_kernel<256><<<grid, k2::kThreads, smem, s>>>(tA, tB, tU, tL2, p);
-  } else {
-    const int smem = k2::Cfg<128>::SMEM_BYTES;
-    if (!set_smem_once<k2::nvfp4_gemm_kernel<128>>(smem, dev)) return SVDQ_ERR_CUDA;
-    k2::nvfp4_gemm_kernel<128><<<grid, k2::kThreads, smem, s>>>(tA, tB, tU, tL2, p);
-  }
+#define SVDQ_GEMM_LAUNCH(BN_)                                                                       \
+  do {                                                                                              \
+    const int smem = k2::Cfg<BN_>::SMEM_BYTES;                                                      \
+    if (!set_smem_once<k2::nvfp4_gemm_kernel<BN_>>(smem, dev)) return SVDQ_ERR_CUDA;                \
+    k2::nvfp4_gemm_kernel<BN_><<<grid, k2::kThreads, smem, s>>>(tA, tB, tSFA, tSFB, tU, tL2, p);     \
+  } while (0)
+  if (BN == 192) SVDQ_GEMM_LAUNCH(192);
+  else if (BN == 256) SVDQ_GEMM_LAUNCH(256);
+  else SVDQ_GEMM_LAUNCH(128);
+#undef SVDQ_GEMM_LAUNCH
   return launch_status();
 }
 
