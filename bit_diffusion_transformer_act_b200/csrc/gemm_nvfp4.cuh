@@ -52,10 +52,12 @@ struct Cfg {
   static constexpr int UCAT_BYTES = BM * 64 * 2;               // low-rank A tile (fits the A slot)
   static constexpr int L2_BYTES = BN_HALF * 32 * 2;            // low-rank B tile (fits the B slot)
   static constexpr int STAGES = BN == 128 ? 7 : (BN == 192 ? 6 : 5);
+  // scale factors of one stage in tensor memory: A 4 columns per MMA, B 4 per 128 rows per MMA;
+  // two such regions alternate between consecutive stages
   static constexpr int SF_COLS = 4 * (BK / 64) + 4 * SFB_ATOMS * (BK / 64);
-  static constexpr int ACC = (2 * BN + SF_COLS <= 512) ? 2 : 1;  // accumulator buffers in tensor memory
-  static constexpr uint32_t TM_SFA = ACC * BN;
-  static constexpr uint32_t TM_SFB = TM_SFA + 4 * (BK / 64);
+  static constexpr int ACC = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;  // accumulator buffers in tensor memory
+  static constexpr uint32_t TM_SF = ACC * BN;
+  static constexpr uint32_t SFB_OFF = 4 * (BK / 64);            // B's columns after A's within a region
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 5;              // full, empty, acc_full[2], acc_empty[2], drain
@@ -63,7 +65,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;      // + slack to align the base to 1024
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
-  static_assert(TM_SFB + 4 * SFB_ATOMS * (BK / 64) <= TMEM_COLS, "tensor memory overflow");
+  static_assert(TM_SF + 2 * SF_COLS <= TMEM_COLS, "tensor memory overflow");
   static_assert(STAGE_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1 KB alignment of swizzled tiles");
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -179,6 +181,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       // ------------------------------------------------------------------ MMA issuer (pair leader)
       const uint32_t id4 = idesc_nvfp4_m256<BN>();
       const uint32_t idb = idesc_bf16_m256<BN>();
+      // descriptor high words (stride, version, layout) never change; the low word is the
+      // start address >> 4 with the leading-byte-offset field set to 1 (16 B) for swizzled tiles
+      constexpr uint32_t kHiSw128 = smem_desc_hi(1024, 2);      // K-major, 128-byte swizzle
+      constexpr uint32_t kHiSw64 = smem_desc_hi(512, 4);        // K-major, 64-byte swizzle
+      constexpr uint32_t kHiSf = smem_desc_hi(128, 0);          // scale atoms: 8 rows x 16 B groups
+      constexpr uint32_t kLbo = 1u << 16;
       uint32_t g = 0;
       int i = 0;
       bool ok = true;
@@ -196,33 +204,37 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           if (!mbar_wait_bounded(full(s), ph, abort_flag, 3)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sb = base + s * C::STAGE_BYTES;
+          const uint32_t a_lo = (sb >> 4) | kLbo;
+          const uint32_t b_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
           if (kb < nkb) {
             const int na = min(BK / 64, natoms - kb * (BK / 64));
-            const uint32_t sfa_s = sb + C::A_BYTES + C::B_BYTES;
-            const uint32_t sfb_s = sfa_s + C::SFA_BYTES;
-            for (int kk = 0; kk < na; ++kk) {
-              tc_copy_32x128b_x4_pair(tmem + C::TM_SFA + 4 * kk, smem_desc(sfa_s + kk * 512, 0, 128, 0));
+            const uint32_t sfa_lo = (sb + C::A_BYTES + C::B_BYTES) >> 4;
+            const uint32_t sfb_lo = sfa_lo + C::SFA_BYTES / 16;
+            const uint32_t tsf = tmem + C::TM_SF + (g & 1u) * C::SF_COLS;
 #pragma unroll
-              for (int a = 0; a < C::SFB_ATOMS; ++a)
-                tc_copy_32x128b_x4_pair(tmem + C::TM_SFB + (kk * C::SFB_ATOMS + a) * 4,
-                                        smem_desc(sfb_s + (a * (BK / 64) + kk) * 512, 0, 128, 0));
+            for (int kk = 0; kk < BK / 64; ++kk) {
+              if (kk < na) {
+                tc_copy_32x128b_x4_pair(tsf + 4 * kk, make_desc(sfa_lo + kk * 32, kHiSf));
+#pragma unroll
+                for (int a = 0; a < C::SFB_ATOMS; ++a)
+                  tc_copy_32x128b_x4_pair(tsf + C::SFB_OFF + (kk * C::SFB_ATOMS + a) * 4,
+                                          make_desc(sfb_lo + (a * (BK / 64) + kk) * 32, kHiSf));
+              }
             }
-            for (int kk = 0; kk < na; ++kk) {
-              // K-major, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart; K step = 32 B
-              const uint64_t ad = smem_desc(sb + kk * 32, 16, 1024, 2);
-              const uint64_t bd = smem_desc(sb + C::A_BYTES + kk * 32, 16, 1024, 2);
-              umma_nvfp4_pair(dacc, ad, bd, id4, tmem + C::TM_SFA + 4 * kk,
-                              tmem + C::TM_SFB + kk * C::SFB_ATOMS * 4 + sfb_shift, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < BK / 64; ++kk) {
+              if (kk < na)
+                umma_nvfp4_pair(dacc, make_desc(a_lo + kk * 2, kHiSw128), make_desc(b_lo + kk * 2, kHiSw128), id4,
+                                tsf + 4 * kk, tsf + C::SFB_OFF + kk * C::SFB_ATOMS * 4 + sfb_shift,
+                                (kb | kk) != 0 ? 1u : 0u);
             }
           } else {
+            // A: [U hi | U lo] / g_a (128-byte swizzle); B: (L2 / g_w)^T (64-byte swizzle),
+            // K steps 0, 16, 0, 16; one K step = 16 bf16 = 32 B
+            const uint32_t l_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              // A: [U hi | U lo] / g_a, K-major, 128-byte swizzle; B: (L2 / g_w)^T, K-major,
-              // 64-byte swizzle, K steps 0, 16, 0, 16.  K step = 16 bf16 = 32 B.
-              const uint64_t ud = smem_desc(sb + j * 32, 16, 1024, 2);
-              const uint64_t ld = smem_desc(sb + C::A_BYTES + (j & 1) * 32, 16, 512, 4);
-              umma_bf16_pair(dacc, ud, ld, idb, 1u);
-            }
+            for (int j = 0; j < 4; ++j)
+              umma_bf16_pair(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(l_lo + (j & 1) * 2, kHiSw64), idb, 1u);
           }
           tc_commit_pair(empty(s), 0x3);
           if (kb == nkb) tc_commit_pair(acc_full(b), 0x3);

@@ -60,12 +60,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with parity `parity` of the mbarrier to complete.  Gives
-// up after kWaitLimitNs, or as soon as *abort becomes non-zero; then records
-// the failure in g_device_status (site in bits 8..15) and returns false.
-__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                               volatile int* abort, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait_bounded (kept out of line).
+__device__ __noinline__ bool mbar_wait_bounded_slow(uint32_t bar, uint32_t parity,
+                                                    volatile int* abort, uint32_t site) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -78,6 +75,15 @@ __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+
+// Waits for the phase with parity `parity` of the mbarrier to complete.  Gives
+// up after kWaitLimitNs, or as soon as *abort becomes non-zero; then records
+// the failure in g_device_status (site in bits 8..15) and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_bounded_slow(bar, parity, abort, site);
 }
 
 // ------------------------------------------------------------------ TMA / bulk
@@ -136,6 +142,15 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 //   bits 32-45 stride byte offset >> 4 bits 46-47 version (1)
 //   bits 49-51 base offset (0)         bit  52    LBO mode (0)
 //   bits 61-63 layout: 0 none, 2 128-byte swizzle, 4 64-byte swizzle, 6 32-byte swizzle
+// High word of a descriptor (stride byte offset, version, layout) and the descriptor
+// assembled from a precomputed high word and a low word ((start >> 4) | (LBO >> 4) << 16).
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo, uint32_t layout) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 7u) << 29);
+}
+__device__ __forceinline__ uint64_t make_desc(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
