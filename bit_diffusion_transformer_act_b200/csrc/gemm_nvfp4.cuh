@@ -141,8 +141,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------------ producer
+    {
+      // ------------------------------------------------------------------ producer (whole warp, one lane issues)
       uint32_t g = 0;
       bool ok = true;
       for (int t = pair; ok && t < p.tiles; t += npairs) {
@@ -154,9 +154,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         for (int kb = 0; kb <= nkb; ++kb) {                        // kb == nkb: the low-rank stage
           const int s = g % S;
           const uint32_t ph = (g / S) & 1u;
-          if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 1)) { ok = false; break; }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 1))) { ok = false; break; }
           const uint32_t fb = map_to_cta(full(s), 0);
           const uint32_t sb = base + s * C::STAGE_BYTES;
+          if (elect_one()) {
           if (kb < nkb) {
             if (leader) mbar_arrive_expect_tx(full(s), C::TX_MAIN);
             tma_load_2d_pair(sb, &tmA, kb * (BK / 2), m0, fb);
@@ -171,14 +172,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             tma_load_2d_pair(sb, &tmU, 0, m0, fb);
             tma_load_2d_pair(sb + C::A_BYTES, &tmL2, 0, bn0, fb);
           }
+          }
+          __syncwarp();
           ++g;
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (leader && lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer (pair leader)
+    if (leader) {
+      // ------------------------------------------------------------------ MMA issuer (pair leader; whole warp, one lane issues)
       const uint32_t id4 = idesc_nvfp4_m256<BN>();
       const uint32_t idb = idesc_bf16_m256<BN>();
       // descriptor high words (stride, version, layout) never change; the low word is the
@@ -194,18 +197,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int nt = t % p.tiles_n;
         const int b = C::ACC == 2 ? (i & 1) : 0;
         const int use = C::ACC == 2 ? (i >> 1) : i;
-        if (!mbar_wait_bounded(acc_empty(b), (use & 1) ^ 1, abort_flag, 2)) break;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_empty(b), (use & 1) ^ 1, abort_flag, 2))) break;
         tc_fence_after();
         const uint32_t dacc = tmem + static_cast<uint32_t>(b * BN);
         const uint32_t sfb_shift = static_cast<uint32_t>(((nt * BN) % 128) / 32);
         for (int kb = 0; kb <= nkb; ++kb) {
           const int s = g % S;
           const uint32_t ph = (g / S) & 1u;
-          if (!mbar_wait_bounded(full(s), ph, abort_flag, 3)) { ok = false; break; }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 3))) { ok = false; break; }
           tc_fence_after();
           const uint32_t sb = base + s * C::STAGE_BYTES;
           const uint32_t a_lo = (sb >> 4) | kLbo;
           const uint32_t b_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
+          if (elect_one()) {
           if (kb < nkb) {
             const int na = min(BK / 64, natoms - kb * (BK / 64));
             const uint32_t sfa_lo = (sb + C::A_BYTES + C::B_BYTES) >> 4;
@@ -238,6 +242,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           }
           tc_commit_pair(empty(s), 0x3);
           if (kb == nkb) tc_commit_pair(acc_full(b), 0x3);
+          }
+          __syncwarp();
           ++g;
         }
       }
@@ -254,7 +260,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int n0 = nt * BN;
       const int b = C::ACC == 2 ? (i & 1) : 0;
       const int use = C::ACC == 2 ? (i >> 1) : i;
-      if (!mbar_wait_bounded(acc_full(b), use & 1, abort_flag, 4)) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(b), use & 1, abort_flag, 4))) break;
       tc_fence_after();
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * BN);
 #pragma unroll 1
@@ -292,8 +298,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   if (*abort_flag) {
     // a wait ran out: let the MMAs and copies already issued finish before the memory goes away
-    if (warp == 1 && lane == 0 && leader) {
-      tc_commit_pair(drain, 0x1);
+    if (warp == 1 && leader) {
+      if (elect_one()) tc_commit_pair(drain, 0x1);
+      __syncwarp();
       mbar_wait_bounded(drain, 0, nullptr, 6);
     }
     if (warp == 0 && lane == 0) {

@@ -27,6 +27,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// True in exactly one lane of the (converged) warp.  Issuing tcgen05 / TMA instructions
+// under this predicate from a converged warp keeps their operands warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{ .reg .b32 r; .reg .pred p; elect.sync r|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
   asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));
