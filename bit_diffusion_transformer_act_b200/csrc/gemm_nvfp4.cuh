@@ -22,9 +22,12 @@
 //           double-buffered fp32 accumulator, and the four bf16 low-rank MMAs
 //           (K = 16); commits release the stage in both CTAs and publish the
 //           accumulator to both epilogues.
-//   warps 2-5  epilogue (both CTAs): tcgen05.ld 32 columns at a time, y = alpha acc
-//           + b (one fma), bf16 stores; then the accumulator buffer is handed back,
-//           so the next tile's mainloop overlaps this one's epilogue.
+//   warps 2-5  epilogue (both CTAs): each warp owns 32 accumulator rows; tcgen05.ld 32
+//           columns at a time (two register sets, so a load is in flight while the
+//           previous chunk is converted), y = alpha acc + b (one fma, bias staged in
+//           shared memory), bf16 into a 64-byte-swizzled 32 x 32 staging tile, TMA
+//           tensor store.  The accumulator buffer is handed back as soon as its last
+//           column is in registers, so the next tile's mainloop overlaps the stores.
 // Every mbarrier wait is bounded (about one second); a wait that runs out records
 // SVDQ_ERR_TIMEOUT in the device status word, the other roles give up, the MMAs in
 // flight are drained (bounded), tensor memory is freed and the kernel returns.
@@ -62,13 +65,17 @@ struct Cfg {
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 5;              // full, empty, acc_full[2], acc_empty[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;      // + slack to align the base to 1024
+  static constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;  // per epilogue warp: the tile's bias (BN bf16)
+  static constexpr int OFF_STAGE = (OFF_BIAS + 4 * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 2 x (32 x 32 bf16)
+  static constexpr int SMEM_BYTES = OFF_STAGE + 4 * 4096 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
   static_assert(TM_SF + 2 * SF_COLS <= TMEM_COLS, "tensor memory overflow");
   static_assert(STAGE_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1 KB alignment of swizzled tiles");
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(OFF_BIAS % 16 == 0, "16-byte shared stores of the bias");
+  static_assert(OFF_STAGE % 1024 == 0, "64-byte-swizzled store staging needs 512-byte alignment");
 };
 
 struct Params {
@@ -94,12 +101,39 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256() {
          (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
+// y = bf16(alpha acc + b) for 32 consecutive columns of one row: fp32 accumulators in r,
+// their bias (32 bf16) in shared memory at bias_smem.  The 64 result bytes go to this
+// lane's row of a 32-row staging tile in the 64-byte swizzle of the store's tensor map
+// (16-byte unit q of row r at r * 64 + 16 (q ^ ((r >> 1) & 3))).
+__device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], uint32_t bias_smem, float alpha,
+                                                 uint32_t tile_smem, uint32_t lane) {
+  const uint32_t row = tile_smem + lane * 64;
+  const uint32_t sw = (lane >> 1) & 3u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t bw[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(bw[0]), "=r"(bw[1]), "=r"(bw[2]), "=r"(bw[3]) : "r"(bias_smem + q * 16));
+    uint32_t o[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = q * 8 + w * 2;
+      const float lo = fmaf(alpha, __uint_as_float(r[j]), bf16lo_to_f32(bw[w]));
+      const float hi = fmaf(alpha, __uint_as_float(r[j + 1]), bf16hi_to_f32(bw[w]));
+      o[w] = pack_bf16x2(lo, hi);
+    }
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(row + ((static_cast<uint32_t>(q) ^ sw) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                 : "memory");
+  }
+}
+
 template <int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap tmY, const Params p) {
   using C = Cfg<BN>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -132,7 +166,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmSFA);
-    prefetch_tmap(&tmSFB); prefetch_tmap(&tmU); prefetch_tmap(&tmL2);
+    prefetch_tmap(&tmSFB); prefetch_tmap(&tmU); prefetch_tmap(&tmL2); prefetch_tmap(&tmY);
   }
   if (warp == 1) tmem_alloc_pair<C::TMEM_COLS>(smem_addr(tmem_slot));
   tc_fence_before();
@@ -252,47 +286,63 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter .. +31
-    const int row = quarter * 32 + lane;
+    const int ew = warp - 2;
+    uint8_t* sbias = gbase + C::OFF_BIAS + ew * 512;
+    const uint32_t sbias_a = smem_addr(sbias);
+    const uint32_t stage_a = base + C::OFF_STAGE + ew * 4096;   // two 2 KB staging tiles
+    uint32_t nst = 0;                              // chunks staged so far (selects the staging tile)
     int i = 0;
     for (int t = pair; t < p.tiles; t += npairs, ++i) {
       const int mt = t / p.tiles_n, nt = t % p.tiles_n;
-      const int m = mt * 256 + static_cast<int>(cta) * BM + row;
+      const int m0 = mt * 256 + static_cast<int>(cta) * BM + quarter * 32;   // this warp's first row
       const int n0 = nt * BN;
       const int b = C::ACC == 2 ? (i & 1) : 0;
       const int use = C::ACC == 2 ? (i >> 1) : i;
+      // the tile's bias goes to this warp's shared-memory slot while the mainloop runs
+      if (lane < BN / 8)
+        *reinterpret_cast<uint4*>(sbias + lane * 16) = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
+      __syncwarp();
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(b), use & 1, abort_flag, 4))) break;
       tc_fence_after();
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * BN);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(trow + c0, r);
-        tmem_wait_ld();
-        if (m < p.M) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0 + c0);
-          uint4 out[4];
-          uint32_t* o = reinterpret_cast<uint32_t*>(out);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 bv = __ldg(bp + q);
-            const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bv);
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const int j = q * 8 + w * 2;
-              const float lo = fmaf(p.alpha, __uint_as_float(r[j]), bf16lo_to_f32(bw[w]));
-              const float hi = fmaf(p.alpha, __uint_as_float(r[j + 1]), bf16hi_to_f32(bw[w]));
-              o[q * 4 + w] = pack_bf16x2(lo, hi);
-            }
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n0 + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = out[q];
+      const bool live = m0 < p.M;                  // warp-uniform: rows past M are clipped by the store
+      // converts one chunk into a staging tile and stores it; the tile was last used two
+      // chunks ago, so at most one earlier store may still be reading shared memory
+      auto emit = [&](const uint32_t (&r)[32], int c0) {
+        const uint32_t tile = stage_a + (nst & 1u) * 2048u;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        epilogue_stage32(r, sbias_a + c0 * 2, p.alpha, tile, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, tile, n0 + c0, m0);
+          bulk_commit_group();
         }
+        ++nst;
+      };
+      // two register sets: the load of chunk c + 1 is in flight while chunk c is converted
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(trow, ra);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 64) {
+        tmem_wait_ld_regs(ra);
+        tmem_ld_32x32b_x32(trow + c0 + 32, rb);
+        if (live) emit(ra, c0);
+        tmem_wait_ld_regs(rb);
+        if (c0 + 64 < BN) {
+          tmem_ld_32x32b_x32(trow + c0 + 64, ra);
+        } else {
+          // every column of the buffer is in registers: hand it back to the leader
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_to_cta(acc_empty(b), 0));
+        }
+        if (live) emit(rb, c0 + 32);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_cta(acc_empty(b), 0));   // hand the buffer back to the leader
     }
+    if (lane == 0) bulk_wait_group<0>();           // stores complete before shared memory goes away
+    __syncwarp();
   }
 
   __syncthreads();

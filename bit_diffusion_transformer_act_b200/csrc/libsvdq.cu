@@ -202,7 +202,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   const int natoms = K / 64;
   const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
   const uint64_t sfb_rows = static_cast<uint64_t>(N / 128) * natoms;
-  CUtensorMap tA, tB, tSFA, tSFB, tU, tL2;
+  CUtensorMap tA, tB, tSFA, tSFB, tU, tL2, tY;
   if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, 128, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, BN / 2,
@@ -214,7 +214,8 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
       !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, 2 * rank, 2 * rank, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN / 2,
-                 CU_TENSOR_MAP_SWIZZLE_64B))
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_tmap(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
 
   const int pairs = std::min(p.tiles, sm_count(dev) / 2);
@@ -224,7 +225,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   do {                                                                                              \
     const int smem = k2::Cfg<BN_>::SMEM_BYTES;                                                      \
     if (!set_smem_once<k2::nvfp4_gemm_kernel<BN_>>(smem, dev)) return SVDQ_ERR_CUDA;                \
-    k2::nvfp4_gemm_kernel<BN_><<<grid, k2::kThreads, smem, s>>>(tA, tB, tSFA, tSFB, tU, tL2, p);     \
+    k2::nvfp4_gemm_kernel<BN_><<<grid, k2::kThreads, smem, s>>>(tA, tB, tSFA, tSFB, tU, tL2, tY, p);     \
   } while (0)
   if (BN == 192) SVDQ_GEMM_LAUNCH(192);
   else if (BN == 256) SVDQ_GEMM_LAUNCH(256);
