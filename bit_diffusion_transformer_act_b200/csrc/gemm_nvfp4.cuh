@@ -58,8 +58,16 @@ struct Cfg {
   // scale factors of one stage in tensor memory: A 4 columns per MMA, B 4 per 128 rows per MMA;
   // two such regions alternate between consecutive stages
   static constexpr int SF_COLS = 4 * (BK / 64) + 4 * SFB_ATOMS * (BK / 64);
-  static constexpr int ACC = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;  // accumulator buffers in tensor memory
-  static constexpr uint32_t TM_SF = ACC * BN;
+  // Two accumulator buffers.  When two full buffers and the scale regions do not fit in
+  // the 512 columns (BN = 256), the second buffer overlaps the end of the first; the
+  // epilogue reads the shared columns first and releases the accumulator as soon as
+  // they are in registers (one barrier stage instead of two).
+  static constexpr bool OVERLAP = 2 * BN + 2 * SF_COLS > 512;
+  static constexpr int ACC1 = OVERLAP ? 512 - 2 * SF_COLS - BN : BN;   // first column of buffer 1
+  static constexpr int NCH = BN / 32;                                  // 32-column epilogue chunks
+  static constexpr int OV_CHUNKS = OVERLAP ? (BN - ACC1 + 31) / 32 : 0;
+  static constexpr int ACC_STAGES = OVERLAP ? 1 : 2;                   // accumulator barrier stages
+  static constexpr uint32_t TM_SF = ACC1 + BN;
   static constexpr uint32_t SFB_OFF = 4 * (BK / 64);            // B's columns after A's within a region
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -71,6 +79,7 @@ struct Cfg {
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
   static_assert(TM_SF + 2 * SF_COLS <= TMEM_COLS, "tensor memory overflow");
+  static_assert(!OVERLAP || (ACC1 % 32 == 0 && ACC1 > 0), "overlap is a whole number of epilogue chunks");
   static_assert(STAGE_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1 KB alignment of swizzled tiles");
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -229,11 +238,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       bool ok = true;
       for (int t = pair; ok && t < p.tiles; t += npairs, ++i) {
         const int nt = t % p.tiles_n;
-        const int b = C::ACC == 2 ? (i & 1) : 0;
-        const int use = C::ACC == 2 ? (i >> 1) : i;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_empty(b), (use & 1) ^ 1, abort_flag, 2))) break;
+        const int b = i & 1;                       // accumulator buffer
+        const int ab = C::ACC_STAGES == 2 ? b : 0; // its barrier stage
+        const int use = C::ACC_STAGES == 2 ? (i >> 1) : i;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_empty(ab), (use & 1) ^ 1, abort_flag, 2))) break;
         tc_fence_after();
-        const uint32_t dacc = tmem + static_cast<uint32_t>(b * BN);
+        const uint32_t dacc = tmem + static_cast<uint32_t>(b * C::ACC1);
         const uint32_t sfb_shift = static_cast<uint32_t>(((nt * BN) % 128) / 32);
         for (int kb = 0; kb <= nkb; ++kb) {
           const int s = g % S;
@@ -275,7 +285,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
               umma_bf16_pair(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(l_lo + (j & 1) * 2, kHiSw64), idb, 1u);
           }
           tc_commit_pair(empty(s), 0x3);
-          if (kb == nkb) tc_commit_pair(acc_full(b), 0x3);
+          if (kb == nkb) tc_commit_pair(acc_full(ab), 0x3);
           }
           __syncwarp();
           ++g;
@@ -296,15 +306,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int mt = t / p.tiles_n, nt = t % p.tiles_n;
       const int m0 = mt * 256 + static_cast<int>(cta) * BM + quarter * 32;   // this warp's first row
       const int n0 = nt * BN;
-      const int b = C::ACC == 2 ? (i & 1) : 0;
-      const int use = C::ACC == 2 ? (i >> 1) : i;
+      const int b = i & 1;
+      const int ab = C::ACC_STAGES == 2 ? b : 0;
+      const int use = C::ACC_STAGES == 2 ? (i >> 1) : i;
       // the tile's bias goes to this warp's shared-memory slot while the mainloop runs
       if (lane < BN / 8)
         *reinterpret_cast<uint4*>(sbias + lane * 16) = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
       __syncwarp();
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(b), use & 1, abort_flag, 4))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(ab), use & 1, abort_flag, 4))) break;
       tc_fence_after();
-      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * BN);
+      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * C::ACC1);
       const bool live = m0 < p.M;                  // warp-uniform: rows past M are clipped by the store
       // converts one chunk into a staging tile and stores it; the tile was last used two
       // chunks ago, so at most one earlier store may still be reading shared memory
@@ -321,24 +332,30 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
         ++nst;
       };
-      // two register sets: the load of chunk c + 1 is in flight while chunk c is converted
+      // Chunk order: with overlapping buffers, the columns shared with the other buffer come
+      // first (the end of buffer 0, the start of buffer 1) and the accumulator is released
+      // once they are in registers; otherwise after the last chunk.
+      const int rot = (C::OVERLAP && b == 0) ? C::NCH - C::OV_CHUNKS : 0;
+      constexpr int kRelease = C::OVERLAP ? C::OV_CHUNKS : C::NCH;   // chunks read before the release
+      auto col = [&](int j) { return ((j + rot) % C::NCH) * 32; };
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(map_to_cta(acc_empty(ab), 0));
+      };
+      // two register sets: the load of chunk j + 1 is in flight while chunk j is converted
       uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(trow, ra);
+      tmem_ld_32x32b_x32(trow + col(0), ra);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 64) {
+      for (int j = 0; j < C::NCH; j += 2) {
         tmem_wait_ld_regs(ra);
-        tmem_ld_32x32b_x32(trow + c0 + 32, rb);
-        if (live) emit(ra, c0);
+        if (j == kRelease - 1) release();
+        tmem_ld_32x32b_x32(trow + col(j + 1), rb);
+        if (live) emit(ra, col(j));
         tmem_wait_ld_regs(rb);
-        if (c0 + 64 < BN) {
-          tmem_ld_32x32b_x32(trow + c0 + 64, ra);
-        } else {
-          // every column of the buffer is in registers: hand it back to the leader
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(map_to_cta(acc_empty(b), 0));
-        }
-        if (live) emit(rb, c0 + 32);
+        if (j + 1 == kRelease - 1) release();
+        if (j + 2 < C::NCH) tmem_ld_32x32b_x32(trow + col(j + 2), ra);
+        if (live) emit(rb, col(j + 1));
       }
     }
     if (lane == 0) bulk_wait_group<0>();           // stores complete before shared memory goes away

@@ -188,7 +188,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   namespace k2 = svdq::k2;
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
-  const int BN = (N % 192 == 0) ? 192 : (N % 256 == 0 ? 256 : 128);
+  const int BN = (N % 256 == 0) ? 256 : (N % 192 == 0 ? 192 : 128);
   k2::Params p;
   p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);

@@ -147,6 +147,9 @@ FULL = [
     ("mlp-down 4608x12288->3072 (gelu)", 4608, 12288, 3072, True),
     ("qkv 64x3072->9216", 64, 3072, 9216, False),
     ("qkv 18432x3072->9216", 18432, 3072, 9216, False),
+    # N not a multiple of 256: 192- and 128-wide output tiles, several per CTA pair
+    ("192-wide tiles 8192x1024->1152", 8192, 1024, 1152, False),
+    ("128-wide tiles 8192x512->640", 8192, 512, 640, False),
 ]
 
 
