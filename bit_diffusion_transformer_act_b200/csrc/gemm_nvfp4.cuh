@@ -25,9 +25,9 @@
 //   warps 2-5  epilogue (both CTAs): each warp owns 32 accumulator rows; tcgen05.ld 32
 //           columns at a time (two register sets, so a load is in flight while the
 //           previous chunk is converted), y = alpha acc + b (one fma, bias staged in
-//           shared memory), bf16 into a 64-byte-swizzled 32 x 32 staging tile, TMA
-//           tensor store.  The accumulator buffer is handed back as soon as its last
-//           column is in registers, so the next tile's mainloop overlaps the stores.
+//           shared memory), bf16 into a 128-byte-swizzled 32 x 64 staging tile, one TMA
+//           tensor store per 64 columns.  The accumulator buffer is handed back as soon
+//           as the columns the next tile will overwrite are in registers.
 // Every mbarrier wait is bounded (about one second); a wait that runs out records
 // SVDQ_ERR_TIMEOUT in the device status word, the other roles give up, the MMAs in
 // flight are drained (bounded), tensor memory is freed and the kernel returns.
@@ -74,7 +74,7 @@ struct Cfg {
   static constexpr int NUM_BARS = 2 * STAGES + 5;              // full, empty, acc_full[2], acc_empty[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;  // per epilogue warp: the tile's bias (BN bf16)
-  static constexpr int OFF_STAGE = (OFF_BIAS + 4 * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 2 x (32 x 32 bf16)
+  static constexpr int OFF_STAGE = (OFF_BIAS + 4 * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 64 bf16
   static constexpr int SMEM_BYTES = OFF_STAGE + 4 * 4096 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
@@ -84,7 +84,8 @@ struct Cfg {
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(OFF_BIAS % 16 == 0, "16-byte shared stores of the bias");
-  static_assert(OFF_STAGE % 1024 == 0, "64-byte-swizzled store staging needs 512-byte alignment");
+  static_assert(OFF_STAGE % 1024 == 0, "128-byte-swizzled store staging needs 1024-byte alignment");
+  static_assert(!OVERLAP || (NCH == 8 && OV_CHUNKS == 3), "chunk order of the overlapping buffers");
 };
 
 struct Params {
@@ -111,28 +112,30 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256() {
 }
 
 // y = bf16(alpha acc + b) for 32 consecutive columns of one row: fp32 accumulators in r,
-// their bias (32 bf16) in shared memory at bias_smem.  The 64 result bytes go to this
-// lane's row of a 32-row staging tile in the 64-byte swizzle of the store's tensor map
-// (16-byte unit q of row r at r * 64 + 16 (q ^ ((r >> 1) & 3))).
-__device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], uint32_t bias_smem, float alpha,
-                                                 uint32_t tile_smem, uint32_t lane) {
-  const uint32_t row = tile_smem + lane * 64;
-  const uint32_t sw = (lane >> 1) & 3u;
+// their bias (32 bf16) at bias (shared memory).  The 64 result bytes are half `half` of
+// this lane's 128-byte row of a 32-row staging tile in the 128-byte swizzle of the
+// store's tensor map (16-byte unit u of row r at r * 128 + 16 (u ^ (r & 7))).
+__device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], const uint4* bias, float alpha,
+                                                 uint32_t row_smem, uint32_t sw, int half) {
+  uint32_t o[16];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t bw[4];
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(bw[0]), "=r"(bw[1]), "=r"(bw[2]), "=r"(bw[3]) : "r"(bias_smem + q * 16));
-    uint32_t o[4];
+    const uint4 bv = bias[q];
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int j = q * 8 + w * 2;
       const float lo = fmaf(alpha, __uint_as_float(r[j]), bf16lo_to_f32(bw[w]));
       const float hi = fmaf(alpha, __uint_as_float(r[j + 1]), bf16hi_to_f32(bw[w]));
-      o[w] = pack_bf16x2(lo, hi);
+      o[q * 4 + w] = pack_bf16x2(lo, hi);
     }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t u = static_cast<uint32_t>(half * 4 + q);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(row + ((static_cast<uint32_t>(q) ^ sw) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                 ::"r"(row_smem + ((u ^ sw) << 4)), "r"(o[q * 4]), "r"(o[q * 4 + 1]), "r"(o[q * 4 + 2]),
+                   "r"(o[q * 4 + 3])
                  : "memory");
   }
 }
@@ -299,8 +302,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int ew = warp - 2;
     uint8_t* sbias = gbase + C::OFF_BIAS + ew * 512;
     const uint32_t sbias_a = smem_addr(sbias);
-    const uint32_t stage_a = base + C::OFF_STAGE + ew * 4096;   // two 2 KB staging tiles
-    uint32_t nst = 0;                              // chunks staged so far (selects the staging tile)
+    const uint32_t stage_row = base + C::OFF_STAGE + ew * 4096 + lane * 128;   // this lane's staging row
+    const uint32_t stage_tile = base + C::OFF_STAGE + ew * 4096;
     int i = 0;
     for (int t = pair; t < p.tiles; t += npairs, ++i) {
       const int mt = t / p.tiles_n, nt = t % p.tiles_n;
@@ -317,45 +320,53 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       tc_fence_after();
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * C::ACC1);
       const bool live = m0 < p.M;                  // warp-uniform: rows past M are clipped by the store
-      // converts one chunk into a staging tile and stores it; the tile was last used two
-      // chunks ago, so at most one earlier store may still be reading shared memory
-      auto emit = [&](const uint32_t (&r)[32], int c0) {
-        const uint32_t tile = stage_a + (nst & 1u) * 2048u;
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
-        epilogue_stage32(r, sbias_a + c0 * 2, p.alpha, tile, lane);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmY, tile, n0 + c0, m0);
-          bulk_commit_group();
-        }
-        ++nst;
+      // Chunk order (32 columns each; consecutive pairs form one 64-column store).  With
+      // overlapping buffers the columns shared with the other buffer come first (chunks
+      // 5-7 of buffer 0, 0-2 of buffer 1) and the accumulator is released once they are
+      // in registers; otherwise it is released after the last chunk.
+      const bool swap = C::OVERLAP && b == 0;
+      auto chunk = [&](int j) {
+        if (!swap) return j;
+        return j < 2 ? 6 + j : (j < 4 ? 7 - j : j - 4);        // 6 7 5 4 0 1 2 3
       };
-      // Chunk order: with overlapping buffers, the columns shared with the other buffer come
-      // first (the end of buffer 0, the start of buffer 1) and the accumulator is released
-      // once they are in registers; otherwise after the last chunk.
-      const int rot = (C::OVERLAP && b == 0) ? C::NCH - C::OV_CHUNKS : 0;
-      constexpr int kRelease = C::OVERLAP ? C::OV_CHUNKS : C::NCH;   // chunks read before the release
-      auto col = [&](int j) { return ((j + rot) % C::NCH) * 32; };
+      constexpr int kRelease = C::OVERLAP ? C::OV_CHUNKS : C::NCH;
       auto release = [&]() {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_to_cta(acc_empty(ab), 0));
+        if (lane == 0) mbar_arrive_remote(map_to_cta(acc_empty(ab), 0));
+      };
+      // converts one chunk into its half of the staging tile; after the second half the
+      // tile goes out with one TMA store (the previous store must have finished reading it)
+      auto emit = [&](const uint32_t (&r)[32], int j) {
+        const int c = chunk(j);
+        const int half = c & 1;
+        if ((j & 1) == 0) {
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        }
+        epilogue_stage32(r, reinterpret_cast<const uint4*>(sbias + c * 64), p.alpha, stage_row, lane & 7u, half);
+        if (j & 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, stage_tile, n0 + (c >> 1) * 64, m0);
+            bulk_commit_group();
+          }
+        }
       };
       // two register sets: the load of chunk j + 1 is in flight while chunk j is converted
       uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(trow + col(0), ra);
+      tmem_ld_32x32b_x32(trow + chunk(0) * 32, ra);
 #pragma unroll 1
       for (int j = 0; j < C::NCH; j += 2) {
         tmem_wait_ld_regs(ra);
         if (j == kRelease - 1) release();
-        tmem_ld_32x32b_x32(trow + col(j + 1), rb);
-        if (live) emit(ra, col(j));
+        tmem_ld_32x32b_x32(trow + chunk(j + 1) * 32, rb);
+        if (live) emit(ra, j);
         tmem_wait_ld_regs(rb);
         if (j + 1 == kRelease - 1) release();
-        if (j + 2 < C::NCH) tmem_ld_32x32b_x32(trow + col(j + 2), ra);
-        if (live) emit(rb, col(j + 1));
+        if (j + 2 < C::NCH) tmem_ld_32x32b_x32(trow + chunk(j + 2) * 32, ra);
+        if (live) emit(rb, j + 1);
       }
     }
     if (lane == 0) bulk_wait_group<0>();           // stores complete before shared memory goes away

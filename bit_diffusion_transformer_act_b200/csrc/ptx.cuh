@@ -346,6 +346,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
+// Arrives on an mbarrier of another CTA of the cluster with the default semantics
+// (release at CTA scope): enough when the arrival only publishes completed tensor-memory
+// reads, and much cheaper than a cluster-scope release.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
 // TMA tile load into this CTA's shared memory whose completion is signalled on an
 // mbarrier that may live in the peer CTA of the pair (used by both CTAs of a pair).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int x, int y,
