@@ -185,6 +185,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   cluster_sync_all();                              // barriers of both CTAs initialised and visible
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above overlaps the previous kernel of the stream; its outputs (this
+  // kernel's inputs) and its reads of Y are complete past this point
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     {
@@ -354,19 +358,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           }
         }
       };
-      // two register sets: the load of chunk j + 1 is in flight while chunk j is converted
-      uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(trow + chunk(0) * 32, ra);
-#pragma unroll 1
-      for (int j = 0; j < C::NCH; j += 2) {
-        tmem_wait_ld_regs(ra);
-        if (j == kRelease - 1) release();
-        tmem_ld_32x32b_x32(trow + chunk(j + 1) * 32, rb);
-        if (live) emit(ra, j);
-        tmem_wait_ld_regs(rb);
-        if (j + 1 == kRelease - 1) release();
-        if (j + 2 < C::NCH) tmem_ld_32x32b_x32(trow + chunk(j + 2) * 32, ra);
-        if (live) emit(rb, j + 1);
+      // Three register sets in rotation: chunks 0-2 are loaded up front; every third chunk
+      // one wait covers the three loads issued while the previous three were converted.
+      // With overlapping buffers the release follows the first wait, otherwise the last.
+      uint32_t R[3][32];
+#pragma unroll
+      for (int j = 0; j < 3 && j < C::NCH; ++j) tmem_ld_32x32b_x32(trow + chunk(j) * 32, R[j]);
+#pragma unroll
+      for (int j = 0; j < C::NCH; ++j) {
+        if (j % 3 == 0) {
+#pragma unroll
+          for (int k = 0; k < 3 && j + k < C::NCH; ++k) tmem_wait_ld_regs(R[k]);
+          if (j + 3 >= kRelease && j < kRelease) release();
+        }
+        if (live) emit(R[j % 3], j);
+        if (j + 3 < C::NCH) tmem_ld_32x32b_x32(trow + chunk(j + 3) * 32, R[j % 3]);
       }
     }
     if (lane == 0) bulk_wait_group<0>();           // stores complete before shared memory goes away

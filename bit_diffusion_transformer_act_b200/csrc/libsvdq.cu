@@ -155,13 +155,15 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   cfg.blockDim = dim3(k1::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = ks;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
@@ -225,7 +227,21 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   do {                                                                                              \
     const int smem = k2::Cfg<BN_>::SMEM_BYTES;                                                      \
     if (!set_smem_once<k2::nvfp4_gemm_kernel<BN_>>(smem, dev)) return SVDQ_ERR_CUDA;                \
-    k2::nvfp4_gemm_kernel<BN_><<<grid, k2::kThreads, smem, s>>>(tA, tB, tSFA, tSFB, tU, tL2, tY, p);     \
+    cudaLaunchConfig_t cfg = {};                                                                    \
+    cfg.gridDim = grid;                                                                             \
+    cfg.blockDim = dim3(k2::kThreads, 1, 1);                                                        \
+    cfg.dynamicSmemBytes = smem;                                                                    \
+    cfg.stream = s;                                                                                 \
+    cudaLaunchAttribute attr[1];                                                                    \
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;                                \
+    attr[0].val.programmaticStreamSerializationAllowed = 1;                                         \
+    cfg.attrs = attr;                                                                               \
+    cfg.numAttrs = 1;                                                                               \
+    if (cudaLaunchKernelEx(&cfg, k2::nvfp4_gemm_kernel<BN_>, tA, tB, tSFA, tSFB, tU, tL2, tY, p) !=  \
+        cudaSuccess) {                                                                              \
+      (void)cudaGetLastError();                                                                     \
+      return SVDQ_ERR_CUDA;                                                                         \
+    }                                                                                               \
   } while (0)
   if (BN == 192) SVDQ_GEMM_LAUNCH(192);
   else if (BN == 256) SVDQ_GEMM_LAUNCH(256);

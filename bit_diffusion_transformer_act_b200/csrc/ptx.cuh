@@ -41,6 +41,15 @@ __device__ __forceinline__ uint32_t lane_id() {
   return l;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Blocks until the grids this one depends on (the previous kernels of the stream) have
+// completed and their memory is visible; a no-op for a normally launched grid.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream be scheduled before this grid completes (it still
+// waits for this grid's completion in its own grid_dependency_wait).
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -152,6 +152,8 @@ quant_act_lowrank_kernel(const Params p) {
   const int kbeg = slice * klen;
   const int nchunks = (klen + kChunk - 1) / kChunk;
 
+  grid_dependency_wait();                          // X and the outputs may belong to the previous kernel
+  grid_launch_dependents();
   load_chunk(s, 0, p, m0, kbeg, min(kChunk, klen));
   for (int i = tid; i < klen; i += kThreads) s.smooth[i] = __bfloat162float(p.smooth[kbeg + i]);
 
