@@ -123,9 +123,7 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   namespace k1 = svdq::k1;
   const svdq::BlobLayout L = svdq::blob_layout(0, K, rank);   // the L1 section does not depend on N
   k1::Params p;
-  p.X = static_cast<const __nv_bfloat16*>(X);
   p.smooth = static_cast<const __nv_bfloat16*>(smooth_inv);
-  p.l1s = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(packed_w) + L.l1s);
   p.codes = static_cast<uint8_t*>(act_codes);
   p.scales = static_cast<uint8_t*>(act_scales);
   p.ucat = static_cast<__nv_bfloat16*>(lowrank_act);
@@ -147,7 +145,13 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   while (ks < 8 && kgroups % (2 * ks) == 0 && rowblocks * ks < 2 * 148) ks *= 2;
   p.kslices = ks;
 
-  const int smem = static_cast<int>(sizeof(k1::Smem));
+  CUtensorMap tX, tL;
+  if (!make_tmap(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, k1::kChunk, k1::kRows,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tL, static_cast<const uint8_t*>(packed_w) + L.l1s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                 2 * k1::kRank, K, k1::kChunk, 2 * k1::kRank, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  const int smem = k1::kSmemBytes;
   if (!set_smem_once<k1::quant_act_lowrank_kernel>(smem, dev)) return SVDQ_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};
@@ -164,7 +168,7 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel, tX, tL, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }

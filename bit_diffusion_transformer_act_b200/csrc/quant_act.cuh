@@ -7,20 +7,28 @@
 // S = RNE(amax / (6 g_a)) and E2M1 codes RNE(clamp(X_hat / (S g_a))); and
 // U = X_hat L1 (rank 32) from the same smoothed activations.
 //
-// Design (sm_100a).  A CTA (8 warps) owns 128 rows and one K slice; the K
-// slices of a row block form a thread-block cluster (1..8 CTAs) so the grid
-// fills the 148 SMs, and the partial U of the slices is summed over
-// distributed shared memory -- no global scratch, no atomics.  X and the L1
-// operand arrive in 128-column chunks, double-buffered in shared memory with
-// cp.async (rows past M zero-filled) and XOR-swizzled against bank conflicts.
-//   * Quantization: each thread owns one row and 64 consecutive columns (four
-//     16-element groups, i.e. one 32-bit word of the scale layout and 32
-//     contiguous code bytes, stored directly).
-//   * Low-rank: X_hat L1 = X (diag(smooth_inv) L1); the packed weights hold
-//     diag(smooth_inv) L1 split exactly into bf16 hi + lo, so ldmatrix feeds
-//     the raw bf16 X tile to mma.sync twice (hi, lo) with fp32 accumulation:
-//     every product is exact.  The result U / g_a is written split into bf16
-//     hi + lo, the operand layout of the GEMM's low-rank MMA.
+// Design (sm_100a).  A CTA owns 128 rows and one K slice; the K slices of a row
+// block form a thread-block cluster (1..8 CTAs) so that the grid fills the SMs
+// (two CTAs per SM), and the slices' partial U are summed over distributed
+// shared memory -- no global scratch, no atomics.  Warp roles:
+//   warp 0     TMA producer: per 64-column chunk the X tile (128 rows, 128-byte
+//              swizzle; rows past M read as zeros) and the matching 64 x 64 tile
+//              of the packed low-rank operand, into a ring of stages.
+//   warp 1     tensor memory and the low-rank MMA: X_hat L1 = X (diag(smooth_inv)
+//              L1), and the packed weights hold diag(smooth_inv) L1 split exactly
+//              into bf16 hi + lo, so one tcgen05 MMA (M = 128, N = 64 = 32 hi + 32
+//              lo columns, K = 16) per 16 columns multiplies the raw X tile with
+//              every product exact, accumulating in fp32 in tensor memory.
+//   warps 2-9  quantizers: a thread owns 32 columns (two groups) of one row of the
+//              chunk, reads X from the swizzled tile, smooths, finds the group
+//              maxima, the E4M3 scales and E2M1 codes, and stores 16 code bytes and
+//              2 scale bytes straight to global memory.
+// A stage is free again when the eight quantizer warps have read it and the MMAs
+// that read it have completed (tcgen05.commit).  At the end, warps 2-5 (one per
+// tensor-memory lane quarter) read U = hi + lo, the cluster sums the slices, and
+// U / g_a is written split into bf16 hi + lo, the operand layout of the GEMM's
+// low-rank MMA.  Every mbarrier wait is bounded; a wait that runs out records
+// SVDQ_ERR_TIMEOUT in the device status word and the CTA winds down.
 //
 // Rounding.  amax/6 is formed by a Markstein-corrected multiplication by the
 // rounded reciprocal of 6 (P. Markstein's correction: with y = RN(1/b) and
@@ -40,60 +48,38 @@
 namespace svdq {
 namespace k1 {
 
-constexpr int kRows = 128;                // rows per CTA
-constexpr int kWarps = 8;                 // 16 rows each for the low-rank MMA
-constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 128;               // K columns per pipeline chunk
+constexpr int kRows = 128;                // rows per CTA (one 128-row scale block)
+constexpr int kChunk = 64;                // K columns per pipeline stage
 constexpr int kRank = 32;
+constexpr int kQuantWarps = 8;
+constexpr int kThreads = (2 + kQuantWarps) * 32;
+constexpr int kStages = 4;
 constexpr int kMaxSlice = 2048;           // longest K slice (columns) held as fp32 smoothing factors
-
-struct __align__(128) Smem {
-  __nv_bfloat16 x[2][kRows * kChunk];     // rows of 256 B, 16-B pieces XOR-swizzled by (row & 7)
-  __nv_bfloat16 lh[2][kRank * kChunk];    // (diag(s) L1)^T high part, same swizzle
-  __nv_bfloat16 ll[2][kRank * kChunk];    // low part
-  float smooth[kMaxSlice];                // this CTA's slice of smooth_inv, as floats
-};
-// The partial U of the CTA (128 x 32 fp32) reuses the X buffers once the K loop is done.
-static_assert(sizeof(__nv_bfloat16) * 2 * kRows * kChunk >= sizeof(float) * kRows * kRank, "upart alias");
-
-// Byte offset of element (row, col) in a swizzled [rows][128] bf16 chunk.
-__device__ __forceinline__ uint32_t swz(int row, int col) {
-  return static_cast<uint32_t>(row * 256 + ((((col >> 3) ^ (row & 7)) << 4)) + ((col & 7) << 1));
-}
+constexpr int kXBytes = kRows * kChunk * 2;          // 16 KB
+constexpr int kLBytes = 2 * kRank * kChunk * 2;      // 8 KB: 64 operand rows (hi, lo) x 64 columns
+constexpr int kStageBytes = kXBytes + kLBytes;
+constexpr int kTmemCols = 64;
 
 struct Params {
-  const __nv_bfloat16* X;          // [M, K]
-  const __nv_bfloat16* smooth;     // [K]
-  const __nv_bfloat16* l1s;        // [2][32][K]: (diag(smooth) L1)^T hi, then lo
   uint8_t* codes;                  // [M, K/2]
   uint8_t* scales;                 // swizzled, rows padded to 128
   __nv_bfloat16* ucat;             // [M, 64]: U / g_a as bf16 hi (0..31) and lo (32..63)
+  const __nv_bfloat16* smooth;     // [K]
   int M, K;
   int kslices;                     // cluster size along K
   float g;                         // per-tensor scale (power of two)
   float inv_g;
 };
 
-__device__ __forceinline__ void load_chunk(Smem& s, int buf, const Params& p, int m0, int kc, int ncols) {
-  const int tid = threadIdx.x;
-  const int pieces = ncols / 8;                       // 16-B pieces per row
-  const uint32_t xbase = smem_addr(s.x[buf]);
-  for (int i = tid; i < kRows * pieces; i += kThreads) {
-    const int r = i / pieces, c = (i % pieces) * 8;
-    const int m = m0 + r;
-    const bool ok = m < p.M;
-    const __nv_bfloat16* src = p.X + (ok ? (static_cast<size_t>(m) * p.K + kc + c) : 0);
-    cp_async_16(xbase + swz(r, c), src, ok ? 16u : 0u);
-  }
-  const uint32_t hbase = smem_addr(s.lh[buf]), lbase = smem_addr(s.ll[buf]);
-  const __nv_bfloat16* lo_src = p.l1s + static_cast<size_t>(kRank) * p.K;
-  for (int i = tid; i < kRank * pieces; i += kThreads) {
-    const int r = i / pieces, c = (i % pieces) * 8;
-    cp_async_16(hbase + swz(r, c), p.l1s + static_cast<size_t>(r) * p.K + kc + c, 16u);
-    cp_async_16(lbase + swz(r, c), lo_src + static_cast<size_t>(r) * p.K + kc + c, 16u);
-  }
-  cp_async_commit();
-}
+// Shared memory (1024-byte aligned base): stages | smooth slice (fp32) | barriers.
+constexpr int kOffSmooth = kStages * kStageBytes;
+constexpr int kOffBar = kOffSmooth + kMaxSlice * 4;
+constexpr int kNumBars = 2 * kStages + 2;           // full, empty, acc_full, drain
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+static_assert(kRows * kRank * 4 <= kStages * kStageBytes, "partial U reuses the stages");
+static_assert(kStageBytes % 1024 == 0 && kXBytes % 1024 == 0, "1 KB alignment of swizzled tiles");
 
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
@@ -118,14 +104,14 @@ __device__ __forceinline__ float div6(float a) {
 }
 
 // Quantizes 16 smoothed values (one group): returns the E4M3 scale code, writes 8 code bytes.
-__device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], const Params& p, uint2& out) {
+__device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], float g, float inv_g, uint2& out) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const uint32_t sc = cvt_e4m3x2(div6(amax) * p.inv_g, 0.f) & 0xFFu;
+  const uint32_t sc = cvt_e4m3x2(div6(amax) * inv_g, 0.f) & 0xFFu;
   float S, unused;
   e4m3x2_to_f32(sc, S, unused);
-  const float D = S * p.g;
+  const float D = S * g;
   if (D == 0.f) {
     out = make_uint2(0u, 0u);
     return 0u;
@@ -138,152 +124,204 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], const P
   return sc;
 }
 
+// kind::f16 instruction descriptor: D f32, A and B bf16, K-major, N = 64, M = 128.
+__device__ __forceinline__ uint32_t idesc_lowrank() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(64 >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
-quant_act_lowrank_kernel(const Params p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
+quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL,
+                         const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + kOffBar;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (kStages + s); };
+  const uint32_t acc_full = bars + 8u * (2 * kStages);
+  const uint32_t drain = bars + 8u * (2 * kStages + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
+  float* smooth = reinterpret_cast<float*>(gbase + kOffSmooth);
 
   const int tid = threadIdx.x;
   const int warp = tid / 32;
   const int lane = tid % 32;
   const int m0 = blockIdx.x * kRows;
-  const int slice = blockIdx.y;
   const int klen = p.K / p.kslices;
-  const int kbeg = slice * klen;
-  const int nchunks = (klen + kChunk - 1) / kChunk;
+  const int kbeg = blockIdx.y * klen;
+  const int nck = klen / kChunk;
 
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), kQuantWarps + 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmL);
+  }
+  if (warp == 1) tmem_alloc<kTmemCols>(smem_addr(tmem_slot));
   grid_dependency_wait();                          // X and the outputs may belong to the previous kernel
   grid_launch_dependents();
-  load_chunk(s, 0, p, m0, kbeg, min(kChunk, klen));
-  for (int i = tid; i < klen; i += kThreads) s.smooth[i] = __bfloat162float(p.smooth[kbeg + i]);
+  for (int i = tid; i < klen; i += kThreads) smooth[i] = __bfloat162float(p.smooth[kbeg + i]);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  float acc[4][4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int t = 0; t < 4; ++t) acc[j][t] = 0.f;
-
-  // quantization role of this thread: row qr, columns [64 qh, 64 qh + 64) of each chunk
-  const int qr = tid >> 1, qh = tid & 1;
-  const int qm = m0 + qr;
-
-  for (int ci = 0; ci < nchunks; ++ci) {
-    const int buf = ci & 1;
-    const int kc = kbeg + ci * kChunk;
-    const int ncols = min(kChunk, kbeg + klen - kc);
-    if (ci + 1 < nchunks) {
-      const int kn = kc + kChunk;
-      load_chunk(s, buf ^ 1, p, m0, kn, min(kChunk, kbeg + klen - kn));
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (one elected lane issues)
+    for (int c = 0; c < nck; ++c) {
+      const int s = c % kStages;
+      const uint32_t ph = (c / kStages) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 11))) break;
+      if (elect_one()) {
+        const uint32_t sb = base + s * kStageBytes;
+        mbar_arrive_expect_tx(full(s), kStageBytes);
+        tma_load_2d(sb, &tmX, kbeg + c * kChunk, m0, full(s));
+        tma_load_2d(sb + kXBytes, &tmL, kbeg + c * kChunk, 0, full(s));
+      }
+      __syncwarp();
     }
-    __syncthreads();
-
-    const uint8_t* xs = reinterpret_cast<const uint8_t*>(s.x[buf]);
-
-    // ---------------------------------------------------------------- quantization
-    if (qh * 64 < ncols) {
-      const float* sm = s.smooth + (kc - kbeg) + qh * 64;
-      uint32_t scw = 0;
-      uint2 cb[4];
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- low-rank MMA (one elected lane issues)
+    constexpr uint32_t kHiSw128 = smem_desc_hi(1024, 2);      // K-major, 128-byte swizzle
+    constexpr uint32_t kLbo = 1u << 16;
+    const uint32_t idesc = idesc_lowrank();
+    for (int c = 0; c < nck; ++c) {
+      const int s = c % kStages;
+      const uint32_t ph = (c / kStages) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 12))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t sb = base + s * kStageBytes;
+        const uint32_t a_lo = (sb >> 4) | kLbo;
+        const uint32_t b_lo = ((sb + kXBytes) >> 4) | kLbo;
 #pragma unroll
-      for (int gq = 0; gq < 4; ++gq) {
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          umma_bf16(tmem, make_desc(a_lo + kk * 2, kHiSw128), make_desc(b_lo + kk * 2, kHiSw128), idesc,
+                    (c | kk) != 0 ? 1u : 0u);
+        tc_commit(empty(s));
+        if (c == nck - 1) tc_commit(acc_full);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ---------------------------------------------------------------- quantizers
+    const int qt = tid - 64;                      // 0..255
+    const int r = qt >> 1;                        // row of the chunk
+    const int h = qt & 1;                         // columns [32 h, 32 h + 32) of the chunk
+    const int m = m0 + r;
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    uint8_t* code_row = p.codes + static_cast<size_t>(m) * (p.K / 2) + kbeg / 2 + h * 16;
+    // scale bytes 2h, 2h + 1 of this row's word in the chunk's 512-byte atom
+    uint8_t* scale_base = p.scales + static_cast<size_t>(m0 / 128) * (p.K / 64) * 512 + (r % 32) * 16 +
+                          (r / 32) * 4 + 2 * h;
+    for (int c = 0; c < nck; ++c) {
+      const int s = c % kStages;
+      const uint32_t ph = (c / kStages) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 13))) break;
+      const uint32_t row = base + s * kStageBytes + r * 128;
+      const float* sm = smooth + c * kChunk + h * 32;
+      uint32_t sc2 = 0;
+      uint2 cb[2];
+#pragma unroll
+      for (int gq = 0; gq < 2; ++gq) {
         float v[16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col = qh * 64 + gq * 16 + h * 8;
-          const uint4 xv = *reinterpret_cast<const uint4*>(xs + swz(qr, col));
-          const float4 s0 = *reinterpret_cast<const float4*>(sm + gq * 16 + h * 8);
-          const float4 s1 = *reinterpret_cast<const float4*>(sm + gq * 16 + h * 8 + 4);
-          v[h * 8 + 0] = bf16lo_to_f32(xv.x) * s0.x;
-          v[h * 8 + 1] = bf16hi_to_f32(xv.x) * s0.y;
-          v[h * 8 + 2] = bf16lo_to_f32(xv.y) * s0.z;
-          v[h * 8 + 3] = bf16hi_to_f32(xv.y) * s0.w;
-          v[h * 8 + 4] = bf16lo_to_f32(xv.z) * s1.x;
-          v[h * 8 + 5] = bf16hi_to_f32(xv.z) * s1.y;
-          v[h * 8 + 6] = bf16lo_to_f32(xv.w) * s1.z;
-          v[h * 8 + 7] = bf16hi_to_f32(xv.w) * s1.w;
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t u = static_cast<uint32_t>(h * 4 + gq * 2 + hh);     // 16-byte unit of the row
+          uint32_t x0, x1, x2, x3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(row + ((u ^ sw) << 4)));
+          const float4 s0 = *reinterpret_cast<const float4*>(sm + gq * 16 + hh * 8);
+          const float4 s1 = *reinterpret_cast<const float4*>(sm + gq * 16 + hh * 8 + 4);
+          v[hh * 8 + 0] = bf16lo_to_f32(x0) * s0.x;
+          v[hh * 8 + 1] = bf16hi_to_f32(x0) * s0.y;
+          v[hh * 8 + 2] = bf16lo_to_f32(x1) * s0.z;
+          v[hh * 8 + 3] = bf16hi_to_f32(x1) * s0.w;
+          v[hh * 8 + 4] = bf16lo_to_f32(x2) * s1.x;
+          v[hh * 8 + 5] = bf16hi_to_f32(x2) * s1.y;
+          v[hh * 8 + 6] = bf16lo_to_f32(x3) * s1.z;
+          v[hh * 8 + 7] = bf16hi_to_f32(x3) * s1.w;
         }
-        scw |= quantize_group(v, p, cb[gq]) << (8 * gq);
+        sc2 |= quantize_group(v, p.g, p.inv_g, cb[gq]) << (8 * gq);
       }
-      const int atom = (kc + qh * 64) / 64;
-      const size_t soff = (static_cast<size_t>(qm / 128) * (p.K / 64) + atom) * 512 + (qm % 32) * 16 +
-                          ((qm % 128) / 32) * 4;
-      *reinterpret_cast<uint32_t*>(p.scales + soff) = scw;      // rows past M get zero scales
-      if (qm < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(qm) * (p.K / 2) + (kc + qh * 64) / 2);
-        dst[0] = make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y);
-        dst[1] = make_uint4(cb[2].x, cb[2].y, cb[3].x, cb[3].y);
-      }
-    }
-
-    // ---------------------------------------------------------------- low-rank down projection
-    {
-      const uint32_t xbase = smem_addr(s.x[buf]);
-      const uint32_t hbase = smem_addr(s.lh[buf]), lbase = smem_addr(s.ll[buf]);
-      const int mi = lane >> 3;
-      const int steps = ncols / 16;
-      for (int st = 0; st < steps; ++st) {
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(xbase + swz(warp * 16 + (lane & 7) + ((mi & 1) << 3), st * 16 + ((mi >> 1) << 3)),
-                    a0, a1, a2, a3);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int n = half * 16 + ((mi >> 1) << 3) + (lane & 7);
-          const int col = st * 16 + ((mi & 1) << 3);
-          uint32_t h00, h01, h10, h11, l00, l01, l10, l11;
-          ldmatrix_x4(hbase + swz(n, col), h00, h01, h10, h11);
-          ldmatrix_x4(lbase + swz(n, col), l00, l01, l10, l11);
-          mma_bf16_16816(acc[half * 2 + 0], a0, a1, a2, a3, h00, h01);
-          mma_bf16_16816(acc[half * 2 + 1], a0, a1, a2, a3, h10, h11);
-          mma_bf16_16816(acc[half * 2 + 0], a0, a1, a2, a3, l00, l01);
-          mma_bf16_16816(acc[half * 2 + 1], a0, a1, a2, a3, l10, l11);
-        }
-      }
-    }
-    __syncthreads();          // buffer `buf` is free again
-  }
-
-  // partial U of this slice -> shared memory (reusing the X buffers)
-  float* upart = reinterpret_cast<float*>(s.x[0]);
-  {
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int col = 8 * j + 2 * q;
-      const int r0 = warp * 16 + g;
-      upart[r0 * kRank + col] = acc[j][0];
-      upart[r0 * kRank + col + 1] = acc[j][1];
-      upart[(r0 + 8) * kRank + col] = acc[j][2];
-      upart[(r0 + 8) * kRank + col + 1] = acc[j][3];
+      // the tile has been read: release it to the producer (with the MMA's commit)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(s));
+      *reinterpret_cast<uint16_t*>(scale_base + static_cast<size_t>((kbeg / 64) + c) * 512) =
+          static_cast<uint16_t>(sc2);            // rows past M get zero scales
+      if (m < p.M)
+        *reinterpret_cast<uint4*>(code_row + c * 32) = make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y);
     }
   }
 
-  // sum the slices' partials across the cluster; CTA `rank` finishes rows [rank*rpc, (rank+1)*rpc)
-  const int ks = p.kslices;
-  if (ks > 1) cluster_sync_all(); else __syncthreads();
-  const uint32_t rank = ks > 1 ? cluster_ctarank() : 0u;
-  const int rpc = kRows / ks;
-  for (int i = tid; i < rpc * kRank; i += kThreads) {
-    const int r = static_cast<int>(rank) * rpc + i / kRank;
-    const int c = i % kRank;
-    float sum = 0.f;
-    if (ks > 1) {
-      for (int src = 0; src < ks; ++src) sum += ld_dsmem_f32(&upart[r * kRank + c], static_cast<uint32_t>(src));
+  // ---------------------------------------------------------------- U = hi + lo, summed over the cluster
+  __syncthreads();                                 // every stage has been consumed: reuse them for U
+  float* upart = reinterpret_cast<float*>(gbase); // [128][32] fp32, 16-byte pieces rotated by the row
+  if (warp >= 2 && warp < 6) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    float u[32];
+    if (__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full, 0, abort_flag, 14))) {
+      tc_fence_after();
+      uint32_t hi[32], lo[32];
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16), hi);
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 32u, lo);
+      tmem_wait_ld_regs(hi);
+      tmem_wait_ld_regs(lo);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) u[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
     } else {
-      sum = upart[r * kRank + c];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) u[j] = 0.f;
     }
-    const int m = m0 + r;
-    if (m < p.M) {
-      const float u = sum * p.inv_g;                   // exact: a power of two
-      const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
-      p.ucat[static_cast<size_t>(m) * (2 * kRank) + c] = hi;
-      p.ucat[static_cast<size_t>(m) * (2 * kRank) + kRank + c] = lo;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(upart + row * 32 + ((j + row) & 7) * 4) =
+          make_float4(u[j * 4], u[j * 4 + 1], u[j * 4 + 2], u[j * 4 + 3]);
+  }
+  const int ks = p.kslices;
+  tc_fence_before();
+  cluster_sync_all();                              // partials of every slice in shared memory
+  const uint32_t crank = cluster_ctarank();
+  const int rpc = kRows / ks;                      // rows finished by this CTA
+  for (int i = tid; i < rpc * kRank; i += kThreads) {
+    const int rr = static_cast<int>(crank) * rpc + i / kRank;
+    const int col = i % kRank;
+    const float* src_addr = upart + rr * 32 + (((col >> 2) + rr) & 7) * 4 + (col & 3);
+    float sum = 0.f;
+    for (int src = 0; src < ks; ++src) sum += ld_dsmem_f32(src_addr, static_cast<uint32_t>(src));
+    const int mm = m0 + rr;
+    if (mm < p.M) {
+      const float uu = sum * p.inv_g;             // exact: a power of two
+      const __nv_bfloat16 hb = __float2bfloat16_rn(uu);
+      const __nv_bfloat16 lb = __float2bfloat16_rn(uu - __bfloat162float(hb));
+      p.ucat[static_cast<size_t>(mm) * (2 * kRank) + col] = hb;
+      p.ucat[static_cast<size_t>(mm) * (2 * kRank) + kRank + col] = lb;
     }
   }
-  if (ks > 1) cluster_sync_all();   // keep this CTA's shared memory alive until the others have read it
+  if (*abort_flag) {
+    // a wait ran out: let the MMAs and copies already issued finish before the memory goes away
+    if (warp == 1) {
+      if (elect_one()) tc_commit(drain);
+      __syncwarp();
+      mbar_wait_bounded(drain, 0, nullptr, 15);
+    }
+    if (warp == 0 && lane == 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 2000000ull) { }
+    }
+  }
+  cluster_sync_all();                              // the other CTAs are done reading this CTA's partials
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<kTmemCols>(tmem);
+  }
 }
 
 }  // namespace k1
