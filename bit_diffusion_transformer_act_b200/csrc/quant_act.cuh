@@ -40,7 +40,12 @@
 // either exactly a midpoint -- and then the corrected value is that midpoint
 // exactly -- or at least 2^-16 (relative) away from one, far beyond the
 // few-ulp error of q.  cvt.rn.satfinite.e2m1x2 then rounds to nearest even.
-// The sign of q is copied from x_hat so that negative zero keeps its sign.
+// The quantizers hold -x_hat (the smoothing factors are stored negated) and
+// form the residual as e' = q0 D - x_hat and the quotient as q0 - e' r; the
+// values are those of the textbook form, and a zero x_hat keeps its sign in q
+// (for x_hat = -0: q0 = -0, e' = +0, q = -0 + -0 = -0).  Pairs of values go
+// through the packed fp32x2 multiply and fma of sm_100, each half rounded to
+// nearest as its scalar counterpart.
 #pragma once
 
 #include "ptx.cuh"
@@ -87,14 +92,6 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// Quotient x / D for the E2M1 decision (see the rounding note above); r ~ 1/D.
-__device__ __forceinline__ float quotient(float x, float D, float r) {
-  const float q0 = x * r;
-  const float e = fmaf(-q0, D, x);
-  const float q = fmaf(e, r, q0);
-  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
-}
-
 // RN(a / 6) for a >= 0 (Markstein correction of a * RN(1/6)).
 __device__ __forceinline__ float div6(float a) {
   const float y = 0.16666667163372039794921875f;      // RN(1/6) in binary32
@@ -103,11 +100,15 @@ __device__ __forceinline__ float div6(float a) {
   return fmaf(e, y, q0);
 }
 
-// Quantizes 16 smoothed values (one group): returns the E4M3 scale code, writes 8 code bytes.
-__device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], float g, float inv_g, uint2& out) {
+// Quantizes one group of 16 smoothed values given as 8 pairs of -x_hat (see the
+// rounding note above): returns the E4M3 scale code and writes 8 code bytes.
+__device__ __forceinline__ uint32_t quantize_group(const uint64_t (&nx)[8], float g, float inv_g, uint2& out) {
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f32x2_unpack(nx[i], a[2 * i], a[2 * i + 1]);
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  for (int i = 0; i < 16; i += 2) amax = fmax3(amax, fabsf(a[i]), fabsf(a[i + 1]));
   const uint32_t sc = cvt_e4m3x2(div6(amax) * inv_g, 0.f) & 0xFFu;
   float S, unused;
   e4m3x2_to_f32(sc, S, unused);
@@ -116,11 +117,17 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&v)[16], float g
     out = make_uint2(0u, 0u);
     return 0u;
   }
-  const float r = rcp_approx(D);
-  out.x = cvt_e2m1x8(quotient(v[0], D, r), quotient(v[1], D, r), quotient(v[2], D, r), quotient(v[3], D, r),
-                     quotient(v[4], D, r), quotient(v[5], D, r), quotient(v[6], D, r), quotient(v[7], D, r));
-  out.y = cvt_e2m1x8(quotient(v[8], D, r), quotient(v[9], D, r), quotient(v[10], D, r), quotient(v[11], D, r),
-                     quotient(v[12], D, r), quotient(v[13], D, r), quotient(v[14], D, r), quotient(v[15], D, r));
+  const float rn = -rcp_approx(D);
+  const uint64_t rn2 = f32x2_pack(rn, rn), D2 = f32x2_pack(D, D);
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint64_t q0 = f32x2_mul(nx[i], rn2);            // x_hat r
+    const uint64_t e = f32x2_fma(q0, D2, nx[i]);          // q0 D - x_hat, exact
+    f32x2_unpack(f32x2_fma(e, rn2, q0), q[2 * i], q[2 * i + 1]);   // q0 - e r
+  }
+  out.x = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out.y = cvt_e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
   return sc;
 }
 
@@ -144,7 +151,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   const uint32_t drain = bars + 8u * (2 * kStages + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
-  float* smooth = reinterpret_cast<float*>(gbase + kOffSmooth);
+  float* smooth = reinterpret_cast<float*>(gbase + kOffSmooth);   // -smooth_inv of this K slice
 
   const int tid = threadIdx.x;
   const int warp = tid / 32;
@@ -166,7 +173,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   if (warp == 1) tmem_alloc<kTmemCols>(smem_addr(tmem_slot));
   grid_dependency_wait();                          // X and the outputs may belong to the previous kernel
   grid_launch_dependents();
-  for (int i = tid; i < klen; i += kThreads) smooth[i] = __bfloat162float(p.smooth[kbeg + i]);
+  for (int i = tid; i < klen; i += kThreads) smooth[i] = -__bfloat162float(p.smooth[kbeg + i]);   // negated
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -230,25 +237,21 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
       uint2 cb[2];
 #pragma unroll
       for (int gq = 0; gq < 2; ++gq) {
-        float v[16];
+        uint64_t nx[8];                            // -x_hat, in pairs
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const uint32_t u = static_cast<uint32_t>(h * 4 + gq * 2 + hh);     // 16-byte unit of the row
-          uint32_t x0, x1, x2, x3;
+          uint32_t xw[4];
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(row + ((u ^ sw) << 4)));
-          const float4 s0 = *reinterpret_cast<const float4*>(sm + gq * 16 + hh * 8);
-          const float4 s1 = *reinterpret_cast<const float4*>(sm + gq * 16 + hh * 8 + 4);
-          v[hh * 8 + 0] = bf16lo_to_f32(x0) * s0.x;
-          v[hh * 8 + 1] = bf16hi_to_f32(x0) * s0.y;
-          v[hh * 8 + 2] = bf16lo_to_f32(x1) * s0.z;
-          v[hh * 8 + 3] = bf16hi_to_f32(x1) * s0.w;
-          v[hh * 8 + 4] = bf16lo_to_f32(x2) * s1.x;
-          v[hh * 8 + 5] = bf16hi_to_f32(x2) * s1.y;
-          v[hh * 8 + 6] = bf16lo_to_f32(x3) * s1.z;
-          v[hh * 8 + 7] = bf16hi_to_f32(x3) * s1.w;
+                       : "=r"(xw[0]), "=r"(xw[1]), "=r"(xw[2]), "=r"(xw[3]) : "r"(row + ((u ^ sw) << 4)));
+          const ulonglong2 s01 = *reinterpret_cast<const ulonglong2*>(sm + gq * 16 + hh * 8);
+          const ulonglong2 s23 = *reinterpret_cast<const ulonglong2*>(sm + gq * 16 + hh * 8 + 4);
+          const uint64_t sp[4] = {s01.x, s01.y, s23.x, s23.y};
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            nx[hh * 4 + w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(xw[w]), bf16hi_to_f32(xw[w])), sp[w]);
         }
-        sc2 |= quantize_group(v, p.g, p.inv_g, cb[gq]) << (8 * gq);
+        sc2 |= quantize_group(nx, p.g, p.inv_g, cb[gq]) << (8 * gq);
       }
       // the tile has been read: release it to the producer (with the MMA's commit)
       __syncwarp();
@@ -290,19 +293,32 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   cluster_sync_all();                              // partials of every slice in shared memory
   const uint32_t crank = cluster_ctarank();
   const int rpc = kRows / ks;                      // rows finished by this CTA
-  for (int i = tid; i < rpc * kRank; i += kThreads) {
-    const int rr = static_cast<int>(crank) * rpc + i / kRank;
-    const int col = i % kRank;
-    const float* src_addr = upart + rr * 32 + (((col >> 2) + rr) & 7) * 4 + (col & 3);
-    float sum = 0.f;
-    for (int src = 0; src < ks; ++src) sum += ld_dsmem_f32(src_addr, static_cast<uint32_t>(src));
+  for (int i = tid; i < rpc * 8; i += kThreads) {  // one 4-column piece of one row per thread
+    const int rr = static_cast<int>(crank) * rpc + i / 8;
+    const int piece = i % 8;
+    const float* src_addr = upart + rr * 32 + ((piece + rr) & 7) * 4;
+    float4 v[8];
+#pragma unroll
+    for (int src = 0; src < 8; ++src)             // all loads in flight before the sum
+      if (src < ks) v[src] = ld_dsmem_f32x4(src_addr, static_cast<uint32_t>(src));
+    float4 sum = v[0];
+#pragma unroll
+    for (int src = 1; src < 8; ++src)
+      if (src < ks) { sum.x += v[src].x; sum.y += v[src].y; sum.z += v[src].z; sum.w += v[src].w; }
     const int mm = m0 + rr;
     if (mm < p.M) {
-      const float uu = sum * p.inv_g;             // exact: a power of two
-      const __nv_bfloat16 hb = __float2bfloat16_rn(uu);
-      const __nv_bfloat16 lb = __float2bfloat16_rn(uu - __bfloat162float(hb));
-      p.ucat[static_cast<size_t>(mm) * (2 * kRank) + col] = hb;
-      p.ucat[static_cast<size_t>(mm) * (2 * kRank) + kRank + col] = lb;
+      const float uu[4] = {sum.x * p.inv_g, sum.y * p.inv_g, sum.z * p.inv_g, sum.w * p.inv_g};  // exact
+      uint32_t hw[2], lw[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float h0 = __bfloat162float(__float2bfloat16_rn(uu[2 * j]));
+        const float h1 = __bfloat162float(__float2bfloat16_rn(uu[2 * j + 1]));
+        hw[j] = pack_bf16x2(h0, h1);
+        lw[j] = pack_bf16x2(uu[2 * j] - h0, uu[2 * j + 1] - h1);
+      }
+      __nv_bfloat16* dst = p.ucat + static_cast<size_t>(mm) * (2 * kRank) + piece * 4;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(hw[0], hw[1]);
+      *reinterpret_cast<uint2*>(dst + kRank) = make_uint2(lw[0], lw[1]);
     }
   }
   if (*abort_flag) {
