@@ -1,7 +1,7 @@
 // Byte layouts shared by the host packer and the CUDA launchers.
 //
 // Packed weight blob (device-private; produced on the host by svdq_pack_weights):
-//   [0, 256)     header: "SVDQNVF4", abi version, N, K, rank, g_w
+//   [0, 1024)    header: "SVDQNVF4", abi version, N, K, rank, g_w (zero padded)
 //   l1s          bf16 [2][rank][K] (diag(smooth_inv) L1)^T split exactly into a
 //                                 high and a low bf16 part (K contiguous) -- read
 //                                 by the activation kernel, which knows K but not

@@ -114,8 +114,8 @@ int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
 size_t svdq_act_scale_bytes(int M, int K);
 
 /* Kernel 1: smoothing, NVFP4 quantization and the rank-32 down-projection, in
- * one pass over X (the article's "16-bit low-rank branch" is fed from the same
- * smoothed values that are quantized).
+ * one pass over X (the low-rank branch, kept in 16-bit precision, is fed from
+ * the same smoothed values that are quantized).
  *   X           device bf16 [M, K] (16-byte aligned rows: K % 64 == 0)
  *   smooth_inv  device bf16 [K], the per-channel 1/lambda
  *   packed_w    device copy of the blob from svdq_pack_weights (its L1 is used;
