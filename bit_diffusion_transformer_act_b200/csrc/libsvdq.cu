@@ -268,8 +268,6 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
 
   namespace k3 = svdq::k3;
   k3::Params p;
-  p.X = static_cast<const __nv_bfloat16*>(X);
-  p.qw = static_cast<const uint8_t*>(qweight);
   p.scales = static_cast<const __nv_bfloat16*>(scales);
   p.zeros = static_cast<const __nv_bfloat16*>(zeros);
   p.bias = static_cast<const __nv_bfloat16*>(bias);
@@ -277,19 +275,38 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   p.M = M;
   p.N = N;
   p.K = K;
-  const dim3 grid(N / k3::kRows, 1, 1);
+  const int nt = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));   // 8-token MMA tiles
+  CUtensorMap tW, tX;
+  if (!make_tmap(&tW, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, k3::kRows,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, 8 * nt, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  const dim3 grid((N + k3::kRows - 1) / k3::kRows, 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-#define SVDQ_AWQ_LAUNCH(NT_)                                                              \
-  do {                                                                                    \
-    const int smem = static_cast<int>(sizeof(k3::Smem<NT_>));                             \
-    if (!set_smem_once<k3::awq_gemm_kernel<NT_>>(smem, dev)) return SVDQ_ERR_CUDA;        \
-    k3::awq_gemm_kernel<NT_><<<grid, k3::kThreads, smem, s>>>(p);                          \
+#define SVDQ_AWQ_LAUNCH(NT_)                                                                    \
+  do {                                                                                          \
+    const int smem = k3::Cfg<NT_>::SMEM;                                                        \
+    if (!set_smem_once<k3::awq_gemm_kernel<NT_>>(smem, dev)) return SVDQ_ERR_CUDA;              \
+    cudaLaunchConfig_t cfg = {};                                                                \
+    cfg.gridDim = grid;                                                                         \
+    cfg.blockDim = dim3(k3::kThreads, 1, 1);                                                    \
+    cfg.dynamicSmemBytes = smem;                                                                \
+    cfg.stream = s;                                                                             \
+    cudaLaunchAttribute attr[1];                                                                \
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;                            \
+    attr[0].val.programmaticStreamSerializationAllowed = 1;                                     \
+    cfg.attrs = attr;                                                                           \
+    cfg.numAttrs = 1;                                                                           \
+    if (cudaLaunchKernelEx(&cfg, k3::awq_gemm_kernel<NT_>, tW, tX, p) != cudaSuccess) {         \
+      (void)cudaGetLastError();                                                                 \
+      return SVDQ_ERR_CUDA;                                                                     \
+    }                                                                                           \
   } while (0)
 
-  if (M <= 8) SVDQ_AWQ_LAUNCH(1);
-  else if (M <= 16) SVDQ_AWQ_LAUNCH(2);
-  else if (M <= 32) SVDQ_AWQ_LAUNCH(4);
+  if (nt == 1) SVDQ_AWQ_LAUNCH(1);
+  else if (nt == 2) SVDQ_AWQ_LAUNCH(2);
+  else if (nt == 4) SVDQ_AWQ_LAUNCH(4);
   else SVDQ_AWQ_LAUNCH(8);
 #undef SVDQ_AWQ_LAUNCH
   return launch_status();
