@@ -222,6 +222,13 @@ class Workload:
         P.awq_w4a16_linear(s["X"][m], s["qw"], s["s"], s["z"], None, s["Y"][m])
 
 
+# DRAM bytes (read + write) of one nvfp4_gemm_kernel<256> launch at the attention shape,
+# from the ncu capture summarised in profiles/nvfp4_gemm_attention_4096x3072x3072.md
+# (13.15 MB read = the algorithmic input bytes; the bf16 output stays in L2 within the
+# launch).  Must be re-measured whenever the GEMM kernel changes.
+GEMM_DRAM_BYTES_PER_LAUNCH = 13151488
+
+
 def svdq_flops():
     M, K, N = SVDQ_SHAPE
     return 2.0 * M * N * K
@@ -372,7 +379,9 @@ def run_ours(args, world, rank, local):
         "svdq_ms_per_step": svdq_ms_max / args.steps,
         "roofline": {
             "bound": "tensor", "achieved": k2_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-            "frac": k2_tflops / fp4_peak, "traffic": None,
+            "frac": k2_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
+            "traffic_unit": "bytes per launch (dram read + write, ncu, cold caches)",
+            "traffic_source": "profiles/nvfp4_gemm_attention_4096x3072x3072.md",
             "kernel": "nvfp4_gemm_kernel<256>",
             "peak_note": "dense FP4 = 4 x measured bf16 burst (%s), nominal 9/2.25 ratio" % peaks["source"],
         },
