@@ -222,10 +222,10 @@ class Workload:
         P.awq_w4a16_linear(s["X"][m], s["qw"], s["s"], s["z"], None, s["Y"][m])
 
 
-# DRAM bytes (read + write) of one nvfp4_gemm_kernel<256> launch at the attention shape,
-# from the ncu capture summarised in profiles/nvfp4_gemm_attention_4096x3072x3072.md
-# (13.15 MB read = the algorithmic input bytes; the bf16 output stays in L2 within the
-# launch).  Must be re-measured whenever the GEMM kernel changes.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one nvfp4_gemm_kernel<256>
+# launch at the attention shape, from an ncu capture with cold caches (13.15 MB read = the
+# algorithmic input bytes; the bf16 output stays in L2 within the launch).  Must be
+# re-measured whenever the GEMM kernel changes.
 GEMM_DRAM_BYTES_PER_LAUNCH = 13151488
 
 
