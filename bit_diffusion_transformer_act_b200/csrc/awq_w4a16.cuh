@@ -228,7 +228,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty(s));       // this warp is done with the stage
+      if (lane == 0) mbar_arrive_relaxed(empty(s));   // this warp is done with the stage
     }
 
     const int ra = n0 + rg, rb = ra + 8;

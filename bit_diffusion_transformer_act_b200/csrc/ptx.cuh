@@ -64,6 +64,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(bar) : "memory");
 }
 
+// Arrival without release semantics: for a consumer handing a stage back once every
+// value it read from the stage is in registers -- it does not wait for the thread's
+// earlier global loads or stores, as a release arrival would.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }"
                ::"r"(bar), "r"(bytes) : "memory");

@@ -173,11 +173,15 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   if (warp == 1) tmem_alloc<kTmemCols>(smem_addr(tmem_slot));
   grid_dependency_wait();                          // X and the outputs may belong to the previous kernel
   grid_launch_dependents();
-  for (int i = tid; i < klen; i += kThreads) smooth[i] = -__bfloat162float(p.smooth[kbeg + i]);   // negated
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp >= 2) {
+    // the quantizers fetch the smoothing factors while the first tiles are in flight
+    for (int i = tid - 64; i < klen; i += kThreads - 64) smooth[i] = -__bfloat162float(p.smooth[kbeg + i]);
+    asm volatile("bar.sync 1, %0;" ::"n"(kQuantWarps * 32) : "memory");   // quantizer warps only
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (one elected lane issues)
@@ -255,7 +259,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
       }
       // the tile has been read: release it to the producer (with the MMA's commit)
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty(s));
+      if (lane == 0) mbar_arrive_relaxed(empty(s));
       *reinterpret_cast<uint16_t*>(scale_base + static_cast<size_t>((kbeg / 64) + c) * 512) =
           static_cast<uint16_t>(sc2);            // rows past M get zero scales
       if (m < p.M)
