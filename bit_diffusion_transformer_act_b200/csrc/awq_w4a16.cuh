@@ -13,22 +13,23 @@
 // (128-byte swizzle) and the tokens' activations as four 64-column sub-tiles
 // (128-byte swizzle, rows past M read as zeros), into a deep ring of stages (the
 // activations are shared by every CTA and come from L2).  Warps 0-7 own 16
-// weight rows each; per stage they wait on the stage's barrier, and release it
-// with one arrival per warp -- no block-wide barrier.  The weights are the A
-// operand of mma.sync m16n8k16 (16 weight rows x 8 tokens), dequantized in
-// registers: a nibble q becomes the bf16 128 + q by bit placement (exact).
-// Inside every 32-K step the K order is permuted (the same permutation for A and
-// B): lane quad position p takes real K elements 8p..8p+7, i.e. one 32-bit word
-// of nibbles per weight row and one 16-byte load of activations per token tile.
-// The zero point:
-//   * M <= 8: sum_k (128 + q) x is accumulated as is and corrected per group,
-//       s (sum (128 + q) x - (128 + z) sum x); sum x comes from a second MMA with
-//       an all-ones A operand on the same activation fragment, so no per-weight
-//       subtraction is needed.
-//   * M > 8: one packed bf16 subtraction of 128 + z gives q - z exactly.
-// Either way every product is exact and each group's fp32 partial sum is scaled
-// by s once.  Scales and zeros are read from global memory one stage ahead.
-// Every mbarrier wait is bounded.
+// weight rows each and release a stage with one relaxed arrival per warp -- no
+// block-wide barrier in the loop.  The weights are the A operand of mma.sync
+// m16n8k16 (16 weight rows x 8 tokens), dequantized in registers: a nibble q
+// becomes the bf16 128 + q by bit placement (exact).  A lane's 32-bit word of
+// nibbles (one ldmatrix fetches the four words of a group) covers real K elements
+// 8p..8p+7 of a 32-K step (p = lane % 4); the MMA's K slots are a permutation of
+// them, the same for A and B.
+//   * M <= 8: warp 9 prepares each stage before the consumers see it: it reorders
+//     every 8-element activation unit to (k0,k4) (k1,k5) (k2,k6) (k3,k7), so that a
+//     pair of nibbles (p, p + 4) of a word becomes a bf16x2 operand with one shift
+//     and one logic operation, and it sums each token's 64 activations of each group.
+//     The zero point then enters once per group: s (sum (128 + q) x - (128 + z) sum x).
+//   * M > 8: pairs (2b, 2b + 1) through a byte permute, and one packed bf16
+//     subtraction of 128 + z gives q - z exactly.
+// Either way every product is exact and each group's fp32 partial sum is scaled by
+// s once.  Scales and zeros are read from global memory two stages ahead.  Every
+// mbarrier wait is bounded.
 #pragma once
 
 #include "ptx.cuh"
@@ -38,18 +39,20 @@ namespace k3 {
 
 constexpr int kRows = 128;                 // output rows (weight rows) per CTA
 constexpr int kComputeWarps = 8;           // 16 weight rows each
-constexpr int kThreads = (kComputeWarps + 1) * 32;
 constexpr int kChunk = 256;                // K per stage
 constexpr int kGroup = 64;
 constexpr int kWBytes = kRows * 128;       // 16 KB of packed weights per stage
 
 template <int NT>
 struct Cfg {
+  static constexpr bool PREP = NT == 1;                     // activation reorder + group sums (warp 9)
+  static constexpr int THREADS = (kComputeWarps + (PREP ? 2 : 1)) * 32;
   static constexpr int XSUB = NT * 8 * 128;                 // one 64-column activation sub-tile
-  static constexpr int STAGE = kWBytes + 4 * XSUB;
-  static constexpr int STAGES = NT == 1 ? 10 : (NT == 2 ? 8 : (NT == 4 ? 6 : 4));
+  static constexpr int OFF_SX = kWBytes + 4 * XSUB;         // group sums: [4 groups][NT * 8 tokens] fp32
+  static constexpr int STAGE = (OFF_SX + (PREP ? 4 * NT * 8 * 4 : 0) + 1023) / 1024 * 1024;
+  static constexpr int STAGES = NT == 1 ? 9 : (NT == 2 ? 7 : (NT == 4 ? 6 : 4));
   static constexpr int OFF_BAR = STAGES * STAGE;
-  static constexpr int SMEM = OFF_BAR + 8 * 2 * STAGES + 16 + 1024;
+  static constexpr int SMEM = OFF_BAR + 8 * 3 * STAGES + 16 + 1024;
   static_assert(STAGE % 1024 == 0, "1 KB alignment of swizzled tiles");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -70,17 +73,36 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t w4, uint32_t s
   return (r & 0x000F000Fu) | 0x43004300u;
 }
 
+// bf16x2 {128 + nibble 0 of v, 128 + nibble 4 of v}
+__device__ __forceinline__ uint32_t nib04(uint32_t v) { return (v & 0x000F000Fu) | 0x43004300u; }
+
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// D (16x8 fp32) = A (16x16 bf16, row) x B (16x8 bf16, col) + D, or + 0.  Not volatile:
+// pure functions of their registers, so independent MMAs and loads may be interleaved.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_zero_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<NT>::THREADS, 1)
 awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
   using C = Cfg<NT>;
   constexpr int S = C::STAGES;
-  constexpr bool kSumX = NT == 1;                  // zero point through sum x (see above)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -88,14 +110,20 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   const uint32_t bars = base + C::OFF_BAR;
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 16 * S);
+  auto ready = [&](int s) { return bars + 8u * (2 * S + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 24 * S);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n0 = blockIdx.x * kRows;
   const int nkb = p.K / kChunk;
+  constexpr int kProducer = kComputeWarps, kPrepWarp = kComputeWarps + 1;
 
-  if (warp == kComputeWarps && lane == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), kComputeWarps); }
+  if (warp == kProducer && lane == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), kComputeWarps);
+      mbar_init(ready(s), 32);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmW);
@@ -105,7 +133,13 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
 
-  if (warp == kComputeWarps) {
+  float tot[NT][4];                                // consumers: this lane's sums (D fragment layout)
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) tot[j][t] = 0.f;
+
+  if (warp == kProducer) {
     // ---------------------------------------------------------------- TMA producer
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % S;
@@ -113,112 +147,147 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 21))) break;
       if (elect_one()) {
         const uint32_t sb = base + s * C::STAGE;
-        mbar_arrive_expect_tx(full(s), C::STAGE);
+        mbar_arrive_expect_tx(full(s), kWBytes + 4 * C::XSUB);
         tma_load_2d(sb, &tmW, kb * (kChunk / 2), n0, full(s));
 #pragma unroll
         for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * C::XSUB, &tmX, kb * kChunk + j * 64, 0, full(s));
       }
       __syncwarp();
     }
+  } else if (warp == kPrepWarp) {
+    if constexpr (C::PREP) {
+      // ---------------------------------------------------------------- activation reorder + group sums
+      // lane -> (token, group) items: token = item % (NT * 8), group = item / (NT * 8)
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1u;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 23))) break;
+        uint8_t* st = gbase + s * C::STAGE;
+#pragma unroll
+        for (int it = 0; it < NT; ++it) {
+          const int item = lane + 32 * it;
+          const int tok = item % (NT * 8), grp = item / (NT * 8);
+          uint8_t* row = st + kWBytes + grp * C::XSUB + tok * 128;
+          float sum = 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            uint4* up = reinterpret_cast<uint4*>(row + ((u ^ (tok & 7)) << 4));
+            const uint4 v = *up;
+            const float a0 = bf16lo_to_f32(v.x) + bf16hi_to_f32(v.x), a1 = bf16lo_to_f32(v.y) + bf16hi_to_f32(v.y);
+            const float a2 = bf16lo_to_f32(v.z) + bf16hi_to_f32(v.z), a3 = bf16lo_to_f32(v.w) + bf16hi_to_f32(v.w);
+            sum += (a0 + a1) + (a2 + a3);
+            uint4 n;
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.x) : "r"(v.x), "r"(v.z));   // (k0, k4)
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.y) : "r"(v.x), "r"(v.z));   // (k1, k5)
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.z) : "r"(v.y), "r"(v.w));   // (k2, k6)
+            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.w) : "r"(v.y), "r"(v.w));   // (k3, k7)
+            *up = n;
+          }
+          reinterpret_cast<float*>(st + C::OFF_SX)[grp * (NT * 8) + tok] = sum;
+        }
+        fence_proxy_async_smem();                  // the next TMA into this stage comes after these stores
+        mbar_arrive(ready(s));                     // release: this lane's stores are visible to the consumers
+      }
+    }
   } else {
     // ---------------------------------------------------------------- dequantize + mma.sync
     const int g = lane >> 2, q = lane & 3;
     const int rg = warp * 16 + g;                  // this lane's weight rows: rg and rg + 8
-    const uint32_t sw = static_cast<uint32_t>(rg & 7);   // (rg + 8) & 7 is the same
     const int gpr = p.K / kGroup;                  // groups per weight row
     const int na = min(n0 + rg, p.N - 1), nb = min(n0 + rg + 8, p.N - 1);   // clamped for the loads
     const uint2* sa = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(na) * gpr);
     const uint2* sb_ = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(nb) * gpr);
     const uint2* za = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(na) * gpr);
     const uint2* zb = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(nb) * gpr);
-    constexpr uint32_t kOnes = 0x3F803F80u;        // bf16x2 {1, 1}
-
-    float tot[NT][4];
+    // ldmatrix: this lane's row address (matrices: rows 0-7 / 8-15 of the slice, 32-K steps 2 grp / 2 grp + 1)
+    const int lrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    uint32_t woff[4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int t = 0; t < 4; ++t) tot[j][t] = 0.f;
+    for (int grp = 0; grp < 4; ++grp)
+      woff[grp] = static_cast<uint32_t>(lrow * 128) +
+                  ((static_cast<uint32_t>(2 * grp + (lane >> 4)) ^ static_cast<uint32_t>(lane & 7)) << 4);
+    // activation unit of this lane in a sub-tile (token row g of each 8-token tile), per 32-K step
+    const uint32_t xoff0 = static_cast<uint32_t>(g * 128) + ((static_cast<uint32_t>(q) ^ static_cast<uint32_t>(g)) << 4);
+    const uint32_t xoff1 = static_cast<uint32_t>(g * 128) + ((static_cast<uint32_t>(4 + q) ^ static_cast<uint32_t>(g)) << 4);
 
-    // scales and zeros of the 4 groups of a stage: 8 bytes per row, one stage ahead
-    uint2 s_a = __ldg(sa), s_b = __ldg(sb_), z_a = __ldg(za), z_b = __ldg(zb);
+    // scales and zeros of the 4 groups of a stage (8 bytes per row), two stages ahead
+    uint2 pa[4], pb[4];
+    {
+      const int k1 = min(1, nkb - 1);
+      pa[0] = __ldg(sa); pa[1] = __ldg(sb_); pa[2] = __ldg(za); pa[3] = __ldg(zb);
+      pb[0] = __ldg(sa + k1); pb[1] = __ldg(sb_ + k1); pb[2] = __ldg(za + k1); pb[3] = __ldg(zb + k1);
+    }
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % S;
       const uint32_t ph = (kb / S) & 1u;
-      const uint2 cs_a = s_a, cs_b = s_b, cz_a = z_a, cz_b = z_b;
-      if (kb + 1 < nkb) {
-        s_a = __ldg(sa + kb + 1); s_b = __ldg(sb_ + kb + 1);
-        z_a = __ldg(za + kb + 1); z_b = __ldg(zb + kb + 1);
+      const uint2 cur[4] = {pa[0], pa[1], pa[2], pa[3]};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) pa[t] = pb[t];
+      {
+        const int kk = min(kb + 2, nkb - 1);
+        pb[0] = __ldg(sa + kk); pb[1] = __ldg(sb_ + kk); pb[2] = __ldg(za + kk); pb[3] = __ldg(zb + kk);
       }
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 22))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(C::PREP ? ready(s) : full(s), ph, abort_flag, 22))) break;
       const uint32_t wst = base + s * C::STAGE;
-      const uint32_t xst = wst + kWBytes;
-      const uint32_t wrow_g = wst + rg * 128 + 4 * q;
-      const uint32_t wrow_h = wrow_g + 8 * 128;
+      const float* sxs = reinterpret_cast<const float*>(gbase + s * C::STAGE + C::OFF_SX);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
-        const uint32_t sw2a = grp < 2 ? cs_a.x : cs_a.y, sw2b = grp < 2 ? cs_b.x : cs_b.y;
-        const uint32_t zw2a = grp < 2 ? cz_a.x : cz_a.y, zw2b = grp < 2 ? cz_b.x : cz_b.y;
-        const float sg = (grp & 1) ? bf16hi_to_f32(sw2a) : bf16lo_to_f32(sw2a);
-        const float sh = (grp & 1) ? bf16hi_to_f32(sw2b) : bf16lo_to_f32(sw2b);
-        const float zg = ((grp & 1) ? bf16hi_to_f32(zw2a) : bf16lo_to_f32(zw2a)) + 128.f;
-        const float zh = ((grp & 1) ? bf16hi_to_f32(zw2b) : bf16lo_to_f32(zw2b)) + 128.f;
+        const uint32_t w0 = grp < 2 ? cur[0].x : cur[0].y, w1 = grp < 2 ? cur[1].x : cur[1].y;
+        const uint32_t w2 = grp < 2 ? cur[2].x : cur[2].y, w3 = grp < 2 ? cur[3].x : cur[3].y;
+        const float sg = (grp & 1) ? bf16hi_to_f32(w0) : bf16lo_to_f32(w0);
+        const float sh = (grp & 1) ? bf16hi_to_f32(w1) : bf16lo_to_f32(w1);
+        const float zg = ((grp & 1) ? bf16hi_to_f32(w2) : bf16lo_to_f32(w2)) + 128.f;
+        const float zh = ((grp & 1) ? bf16hi_to_f32(w3) : bf16lo_to_f32(w3)) + 128.f;
 
+        uint32_t wq[4];                            // {row g, row g+8} x {32-K step 0, 1}
+        ldmatrix_x4(wst + woff[grp], wq[0], wq[1], wq[2], wq[3]);
+        const uint32_t xsub = wst + kWBytes + grp * C::XSUB;
         float ga[NT][4];
-        float sx[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int t = 0; t < 4; ++t) ga[j][t] = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const uint32_t t32 = static_cast<uint32_t>(grp * 2 + half);   // 32-K step: 16-byte unit of a row
-          uint32_t wg, wh;
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(wg) : "r"(wrow_g + ((t32 ^ sw) << 4)));
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(wh) : "r"(wrow_h + ((t32 ^ sw) << 4)));
-          const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
-          // pair b (real K elements 8q + 2b, 8q + 2b + 1) = byte b of w (low and high nibble)
+          const uint32_t wg = wq[2 * half], wh = wq[2 * half + 1];
           uint32_t A[2][4];
+          if constexpr (C::PREP) {
+            // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
+            const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
+            A[0][0] = nib04(wg);       A[0][1] = nib04(wh);
+            A[0][2] = nib04(wg4);      A[0][3] = nib04(wh4);
+            A[1][0] = nib04(wg >> 8);  A[1][1] = nib04(wh >> 8);
+            A[1][2] = nib04(wg4 >> 8); A[1][3] = nib04(wh4 >> 8);
+          } else {
+            // pair b (real K elements 8q + 2b, 8q + 2b + 1) = byte b of w (low and high nibble)
+            const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
+            const uint32_t zzg = pack_bf16x2(zg, zg), zzh = pack_bf16x2(zh, zh);
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint32_t sel0 = static_cast<uint32_t>(2 * ks) | (static_cast<uint32_t>(4 + 2 * ks) << 8);
-            const uint32_t sel1 = static_cast<uint32_t>(2 * ks + 1) | (static_cast<uint32_t>(5 + 2 * ks) << 8);
-            A[ks][0] = nib_pair(wg, wg4, sel0);   // row g,   logical k 2q, 2q+1
-            A[ks][1] = nib_pair(wh, wh4, sel0);   // row g+8
-            A[ks][2] = nib_pair(wg, wg4, sel1);   // row g,   logical k 2q+8, 2q+9
-            A[ks][3] = nib_pair(wh, wh4, sel1);
-            if (!kSumX) {
-              const uint32_t zzg = pack_bf16x2(zg, zg), zzh = pack_bf16x2(zh, zh);
-              A[ks][0] = bf16x2_sub(A[ks][0], zzg);
-              A[ks][1] = bf16x2_sub(A[ks][1], zzh);
-              A[ks][2] = bf16x2_sub(A[ks][2], zzg);
-              A[ks][3] = bf16x2_sub(A[ks][3], zzh);
+            for (int ks = 0; ks < 2; ++ks) {
+              const uint32_t sel0 = static_cast<uint32_t>(2 * ks) | (static_cast<uint32_t>(4 + 2 * ks) << 8);
+              const uint32_t sel1 = static_cast<uint32_t>(2 * ks + 1) | (static_cast<uint32_t>(5 + 2 * ks) << 8);
+              A[ks][0] = bf16x2_sub(nib_pair(wg, wg4, sel0), zzg);
+              A[ks][1] = bf16x2_sub(nib_pair(wh, wh4, sel0), zzh);
+              A[ks][2] = bf16x2_sub(nib_pair(wg, wg4, sel1), zzg);
+              A[ks][3] = bf16x2_sub(nib_pair(wh, wh4, sel1), zzh);
             }
           }
-          const uint32_t xsub = xst + (t32 >> 1) * C::XSUB;          // 64-column sub-tile
-          const uint32_t unit = (t32 & 1u) * 4u + static_cast<uint32_t>(q);
+          const uint32_t xa = xsub + (half ? xoff1 : xoff0);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
-            const int tr = 8 * j + g;                                 // token row
             uint32_t x0, x1, x2, x3;
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                         : "r"(xsub + tr * 128 + ((unit ^ static_cast<uint32_t>(tr & 7)) << 4)));
-            mma_bf16_16816(ga[j], A[0][0], A[0][1], A[0][2], A[0][3], x0, x1);
-            mma_bf16_16816(ga[j], A[1][0], A[1][1], A[1][2], A[1][3], x2, x3);
-            if (kSumX) {
-              mma_bf16_16816(sx, kOnes, kOnes, kOnes, kOnes, x0, x1);
-              mma_bf16_16816(sx, kOnes, kOnes, kOnes, kOnes, x2, x3);
-            }
+                         : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(xa + j * 1024));
+            if (half == 0) mma16816_zero_c(ga[j], A[0][0], A[0][1], A[0][2], A[0][3], x0, x1);
+            else mma16816(ga[j], A[0][0], A[0][1], A[0][2], A[0][3], x0, x1);
+            mma16816(ga[j], A[1][0], A[1][1], A[1][2], A[1][3], x2, x3);
           }
         }
         // D fragment: c0 (row g, token 2q), c1 (row g, token 2q+1), c2/c3 the same for row g+8
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          if (kSumX) {
-            tot[j][0] = fmaf(sg, fmaf(-zg, sx[0], ga[j][0]), tot[j][0]);
-            tot[j][1] = fmaf(sg, fmaf(-zg, sx[1], ga[j][1]), tot[j][1]);
-            tot[j][2] = fmaf(sh, fmaf(-zh, sx[2], ga[j][2]), tot[j][2]);
-            tot[j][3] = fmaf(sh, fmaf(-zh, sx[3], ga[j][3]), tot[j][3]);
+          if constexpr (C::PREP) {
+            const float2 sx = *reinterpret_cast<const float2*>(sxs + grp * (NT * 8) + 8 * j + 2 * q);
+            tot[j][0] = fmaf(sg, fmaf(-zg, sx.x, ga[j][0]), tot[j][0]);
+            tot[j][1] = fmaf(sg, fmaf(-zg, sx.y, ga[j][1]), tot[j][1]);
+            tot[j][2] = fmaf(sh, fmaf(-zh, sx.x, ga[j][2]), tot[j][2]);
+            tot[j][3] = fmaf(sh, fmaf(-zh, sx.y, ga[j][3]), tot[j][3]);
           } else {
             tot[j][0] = fmaf(sg, ga[j][0], tot[j][0]);
             tot[j][1] = fmaf(sg, ga[j][1], tot[j][1]);
@@ -248,7 +317,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     }
   }
   __syncthreads();
-  if (*abort_flag && warp == kComputeWarps && lane == 0) {
+  if (*abort_flag && warp == kProducer && lane == 0) {
     // a wait ran out: let the copies already issued land before shared memory goes away
     const uint64_t t0 = global_timer_ns();
     while (global_timer_ns() - t0 < 2000000ull) { }

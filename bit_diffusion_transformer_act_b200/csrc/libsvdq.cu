@@ -290,7 +290,7 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     if (!set_smem_once<k3::awq_gemm_kernel<NT_>>(smem, dev)) return SVDQ_ERR_CUDA;              \
     cudaLaunchConfig_t cfg = {};                                                                \
     cfg.gridDim = grid;                                                                         \
-    cfg.blockDim = dim3(k3::kThreads, 1, 1);                                                    \
+    cfg.blockDim = dim3(k3::Cfg<NT_>::THREADS, 1, 1);                                           \
     cfg.dynamicSmemBytes = smem;                                                                \
     cfg.stream = s;                                                                             \
     cudaLaunchAttribute attr[1];                                                                \
