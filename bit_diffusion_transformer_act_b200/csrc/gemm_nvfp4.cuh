@@ -21,7 +21,8 @@
 //           CTAs), the block-scaled MMAs (kind::mxf4nvf4, block16, K = 64) into a
 //           double-buffered fp32 accumulator, and the four bf16 low-rank MMAs
 //           (K = 16); commits release the stage in both CTAs and publish the
-//           accumulator to both epilogues.
+//           accumulator to both epilogues.  Two stages are issued per wait, which
+//           halves the per-stage synchronisation cost of the issuing thread.
 //   warps 2-5  epilogue (both CTAs): each warp owns 32 accumulator rows; tcgen05.ld 32
 //           columns at a time (two register sets, so a load is in flight while the
 //           previous chunk is converted), y = alpha acc + b (one fma, bias staged in
@@ -185,6 +186,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   cluster_sync_all();                              // barriers of both CTAs initialised and visible
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp == 0 && lane == 0 && pair < p.tiles) {
+    // the weights do not depend on the previous kernel: start pulling this CTA's first B
+    // tiles into L2 before waiting for it
+    const int bn_first = (pair % p.tiles_n) * BN + static_cast<int>(cta) * C::BN_HALF;
+    for (int kb = 0; kb < S && kb < nkb; ++kb) tma_prefetch_l2_2d(&tmB, kb * (BK / 2), bn_first);
+  }
   // everything above overlaps the previous kernel of the stream; its outputs (this
   // kernel's inputs) and its reads of Y are complete past this point
   grid_dependency_wait();
@@ -252,50 +259,59 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         tc_fence_after();
         const uint32_t dacc = tmem + static_cast<uint32_t>(b * C::ACC1);
         const uint32_t sfb_shift = static_cast<uint32_t>(((nt * BN) % 128) / 32);
-        for (int kb = 0; kb <= nkb; ++kb) {
-          const int s = g % S;
-          const uint32_t ph = (g / S) & 1u;
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 3))) { ok = false; break; }
+        // two 256-K stages per iteration (one wait, one elect), the tile's odd stage alone
+        for (int kb = 0; kb <= nkb;) {
+          const int cnt = kb + 1 < nkb ? 2 : 1;
+          bool okw = mbar_wait_bounded(full(g % S), (g / S) & 1u, abort_flag, 3);
+          if (cnt == 2) okw = okw && mbar_wait_bounded(full((g + 1) % S), ((g + 1) / S) & 1u, abort_flag, 3);
+          if (!__all_sync(0xFFFFFFFFu, okw)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sb = base + s * C::STAGE_BYTES;
-          const uint32_t a_lo = (sb >> 4) | kLbo;
-          const uint32_t b_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
           if (elect_one()) {
-          if (kb < nkb) {
-            const int na = min(BK / 64, natoms - kb * (BK / 64));
-            const uint32_t sfa_lo = (sb + C::A_BYTES + C::B_BYTES) >> 4;
-            const uint32_t sfb_lo = sfa_lo + C::SFA_BYTES / 16;
-            const uint32_t tsf = tmem + C::TM_SF + (g & 1u) * C::SF_COLS;
+            for (int c = 0; c < cnt; ++c) {
+              const uint32_t gg = g + c;
+              const int kbb = kb + c;
+              const int s = gg % S;
+              const uint32_t sb = base + s * C::STAGE_BYTES;
+              const uint32_t a_lo = (sb >> 4) | kLbo;
+              const uint32_t b_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
+              if (kbb < nkb) {
+                const int na = min(BK / 64, natoms - kbb * (BK / 64));
+                const uint32_t sfa_lo = (sb + C::A_BYTES + C::B_BYTES) >> 4;
+                const uint32_t sfb_lo = sfa_lo + C::SFA_BYTES / 16;
+                const uint32_t tsf = tmem + C::TM_SF + (gg & 1u) * C::SF_COLS;
 #pragma unroll
-            for (int kk = 0; kk < BK / 64; ++kk) {
-              if (kk < na) {
-                tc_copy_32x128b_x4_pair(tsf + 4 * kk, make_desc(sfa_lo + kk * 32, kHiSf));
+                for (int kk = 0; kk < BK / 64; ++kk) {
+                  if (kk < na) {
+                    tc_copy_32x128b_x4_pair(tsf + 4 * kk, make_desc(sfa_lo + kk * 32, kHiSf));
 #pragma unroll
-                for (int a = 0; a < C::SFB_ATOMS; ++a)
-                  tc_copy_32x128b_x4_pair(tsf + C::SFB_OFF + (kk * C::SFB_ATOMS + a) * 4,
-                                          make_desc(sfb_lo + (a * (BK / 64) + kk) * 32, kHiSf));
+                    for (int a = 0; a < C::SFB_ATOMS; ++a)
+                      tc_copy_32x128b_x4_pair(tsf + C::SFB_OFF + (kk * C::SFB_ATOMS + a) * 4,
+                                              make_desc(sfb_lo + (a * (BK / 64) + kk) * 32, kHiSf));
+                  }
+                }
+#pragma unroll
+                for (int kk = 0; kk < BK / 64; ++kk) {
+                  if (kk < na)
+                    umma_nvfp4_pair(dacc, make_desc(a_lo + kk * 2, kHiSw128), make_desc(b_lo + kk * 2, kHiSw128),
+                                    id4, tsf + 4 * kk, tsf + C::SFB_OFF + kk * C::SFB_ATOMS * 4 + sfb_shift,
+                                    (kbb | kk) != 0 ? 1u : 0u);
+                }
+              } else {
+                // A: [U hi | U lo] / g_a (128-byte swizzle); B: (L2 / g_w)^T (64-byte swizzle),
+                // K steps 0, 16, 0, 16; one K step = 16 bf16 = 32 B
+                const uint32_t l_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  umma_bf16_pair(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(l_lo + (j & 1) * 2, kHiSw64),
+                                 idb, 1u);
               }
+              tc_commit_pair(empty(s), 0x3);
             }
-#pragma unroll
-            for (int kk = 0; kk < BK / 64; ++kk) {
-              if (kk < na)
-                umma_nvfp4_pair(dacc, make_desc(a_lo + kk * 2, kHiSw128), make_desc(b_lo + kk * 2, kHiSw128), id4,
-                                tsf + 4 * kk, tsf + C::SFB_OFF + kk * C::SFB_ATOMS * 4 + sfb_shift,
-                                (kb | kk) != 0 ? 1u : 0u);
-            }
-          } else {
-            // A: [U hi | U lo] / g_a (128-byte swizzle); B: (L2 / g_w)^T (64-byte swizzle),
-            // K steps 0, 16, 0, 16; one K step = 16 bf16 = 32 B
-            const uint32_t l_lo = ((sb + C::A_BYTES) >> 4) | kLbo;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              umma_bf16_pair(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(l_lo + (j & 1) * 2, kHiSw64), idb, 1u);
-          }
-          tc_commit_pair(empty(s), 0x3);
-          if (kb == nkb) tc_commit_pair(acc_full(ab), 0x3);
+            if (kb + cnt - 1 == nkb) tc_commit_pair(acc_full(ab), 0x3);
           }
           __syncwarp();
-          ++g;
+          g += cnt;
+          kb += cnt;
         }
       }
     }
