@@ -23,12 +23,12 @@
 //           (K = 16); commits release the stage in both CTAs and publish the
 //           accumulator to both epilogues.  Two stages are issued per wait, which
 //           halves the per-stage synchronisation cost of the issuing thread.
-//   warps 2-5  epilogue (both CTAs): each warp owns 32 accumulator rows; tcgen05.ld 32
-//           columns at a time (two register sets, so a load is in flight while the
-//           previous chunk is converted), y = alpha acc + b (one fma, bias staged in
-//           shared memory), bf16 into a 128-byte-swizzled 32 x 64 staging tile, one TMA
-//           tensor store per 64 columns.  The accumulator buffer is handed back as soon
-//           as the columns the next tile will overwrite are in registers.
+//   warps 2-9  epilogue (both CTAs): two warps per tensor-memory lane quarter (32
+//           accumulator rows), each taking every other 32-column chunk; tcgen05.ld in a
+//           three-register-set rotation, y = alpha acc + b (one fma, bias staged in
+//           shared memory), bf16 into a 64-byte-swizzled 32 x 32 staging tile, one TMA
+//           tensor store per chunk.  The accumulator buffer is handed back as soon as the
+//           columns the next tile will overwrite are in registers.
 // Every mbarrier wait is bounded (about one second); a wait that runs out records
 // SVDQ_ERR_TIMEOUT in the device status word, the other roles give up, the MMAs in
 // flight are drained (bounded), tensor memory is freed and the kernel returns.
@@ -41,7 +41,8 @@ namespace k2 {
 
 constexpr int BM = 128;                    // A rows per CTA (256 per pair)
 constexpr int BK = 256;                    // K elements per pipeline stage
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                // two per tensor-memory lane quarter
+constexpr int kThreads = (2 + kEpiWarps) * 32;
 
 template <int BN>
 struct Cfg {
@@ -75,8 +76,8 @@ struct Cfg {
   static constexpr int NUM_BARS = 2 * STAGES + 5;              // full, empty, acc_full[2], acc_empty[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;  // per epilogue warp: the tile's bias (BN bf16)
-  static constexpr int OFF_STAGE = (OFF_BIAS + 4 * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 64 bf16
-  static constexpr int SMEM_BYTES = OFF_STAGE + 4 * 4096 + 1024;  // + slack to align the base to 1024
+  static constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 32 bf16
+  static constexpr int SMEM_BYTES = OFF_STAGE + kEpiWarps * 2048 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
   static_assert(TM_SF + 2 * SF_COLS <= TMEM_COLS, "tensor memory overflow");
@@ -85,7 +86,7 @@ struct Cfg {
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(OFF_BIAS % 16 == 0, "16-byte shared stores of the bias");
-  static_assert(OFF_STAGE % 1024 == 0, "128-byte-swizzled store staging needs 1024-byte alignment");
+  static_assert(OFF_STAGE % 1024 == 0, "64-byte-swizzled store staging needs 512-byte alignment");
   static_assert(!OVERLAP || (NCH == 8 && OV_CHUNKS == 3), "chunk order of the overlapping buffers");
 };
 
@@ -113,11 +114,11 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256() {
 }
 
 // y = bf16(alpha acc + b) for 32 consecutive columns of one row: fp32 accumulators in r,
-// their bias (32 bf16) at bias (shared memory).  The 64 result bytes are half `half` of
-// this lane's 128-byte row of a 32-row staging tile in the 128-byte swizzle of the
-// store's tensor map (16-byte unit u of row r at r * 128 + 16 (u ^ (r & 7))).
+// their bias (32 bf16) at bias (shared memory).  The 64 result bytes are this lane's row
+// of a 32 x 32 staging tile in the 64-byte swizzle of the store's tensor map (16-byte
+// unit u of row r at r * 64 + 16 (u ^ ((r >> 1) & 3))).
 __device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], const uint4* bias, float alpha,
-                                                 uint32_t row_smem, uint32_t sw, int half) {
+                                                 uint32_t row_smem, uint32_t sw) {
   uint32_t o[16];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -132,13 +133,11 @@ __device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], const 
     }
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t u = static_cast<uint32_t>(half * 4 + q);
+  for (int q = 0; q < 4; ++q)
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(row_smem + ((u ^ sw) << 4)), "r"(o[q * 4]), "r"(o[q * 4 + 1]), "r"(o[q * 4 + 2]),
-                   "r"(o[q * 4 + 3])
+                 ::"r"(row_smem + ((static_cast<uint32_t>(q) ^ sw) << 4)), "r"(o[q * 4]), "r"(o[q * 4 + 1]),
+                   "r"(o[q * 4 + 2]), "r"(o[q * 4 + 3])
                  : "memory");
-  }
 }
 
 template <int BN>
@@ -174,7 +173,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(acc_full(b), 1); mbar_init(acc_empty(b), 8); }
+    for (int b = 0; b < 2; ++b) { mbar_init(acc_full(b), 1); mbar_init(acc_empty(b), 2 * kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -320,10 +319,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter .. +31
     const int ew = warp - 2;
+    const int eh = ew >> 2;                        // this warp takes every other chunk, starting at eh
+    constexpr int NCW = C::NCH / 2;                // chunks per warp per tile
     uint8_t* sbias = gbase + C::OFF_BIAS + ew * 512;
-    const uint32_t sbias_a = smem_addr(sbias);
-    const uint32_t stage_row = base + C::OFF_STAGE + ew * 4096 + lane * 128;   // this lane's staging row
-    const uint32_t stage_tile = base + C::OFF_STAGE + ew * 4096;
+    const uint32_t stage_tile = base + C::OFF_STAGE + ew * 2048;
+    const uint32_t stage_row = stage_tile + lane * 64;                      // this lane's staging row
+    const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
     int i = 0;
     for (int t = pair; t < p.tiles; t += npairs, ++i) {
       const int mt = t / p.tiles_n, nt = t % p.tiles_n;
@@ -340,55 +341,53 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       tc_fence_after();
       const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * C::ACC1);
       const bool live = m0 < p.M;                  // warp-uniform: rows past M are clipped by the store
-      // Chunk order (32 columns each; consecutive pairs form one 64-column store).  With
-      // overlapping buffers the columns shared with the other buffer come first (chunks
-      // 5-7 of buffer 0, 0-2 of buffer 1) and the accumulator is released once they are
-      // in registers; otherwise it is released after the last chunk.
+      // Processing order of the tile's 32-column chunks.  With overlapping buffers the
+      // columns shared with the other buffer come first (chunks 5-7 of buffer 0, 0-2 of
+      // buffer 1) and each warp releases the accumulator once its share of them is in
+      // registers; otherwise after its last chunk.  This warp takes positions eh, eh + 2, ...
       const bool swap = C::OVERLAP && b == 0;
-      auto chunk = [&](int j) {
+      auto chunk = [&](int jj) {
+        const int j = 2 * jj + eh;
         if (!swap) return j;
         return j < 2 ? 6 + j : (j < 4 ? 7 - j : j - 4);        // 6 7 5 4 0 1 2 3
       };
       constexpr int kRelease = C::OVERLAP ? C::OV_CHUNKS : C::NCH;
+      const int nrel = (kRelease - eh + 1) / 2;    // this warp's chunks among the first kRelease
+      const int jrel = 3 * ((nrel - 1) / 3);       // the wait that covers the last of them
       auto release = [&]() {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(map_to_cta(acc_empty(ab), 0));
       };
-      // converts one chunk into its half of the staging tile; after the second half the
-      // tile goes out with one TMA store (the previous store must have finished reading it)
-      auto emit = [&](const uint32_t (&r)[32], int j) {
-        const int c = chunk(j);
-        const int half = c & 1;
-        if ((j & 1) == 0) {
-          if (lane == 0) bulk_wait_group_read<0>();
-          __syncwarp();
-        }
-        epilogue_stage32(r, reinterpret_cast<const uint4*>(sbias + c * 64), p.alpha, stage_row, lane & 7u, half);
-        if (j & 1) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, stage_tile, n0 + (c >> 1) * 64, m0);
-            bulk_commit_group();
-          }
+      // converts one chunk into the staging tile and stores it with one TMA store (the
+      // previous store from the tile must have finished reading it)
+      auto emit = [&](const uint32_t (&r)[32], int jj) {
+        const int c = chunk(jj);
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        epilogue_stage32(r, reinterpret_cast<const uint4*>(sbias + c * 64), p.alpha, stage_row, sw);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, stage_tile, n0 + c * 32, m0);
+          bulk_commit_group();
         }
       };
-      // Three register sets in rotation: chunks 0-2 are loaded up front; every third chunk
-      // one wait covers the three loads issued while the previous three were converted.
-      // With overlapping buffers the release follows the first wait, otherwise the last.
+      // Three register sets in rotation: this warp's first three chunks are loaded up front;
+      // every third chunk one wait covers the three loads issued while the previous three
+      // were converted.
       uint32_t R[3][32];
 #pragma unroll
-      for (int j = 0; j < 3 && j < C::NCH; ++j) tmem_ld_32x32b_x32(trow + chunk(j) * 32, R[j]);
+      for (int jj = 0; jj < 3 && jj < NCW; ++jj) tmem_ld_32x32b_x32(trow + chunk(jj) * 32, R[jj]);
 #pragma unroll
-      for (int j = 0; j < C::NCH; ++j) {
-        if (j % 3 == 0) {
+      for (int jj = 0; jj < NCW; ++jj) {
+        if (jj % 3 == 0) {
 #pragma unroll
-          for (int k = 0; k < 3 && j + k < C::NCH; ++k) tmem_wait_ld_regs(R[k]);
-          if (j + 3 >= kRelease && j < kRelease) release();
+          for (int k = 0; k < 3 && jj + k < NCW; ++k) tmem_wait_ld_regs(R[k]);
+          if (jj == jrel) release();
         }
-        if (live) emit(R[j % 3], j);
-        if (j + 3 < C::NCH) tmem_ld_32x32b_x32(trow + chunk(j + 3) * 32, R[j % 3]);
+        if (live) emit(R[jj % 3], jj);
+        if (jj + 3 < NCW) tmem_ld_32x32b_x32(trow + chunk(jj + 3) * 32, R[jj % 3]);
       }
     }
     if (lane == 0) bulk_wait_group<0>();           // stores complete before shared memory goes away

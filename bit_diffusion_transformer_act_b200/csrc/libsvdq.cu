@@ -221,7 +221,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, BN / 2,
                  CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_tmap(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
 
   const int pairs = std::min(p.tiles, sm_count(dev) / 2);
