@@ -136,7 +136,7 @@ class ClockSampler:
                 self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self._h is not None:
