@@ -5,7 +5,7 @@ One step is one pass of the whole hot path over one batch of synthetic input:
   * the SVDQ W4A4 NVFP4 attention projection, M=4096, K=N=3072, rank 32, group 16
     (kernel 1: smoothing + NVFP4 quantization + low-rank down; kernel 2: the
     block-scaled tcgen05 GEMM with the low-rank-up/bias epilogue);
-  * the AWQ W4A16 adaLN linear, K=3072, N=18432, group 64, at M = 1, 2, 4, 8, 64.
+  * the AWQ W4A16 adaLN linear, K=3072, N=18432, group 64, at M = 1, 2, 4, 8, 16, 32, 64.
 `value` is the SVDQ layer throughput in TFLOP/s (2MNK per step over the device
 time of kernels 1+2); the AWQ throughput in GB/s is reported under "awq".
 
@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 SVDQ W4A4 linear TFLOPS (% FP4 peak); AWQ W4A16 GB/s (% HBM)"
 SVDQ_SHAPE = (4096, 3072, 3072)              # M, K, N: DiT attention projection, 64x64 latent tokens
-AWQ_K, AWQ_N, AWQ_MS = 3072, 18432, (1, 2, 4, 8, 64)
+AWQ_K, AWQ_N, AWQ_MS = 3072, 18432, (1, 2, 4, 8, 16, 32, 64)
 RANK = 32
 NSETS = 8                                    # rotating copies (> 2x L2 per cycle)
 FP4_OVER_BF16 = 4.0                          # nominal dense ratio (9 / 2.25 PFLOP/s)
@@ -368,7 +368,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": "SVDQ W4A4 NVFP4 DiT attention projection M=4096 K=3072 N=3072 rank 32 group 16 "
-                        "+ AWQ W4A16 adaLN K=3072 N=18432 group 64 at M=1,2,4,8,64",
+                        "+ AWQ W4A16 adaLN K=3072 N=18432 group 64 at M=1,2,4,8,16,32,64",
             "svdq": {"M": SVDQ_SHAPE[0], "K": SVDQ_SHAPE[1], "N": SVDQ_SHAPE[2], "rank": RANK, "group": 16},
             "awq": {"M": list(AWQ_MS), "K": AWQ_K, "N": AWQ_N, "group": 64},
             "l2": "inputs, weights and outputs rotate over 8 resident copies (> 2x L2 per cycle); no flush",

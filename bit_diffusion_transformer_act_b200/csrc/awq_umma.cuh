@@ -1,0 +1,337 @@
+// Kernel 4: AWQ-style W4A16 linear for 9 <= M <= 64 tokens on the tcgen05 tensor
+// cores.  Same arithmetic as kernel 3 (awq_w4a16.cuh):
+//
+//   y[m, n] = sum_g s[n, g] * sum_{k in g} (q[n, k] - z[n, g]) x[m, k]  (+ b[n])
+//
+// Method: "Nunchaku Lite" docs, "Supported quantization types" (awq_w4a16 /
+// int4 / group 64).
+//
+// Design (sm_100a).  At M = 64 the product has as many tensor-core flops as there
+// are weight bytes to stream, more than mma.sync sustains; here a CTA owns 128
+// weight rows and all T (16, 32 or 64) token columns, and the weights are the A
+// operand of tcgen05.mma (kind::f16, M = 128, N = T, K = 16) with the fp32
+// accumulator in tensor memory.  448 threads:
+//   warp 0     TMA producer: per 256-K stage the 128 x 128-byte weight-code tile and
+//              the tokens' activations as four 64-column sub-tiles (128-byte swizzle,
+//              rows past M read as zeros) -- the MMA's B operand as they land.
+//   warps 2-9  dequantizers: two threads per weight row; per group of 64 K a thread
+//              turns 16 of the row's code bytes into bf16 q - z (128 + q by bit placement,
+//              one packed subtraction of 128 + z: exact) and writes them into the MMA's
+//              K-major 128-byte-swizzled A layout, one stage's four groups (64 KB) per
+//              unit, two units in rotation.
+//   warp 1     tensor memory and the MMA issue: per unit (four groups) sixteen MMAs into
+//              four of eight T-column accumulators (one tcgen05.commit frees the A unit,
+//              one publishes the four accumulators, one releases the stage) -- the issuing
+//              thread's waits and commits are per unit, its cost when per group.
+//   warps 10-13 epilogue: a thread owns one accumulator row; per group it reads the
+//              T partial sums (tcgen05.ld) and adds s[n, g] times them to fp32
+//              registers, handing accumulators back four at a time; at the end + b, bf16
+//              stores.
+// Every product is exact and each group's fp32 partial sum is scaled by s once, as in
+// kernel 3.  Every mbarrier wait is bounded.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace svdq {
+namespace k4 {
+
+constexpr int kRows = 128;                 // weight rows per CTA = MMA M
+constexpr int kChunk = 256;                // K per stage
+constexpr int kGroup = 64;
+constexpr int kWBytes = kRows * 128;       // packed weight codes of one stage
+constexpr int kASub = kRows * 128;         // one dequantized group: 128 rows x 64 K bf16
+constexpr int kABufs = 2;
+constexpr int kDeqWarps = 8;               // two threads per weight row (half a group each)
+constexpr int kEpiWarp0 = 2 + kDeqWarps;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;
+
+template <int T>
+struct Cfg {
+  static_assert(T == 16 || T == 32 || T == 64, "token columns");
+  static constexpr int XSUB = T * 128;                      // one 64-K activation sub-tile
+  static constexpr int STAGE = kWBytes + 4 * XSUB;
+  // groups per A unit (the MMA warp's step): a whole stage, or half of one at T = 64 where
+  // two 64 KB units would leave room for only two stages
+  static constexpr int UG = T == 64 ? 2 : 4;
+  static constexpr int ABYTES = UG * kASub;
+  static constexpr int STAGES = T == 64 ? 3 : (T == 32 ? 3 : 4);
+  static constexpr int OFF_A = STAGES * STAGE;
+  static constexpr int OFF_BAR = OFF_A + kABufs * ABYTES;
+  static constexpr int DBUFS = 8;                           // accumulators in tensor memory (T columns each)
+  static constexpr int DPAIRS = DBUFS / UG;                 // handed over a unit at a time
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * kABufs + 2 * DPAIRS + 1;   // + drain
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr int TMEM_COLS = DBUFS * T;               // 128, 256 or 512: a power of two
+  static_assert(STAGE % 1024 == 0 && OFF_A % 1024 == 0, "1 KB alignment of swizzled tiles");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct Params {
+  const __nv_bfloat16* scales;     // [N, K/64]
+  const __nv_bfloat16* zeros;      // [N, K/64]
+  const __nv_bfloat16* bias;       // [N] or null
+  __nv_bfloat16* Y;                // [M, N]
+  int M, N, K;
+};
+
+// kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, M = 128, N = T.
+template <int T>
+__device__ __forceinline__ uint32_t idesc_awq() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(T >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// bf16x2 {128 + low nibble, 128 + high nibble} of byte b of w, minus (128 + z) in both halves.
+__device__ __forceinline__ uint32_t deq_pair(uint32_t w, uint32_t w4, uint32_t sel, uint32_t zz) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(w4), "r"(sel));
+  r = (r & 0x000F000Fu) | 0x43004300u;
+  __nv_bfloat162 d = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&r), *reinterpret_cast<__nv_bfloat162*>(&zz));
+  return *reinterpret_cast<uint32_t*>(&d);
+}
+
+// Reads N consecutive 32-bit TMEM columns of this thread's lane (N = 16 or 32) and waits.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32) {
+    tmem_ld_32x32b_x32(taddr, r);
+    tmem_wait_ld_regs(r);
+  } else {
+    static_assert(N == 16, "16 or 32 columns");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+        :
+        : "memory");
+  }
+}
+
+template <int T>
+__global__ void __launch_bounds__(kThreads, 1)
+awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
+  using C = Cfg<T>;
+  constexpr int S = C::STAGES;
+  static_assert(4 % C::UG == 0, "units divide a stage");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + C::OFF_BAR;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (S + s); };
+  auto afull = [&](int a) { return bars + 8u * (2 * S + a); };
+  auto afree = [&](int a) { return bars + 8u * (2 * S + kABufs + a); };
+  constexpr int DP = C::DPAIRS;
+  auto dfull = [&](int d) { return bars + 8u * (2 * S + 2 * kABufs + d); };
+  auto dfree = [&](int d) { return bars + 8u * (2 * S + 2 * kABufs + DP + d); };
+  const uint32_t drain = bars + 8u * (2 * S + 2 * kABufs + 2 * DP);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n0 = blockIdx.x * kRows;
+  const int nkb = p.K / kChunk;
+  const int nunits = nkb * 4 / C::UG;                // C::UG groups per unit
+  const int gpr = p.K / kGroup;                    // groups per weight row
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), kDeqWarps + 1); }
+    for (int a = 0; a < kABufs; ++a) { mbar_init(afull(a), kDeqWarps); mbar_init(afree(a), 1); }
+    for (int d = 0; d < DP; ++d) { mbar_init(dfull(d), 1); mbar_init(dfree(d), 4); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) tmem_alloc<C::TMEM_COLS>(smem_addr(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();                          // X may belong to the previous kernel
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (kb / S) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 31))) break;
+      if (elect_one()) {
+        const uint32_t sb = base + s * C::STAGE;
+        mbar_arrive_expect_tx(full(s), C::STAGE);
+        tma_load_2d(sb, &tmW, kb * (kChunk / 2), n0, full(s));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * C::XSUB, &tmX, kb * kChunk + j * 64, 0, full(s));
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue (one elected lane)
+    constexpr uint32_t kHiSw128 = smem_desc_hi(1024, 2);      // K-major, 128-byte swizzle, 8-row groups
+    constexpr uint32_t kLbo = 1u << 16;
+    const uint32_t idesc = idesc_awq<T>();
+    for (int u = 0; u < nunits; ++u) {
+      const int kb = u * C::UG / 4;
+      const int s = kb % S, a = u % kABufs, dp = u % DP;
+      bool ok = mbar_wait_bounded(full(s), (kb / S) & 1u, abort_flag, 32);
+      ok = ok && mbar_wait_bounded(afull(a), (u / kABufs) & 1u, abort_flag, 33);
+      ok = ok && mbar_wait_bounded(dfree(dp), ((u / DP) & 1u) ^ 1u, abort_flag, 34);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int gi = 0; gi < C::UG; ++gi) {
+          const int grp = (u * C::UG + gi) & 3;
+          const uint32_t a_lo = ((base + C::OFF_A + a * C::ABYTES + gi * kASub) >> 4) | kLbo;
+          const uint32_t b_lo = ((base + s * C::STAGE + kWBytes + grp * C::XSUB) >> 4) | kLbo;
+          const uint32_t dacc = tmem + static_cast<uint32_t>((C::UG * dp + gi) * T);
+#pragma unroll
+          for (int j = 0; j < kGroup / 16; ++j)
+            umma_bf16(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(b_lo + j * 2, kHiSw128), idesc,
+                      j != 0 ? 1u : 0u);
+        }
+        tc_commit(afree(a));
+        tc_commit(dfull(dp));
+        if (((u + 1) * C::UG) % 4 == 0) tc_commit(empty(s));   // the stage's last unit
+      }
+      __syncwarp();
+    }
+  } else if (warp < kEpiWarp0) {
+    // ---------------------------------------------------------------- dequantizers
+    const int dt = threadIdx.x - 64;
+    const int r = dt & (kRows - 1);                // weight row of the tile
+    const int h = dt >> 7;                         // half of each group: code bytes 16 h .. 16 h + 15
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    const uint2* zrow = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
+    uint2 zn = __ldg(zrow);                        // zeros of the 4 groups of the next stage
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint2 zc = zn;
+      if (kb + 1 < nkb) zn = __ldg(zrow + kb + 1);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), (kb / S) & 1u, abort_flag, 35))) break;
+      const uint8_t* wrow = gbase + s * C::STAGE + r * 128;
+      bool ok = true;
+#pragma unroll 1
+      for (int ul = 0; ul < 4 / C::UG; ++ul) {       // the stage's units
+        const int u = kb * (4 / C::UG) + ul;
+        const int a = u % kABufs;
+        // this thread's 16 code bytes of each of the unit's groups (16-byte units 2 grp + h, swizzled)
+        uint4 c[C::UG];
+#pragma unroll
+        for (int gi = 0; gi < C::UG; ++gi)
+          c[gi] = *reinterpret_cast<const uint4*>(wrow + (((2 * (C::UG * ul + gi) + h) ^ rsw) << 4));
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(afree(a), ((u / kABufs) & 1u) ^ 1u, abort_flag, 36))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int gi = 0; gi < C::UG; ++gi) {
+          const int grp = C::UG * ul + gi;
+          const uint32_t zw = grp < 2 ? zc.x : zc.y;
+          const float z = ((grp & 1) ? bf16hi_to_f32(zw) : bf16lo_to_f32(zw)) + 128.f;
+          const uint32_t zz = pack_bf16x2(z, z);
+          const uint32_t cw[4] = {c[gi].x, c[gi].y, c[gi].z, c[gi].w};
+          const uint32_t arow = base + C::OFF_A + a * C::ABYTES + gi * kASub + r * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {             // A unit 4 h + v: K 8(4h + v) .. + 7 = code bytes of word v
+            const uint32_t w = cw[v], w4 = w >> 4;
+            const uint32_t o0 = deq_pair(w, w4, 0x0400u, zz), o1 = deq_pair(w, w4, 0x0501u, zz);
+            const uint32_t o2 = deq_pair(w, w4, 0x0602u, zz), o3 = deq_pair(w, w4, 0x0703u, zz);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         ::"r"(arow + ((static_cast<uint32_t>(4 * h + v) ^ rsw) << 4)), "r"(o0), "r"(o1), "r"(o2),
+                           "r"(o3)
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();                  // the tensor core reads the tile through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull(a));
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed(empty(s));   // this warp's code bytes are in registers
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;                  // tensor-memory lanes 32 quarter .. + 31
+    const int r = quarter * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint2* srow = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
+    float tot[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) tot[t] = 0.f;
+    uint2 sn = __ldg(srow), sc = sn;
+    for (int u = 0; u < nunits; ++u) {
+      const int dp = u % DP;
+      if ((u * C::UG) % 4 == 0) {                   // first unit of a stage
+        sc = sn;
+        if (u * C::UG / 4 + 1 < nkb) sn = __ldg(srow + u * C::UG / 4 + 1);
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(dfull(dp), (u / DP) & 1u, abort_flag, 37))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int gi = 0; gi < C::UG; ++gi) {
+        const int grp = (u * C::UG + gi) & 3;
+        const uint32_t sw = grp < 2 ? sc.x : sc.y;
+        const float sg = (grp & 1) ? bf16hi_to_f32(sw) : bf16lo_to_f32(sw);
+        const uint32_t tcol = trow + static_cast<uint32_t>((C::UG * dp + gi) * T);
+        if constexpr (T == 16) {
+          uint32_t v[16];
+          tmem_ld_cols<16>(tcol, v);
+#pragma unroll
+          for (int t = 0; t < 16; ++t) tot[t] = fmaf(sg, __uint_as_float(v[t]), tot[t]);
+        } else {
+#pragma unroll
+          for (int hh = 0; hh < T / 32; ++hh) {
+            uint32_t v[32];
+            tmem_ld_cols<32>(tcol + hh * 32, v);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) tot[hh * 32 + t] = fmaf(sg, __uint_as_float(v[t]), tot[hh * 32 + t]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed(dfree(dp));
+    }
+    if (n0 + r < p.N) {
+      const float bb = p.bias ? __bfloat162float(p.bias[n0 + r]) : 0.f;
+#pragma unroll
+      for (int t = 0; t < T; ++t)
+        if (t < p.M) p.Y[static_cast<size_t>(t) * p.N + n0 + r] = __float2bfloat16_rn(tot[t] + bb);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // a wait ran out: let the MMAs and copies already issued finish before the memory goes away
+    if (warp == 1) {
+      if (elect_one()) tc_commit(drain);
+      __syncwarp();
+      mbar_wait_bounded(drain, 0, nullptr, 38);
+    }
+    if (warp == 0 && lane == 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 2000000ull) { }
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<C::TMEM_COLS>(tmem);
+  }
+}
+
+}  // namespace k4
+}  // namespace svdq

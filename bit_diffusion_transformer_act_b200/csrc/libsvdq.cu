@@ -15,6 +15,7 @@
 #include "quant_act.cuh"
 #include "gemm_nvfp4.cuh"
 #include "awq_w4a16.cuh"
+#include "awq_umma.cuh"
 
 namespace {
 
@@ -275,22 +276,23 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   p.M = M;
   p.N = N;
   p.K = K;
-  const int nt = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));   // 8-token MMA tiles
+  // M <= 8: mma.sync kernel (one 8-token tile); M > 8: tcgen05 kernel with T = 16, 32 or 64 token columns
+  const int tx = M <= 8 ? 8 : (M <= 16 ? 16 : (M <= 32 ? 32 : 64));
   CUtensorMap tW, tX;
   if (!make_tmap(&tW, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, k3::kRows,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, 8 * nt, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, tx, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
   const dim3 grid((N + k3::kRows - 1) / k3::kRows, 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-#define SVDQ_AWQ_LAUNCH(NT_)                                                                    \
+#define SVDQ_AWQ_LAUNCH(KERNEL, SMEM_, THREADS_, PARAMS_)                                       \
   do {                                                                                          \
-    const int smem = k3::Cfg<NT_>::SMEM;                                                        \
-    if (!set_smem_once<k3::awq_gemm_kernel<NT_>>(smem, dev)) return SVDQ_ERR_CUDA;              \
+    const int smem = SMEM_;                                                                     \
+    if (!set_smem_once<KERNEL>(smem, dev)) return SVDQ_ERR_CUDA;                                \
     cudaLaunchConfig_t cfg = {};                                                                \
     cfg.gridDim = grid;                                                                         \
-    cfg.blockDim = dim3(k3::Cfg<NT_>::THREADS, 1, 1);                                           \
+    cfg.blockDim = dim3(THREADS_, 1, 1);                                                        \
     cfg.dynamicSmemBytes = smem;                                                                \
     cfg.stream = s;                                                                             \
     cudaLaunchAttribute attr[1];                                                                \
@@ -298,16 +300,28 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     attr[0].val.programmaticStreamSerializationAllowed = 1;                                     \
     cfg.attrs = attr;                                                                           \
     cfg.numAttrs = 1;                                                                           \
-    if (cudaLaunchKernelEx(&cfg, k3::awq_gemm_kernel<NT_>, tW, tX, p) != cudaSuccess) {         \
+    if (cudaLaunchKernelEx(&cfg, KERNEL, tW, tX, PARAMS_) != cudaSuccess) {                     \
       (void)cudaGetLastError();                                                                 \
       return SVDQ_ERR_CUDA;                                                                     \
     }                                                                                           \
   } while (0)
 
-  if (nt == 1) SVDQ_AWQ_LAUNCH(1);
-  else if (nt == 2) SVDQ_AWQ_LAUNCH(2);
-  else if (nt == 4) SVDQ_AWQ_LAUNCH(4);
-  else SVDQ_AWQ_LAUNCH(8);
+  if (tx == 8) {
+    SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<1>, k3::Cfg<1>::SMEM, k3::Cfg<1>::THREADS, p);
+  } else {
+    namespace k4 = svdq::k4;
+    k4::Params q;
+    q.scales = p.scales;
+    q.zeros = p.zeros;
+    q.bias = p.bias;
+    q.Y = p.Y;
+    q.M = M;
+    q.N = N;
+    q.K = K;
+    if (tx == 16) SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<16>, k4::Cfg<16>::SMEM, k4::kThreads, q);
+    else if (tx == 32) SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<32>, k4::Cfg<32>::SMEM, k4::kThreads, q);
+    else SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<64>, k4::Cfg<64>::SMEM, k4::kThreads, q);
+  }
 #undef SVDQ_AWQ_LAUNCH
   return launch_status();
 }

@@ -186,8 +186,10 @@ def _run_awq(P, a, bias=None):
     return Y.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (9, 256, 64), (16, 1024, 256),
-                                   (33, 512, 320), (64, 256, 128), (64, 1536, 512)])
+# M <= 8: the mma.sync kernel; 9 <= M <= 64: the tcgen05 kernel with 16, 32 or 64 token columns
+@pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (9, 256, 64), (12, 512, 192),
+                                   (16, 1024, 256), (24, 1024, 384), (33, 512, 320), (48, 768, 448),
+                                   (64, 256, 128), (64, 1536, 512)])
 def test_awq_shapes(P, M, K, N):
     a = synth.awq_workload(M, K, N, seed=M + K)
     b = synth.to_bf16(np.random.default_rng(N).standard_normal(N) * 0.1) if M % 2 else None
@@ -195,10 +197,11 @@ def test_awq_shapes(P, M, K, N):
     check_output(Y, oawq.forward(a.X, a.q, a.scales, a.zeros, b))
 
 
-def test_awq_integer_case_is_exact(P):
+@pytest.mark.parametrize("M", [5, 40])
+def test_awq_integer_case_is_exact(P, M):
     # s = 1, z = 8, small integer activations: every partial sum is an exact integer in fp32
     rng = np.random.default_rng(3)
-    M, K, N = 5, 512, 128
+    K, N = 512, 128
     a = synth.awq_workload(M, K, N)
     a.X[:] = rng.integers(-4, 5, size=(M, K))
     a.scales[:] = 1.0
@@ -215,7 +218,7 @@ def awq_full():
     return a, deq
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 64])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 12, 16, 32, 64])
 def test_awq_adaln_full_size(P, awq_full, M):
     a, deq = awq_full
     sub = synth.AwqWorkload(M, a.K, a.N, a.X[:M].copy(), a.q, a.qweight, a.scales, a.zeros, a.W)
