@@ -84,10 +84,12 @@ __device__ __forceinline__ uint32_t idesc_awq() {
 }
 
 // bf16x2 {128 + low nibble, 128 + high nibble} of byte b of w, minus (128 + z) in both halves.
-__device__ __forceinline__ uint32_t deq_pair(uint32_t w, uint32_t w4, uint32_t sel, uint32_t zz) {
+// magic = 0x43004300 comes in a register, so that the mask-and-place is one three-input logic
+// operation (an instruction takes one immediate).
+__device__ __forceinline__ uint32_t deq_pair(uint32_t w, uint32_t w4, uint32_t sel, uint32_t zz, uint32_t magic) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(w4), "r"(sel));
-  r = (r & 0x000F000Fu) | 0x43004300u;
+  asm("lop3.b32 %0, %0, 0x000F000F, %1, 0xEA;" : "+r"(r) : "r"(magic));
   __nv_bfloat162 d = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&r), *reinterpret_cast<__nv_bfloat162*>(&zz));
   return *reinterpret_cast<uint32_t*>(&d);
 }
@@ -149,6 +151,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     for (int d = 0; d < DP; ++d) { mbar_init(dfull(d), 1); mbar_init(dfree(d), 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    abort_flag[1] = 0x43004300;                    // the dequantization constant, read back as a register
     fence_mbar_init();
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
@@ -213,6 +216,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     const int r = dt & (kRows - 1);                // weight row of the tile
     const int h = dt >> 7;                         // half of each group: code bytes 16 h .. 16 h + 15
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    const uint32_t magic = static_cast<uint32_t>(abort_flag[1]);   // 0x43004300, opaque to the compiler
     const uint2* zrow = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
     uint2 zn = __ldg(zrow);                        // zeros of the 4 groups of the next stage
     for (int kb = 0; kb < nkb; ++kb) {
@@ -246,8 +250,8 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
           for (int v = 0; v < 4; ++v) {             // A unit 4 h + v: K 8(4h + v) .. + 7 = code bytes of word v
             const uint32_t w = cw[v], w4 = w >> 4;
-            const uint32_t o0 = deq_pair(w, w4, 0x0400u, zz), o1 = deq_pair(w, w4, 0x0501u, zz);
-            const uint32_t o2 = deq_pair(w, w4, 0x0602u, zz), o3 = deq_pair(w, w4, 0x0703u, zz);
+            const uint32_t o0 = deq_pair(w, w4, 0x0400u, zz, magic), o1 = deq_pair(w, w4, 0x0501u, zz, magic);
+            const uint32_t o2 = deq_pair(w, w4, 0x0602u, zz, magic), o3 = deq_pair(w, w4, 0x0703u, zz, magic);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
                          ::"r"(arow + ((static_cast<uint32_t>(4 * h + v) ^ rsw) << 4)), "r"(o0), "r"(o1), "r"(o2),
                            "r"(o3)

@@ -73,8 +73,14 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t w4, uint32_t s
   return (r & 0x000F000Fu) | 0x43004300u;
 }
 
-// bf16x2 {128 + nibble 0 of v, 128 + nibble 4 of v}
-__device__ __forceinline__ uint32_t nib04(uint32_t v) { return (v & 0x000F000Fu) | 0x43004300u; }
+// bf16x2 {128 + nibble 0 of v, 128 + nibble 4 of v}: one three-input logic operation,
+// (v & 0x000F000F) | magic, with magic = 0x43004300 held in a register (an instruction takes
+// one immediate; with both constants immediate the compiler spends two operations).
+__device__ __forceinline__ uint32_t nib04(uint32_t v, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, 0x000F000F, %2, 0xEA;" : "=r"(r) : "r"(v), "r"(magic));
+  return r;
+}
 
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
@@ -125,6 +131,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       mbar_init(ready(s), 32);
     }
     *abort_flag = 0;
+    abort_flag[1] = 0x43004300;                    // the dequantization constant, read back as a register
     fence_mbar_init();
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
@@ -168,11 +175,15 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
           const int item = lane + 32 * it;
           const int tok = item % (NT * 8), grp = item / (NT * 8);
           uint8_t* row = st + kWBytes + grp * C::XSUB + tok * 128;
+          // all eight units are loaded before the first store, so the loads overlap
+          uint4 vu[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) vu[u] = *reinterpret_cast<const uint4*>(row + ((u ^ (tok & 7)) << 4));
           float sum = 0.f;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4* up = reinterpret_cast<uint4*>(row + ((u ^ (tok & 7)) << 4));
-            const uint4 v = *up;
+            const uint4 v = vu[u];
             const float a0 = bf16lo_to_f32(v.x) + bf16hi_to_f32(v.x), a1 = bf16lo_to_f32(v.y) + bf16hi_to_f32(v.y);
             const float a2 = bf16lo_to_f32(v.z) + bf16hi_to_f32(v.z), a3 = bf16lo_to_f32(v.w) + bf16hi_to_f32(v.w);
             sum += (a0 + a1) + (a2 + a3);
@@ -192,6 +203,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   } else {
     // ---------------------------------------------------------------- dequantize + mma.sync
     const int g = lane >> 2, q = lane & 3;
+    const uint32_t magic = static_cast<uint32_t>(abort_flag[1]);   // 0x43004300, opaque to the compiler
     const int rg = warp * 16 + g;                  // this lane's weight rows: rg and rg + 8
     const int gpr = p.K / kGroup;                  // groups per weight row
     const int na = min(n0 + rg, p.N - 1), nb = min(n0 + rg + 8, p.N - 1);   // clamped for the loads
@@ -250,10 +262,10 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
           if constexpr (C::PREP) {
             // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
             const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
-            A[0][0] = nib04(wg);       A[0][1] = nib04(wh);
-            A[0][2] = nib04(wg4);      A[0][3] = nib04(wh4);
-            A[1][0] = nib04(wg >> 8);  A[1][1] = nib04(wh >> 8);
-            A[1][2] = nib04(wg4 >> 8); A[1][3] = nib04(wh4 >> 8);
+            A[0][0] = nib04(wg, magic);       A[0][1] = nib04(wh, magic);
+            A[0][2] = nib04(wg4, magic);      A[0][3] = nib04(wh4, magic);
+            A[1][0] = nib04(wg >> 8, magic);  A[1][1] = nib04(wh >> 8, magic);
+            A[1][2] = nib04(wg4 >> 8, magic); A[1][3] = nib04(wh4 >> 8, magic);
           } else {
             // pair b (real K elements 8q + 2b, 8q + 2b + 1) = byte b of w (low and high nibble)
             const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
