@@ -161,6 +161,16 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp == 0 && lane == 0) {
+    // The weights, scales and zeros never come from the previous kernel: start the first
+    // stages' tiles and this CTA's scale and zero rows toward L2 while it finishes (hints;
+    // L2 is coherent, so nothing stale can be read).
+    for (int kb = 0; kb < min(S, nkb); ++kb) tma_prefetch_l2_2d(&tmW, kb * (kChunk / 2), n0);
+    const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
+    const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
+    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
+    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
+  }
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
 
