@@ -7,29 +7,25 @@
 // int4 / group 64, an AWQ-style INT4 weight-only kernel); the Nunchaku Lite
 // article: used for the adaptive-normalisation layers, activations stay 16-bit.
 //
-// Design (sm_100a, memory-bound at small M).  A CTA owns 128 output rows and all
-// M <= 64 tokens and streams its 128 x K/2 bytes of packed weights exactly once.
-// Warp 8 is the TMA producer: per 256-K stage one 128-row x 128-byte weight tile
-// (128-byte swizzle) and the tokens' activations as four 64-column sub-tiles
-// (128-byte swizzle, rows past M read as zeros), into a deep ring of stages (the
-// activations are shared by every CTA and come from L2).  Warps 0-7 own 16
-// weight rows each and release a stage with one relaxed arrival per warp -- no
-// block-wide barrier in the loop.  The weights are the A operand of mma.sync
-// m16n8k16 (16 weight rows x 8 tokens), dequantized in registers: a nibble q
-// becomes the bf16 128 + q by bit placement (exact).  A lane's 32-bit word of
-// nibbles (one ldmatrix fetches the four words of a group) covers real K elements
-// 8p..8p+7 of a 32-K step (p = lane % 4); the MMA's K slots are a permutation of
-// them, the same for A and B.
-//   * M <= 8: warp 9 prepares each stage before the consumers see it: it reorders
-//     every 8-element activation unit to (k0,k4) (k1,k5) (k2,k6) (k3,k7), so that a
-//     pair of nibbles (p, p + 4) of a word becomes a bf16x2 operand with one shift
-//     and one logic operation, and it sums each token's 64 activations of each group.
-//     The zero point then enters once per group: s (sum (128 + q) x - (128 + z) sum x).
-//   * M > 8: pairs (2b, 2b + 1) through a byte permute, and one packed bf16
-//     subtraction of 128 + z gives q - z exactly.
-// Either way every product is exact and each group's fp32 partial sum is scaled by
-// s once.  Scales and zeros are read from global memory two stages ahead.  Every
-// mbarrier wait is bounded.
+// Design (sm_100a, memory-bound).  Used for M <= 8 tokens (9..64 go to the tcgen05
+// kernel, awq_umma.cuh).  A CTA owns 128 output rows and all tokens and streams its
+// 128 x K/2 bytes of packed weights exactly once.  Warp 8 is the TMA producer: per
+// 256-K stage one 128-row x 128-byte weight tile (128-byte swizzle) and the tokens'
+// activations as four 64-column sub-tiles (128-byte swizzle, rows past M read as
+// zeros), into a deep ring of stages (the activations are shared by every CTA and come
+// from L2).  Warp 9 prepares each stage before the consumers see it: it reorders every
+// 8-element activation unit to (k0,k4) (k1,k5) (k2,k6) (k3,k7) and sums each token's
+// 64 activations of each group.  Warps 0-7 own 16 weight rows each and release a stage
+// with one relaxed arrival per warp -- no block-wide barrier in the loop.  The weights
+// are the A operand of mma.sync m16n8k16 (16 weight rows x 8 tokens), dequantized in
+// registers: a nibble q becomes the bf16 128 + q by bit placement (exact).  A lane's
+// 32-bit word of nibbles (one ldmatrix fetches the four words of a group) covers real K
+// elements 8p..8p+7 of a 32-K step (p = lane % 4); with the reordered activations a pair
+// of nibbles (p, p + 4) becomes a bf16x2 operand with one shift and one logic operation,
+// the same K-slot permutation on both operands.  The zero point enters once per group:
+// s (sum (128 + q) x - (128 + z) sum x).  Every product is exact and each group's fp32
+// partial sum is scaled by s once.  Scales and zeros are read from global memory two
+// stages ahead.  Every mbarrier wait is bounded.
 #pragma once
 
 #include "ptx.cuh"
@@ -43,19 +39,16 @@ constexpr int kChunk = 256;                // K per stage
 constexpr int kGroup = 64;
 constexpr int kWBytes = kRows * 128;       // 16 KB of packed weights per stage
 
-template <int NT>
-struct Cfg {
-  static constexpr bool PREP = NT == 1;                     // activation reorder + group sums (warp 9)
-  static constexpr int THREADS = (kComputeWarps + (PREP ? 2 : 1)) * 32;
-  static constexpr int XSUB = NT * 8 * 128;                 // one 64-column activation sub-tile
-  static constexpr int OFF_SX = kWBytes + 4 * XSUB;         // group sums: [4 groups][NT * 8 tokens] fp32
-  static constexpr int STAGE = (OFF_SX + (PREP ? 4 * NT * 8 * 4 : 0) + 1023) / 1024 * 1024;
-  static constexpr int STAGES = NT == 1 ? 9 : (NT == 2 ? 7 : (NT == 4 ? 6 : 4));
-  static constexpr int OFF_BAR = STAGES * STAGE;
-  static constexpr int SMEM = OFF_BAR + 8 * 3 * STAGES + 16 + 1024;
-  static_assert(STAGE % 1024 == 0, "1 KB alignment of swizzled tiles");
-  static_assert(SMEM <= 227 * 1024, "shared memory");
-};
+constexpr int kXSub = 8 * 128;             // one 64-column activation sub-tile (8 tokens)
+constexpr int kOffSx = kWBytes + 4 * kXSub;    // group sums: [4 groups][8 tokens] fp32
+constexpr int kStage = (kOffSx + 4 * 8 * 4 + 1023) / 1024 * 1024;
+constexpr int kStages = 9;
+constexpr int kOffBar = kStages * kStage;
+constexpr int kSmem = kOffBar + 8 * 3 * kStages + 16 + 1024;
+constexpr int kProducer = kComputeWarps, kPrepWarp = kComputeWarps + 1;
+constexpr int kThreads = (kComputeWarps + 2) * 32;
+static_assert(kStage % 1024 == 0, "1 KB alignment of swizzled tiles");
+static_assert(kSmem <= 227 * 1024, "shared memory");
 
 struct Params {
   const __nv_bfloat16* scales;     // [N, K/64]
@@ -65,14 +58,6 @@ struct Params {
   int M, N, K;
 };
 
-// bf16x2 {128 + low nibble of byte b of w, 128 + high nibble of byte b of w};
-// sel picks byte b of w into byte 0 and byte b of w >> 4 into byte 2.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t w4, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(w4), "r"(sel));
-  return (r & 0x000F000Fu) | 0x43004300u;
-}
-
 // bf16x2 {128 + nibble 0 of v, 128 + nibble 4 of v}: one three-input logic operation,
 // (v & 0x000F000F) | magic, with magic = 0x43004300 held in a register (an instruction takes
 // one immediate; with both constants immediate the compiler spends two operations).
@@ -80,11 +65,6 @@ __device__ __forceinline__ uint32_t nib04(uint32_t v, uint32_t magic) {
   uint32_t r;
   asm("lop3.b32 %0, %1, 0x000F000F, %2, 0xEA;" : "=r"(r) : "r"(v), "r"(magic));
   return r;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
 }
 
 // D (16x8 fp32) = A (16x16 bf16, row) x B (16x8 bf16, col) + D, or + 0.  Not volatile:
@@ -104,25 +84,22 @@ __device__ __forceinline__ void mma16816_zero_c(float (&d)[4], uint32_t a0, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-template <int NT>
-__global__ void __launch_bounds__(Cfg<NT>::THREADS, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
-  using C = Cfg<NT>;
-  constexpr int S = C::STAGES;
+  constexpr int S = kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t bars = base + C::OFF_BAR;
+  const uint32_t bars = base + kOffBar;
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
   auto ready = [&](int s) { return bars + 8u * (2 * S + s); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 24 * S);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kOffBar + 24 * S);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n0 = blockIdx.x * kRows;
   const int nkb = p.K / kChunk;
-  constexpr int kProducer = kComputeWarps, kPrepWarp = kComputeWarps + 1;
 
   if (warp == kProducer && lane == 0) {
     for (int s = 0; s < S; ++s) {
@@ -150,12 +127,6 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
 
-  float tot[NT][4];                                // consumers: this lane's sums (D fragment layout)
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int t = 0; t < 4; ++t) tot[j][t] = 0.f;
-
   if (warp == kProducer) {
     // ---------------------------------------------------------------- TMA producer
     for (int kb = 0; kb < nkb; ++kb) {
@@ -163,57 +134,50 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       const uint32_t ph = (kb / S) & 1u;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 21))) break;
       if (elect_one()) {
-        const uint32_t sb = base + s * C::STAGE;
-        mbar_arrive_expect_tx(full(s), kWBytes + 4 * C::XSUB);
+        const uint32_t sb = base + s * kStage;
+        mbar_arrive_expect_tx(full(s), kWBytes + 4 * kXSub);
         tma_load_2d(sb, &tmW, kb * (kChunk / 2), n0, full(s));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * C::XSUB, &tmX, kb * kChunk + j * 64, 0, full(s));
+        for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * kXSub, &tmX, kb * kChunk + j * 64, 0, full(s));
       }
       __syncwarp();
     }
   } else if (warp == kPrepWarp) {
-    if constexpr (C::PREP) {
-      // ---------------------------------------------------------------- activation reorder + group sums
-      // lane -> (token, group) items: token = item % (NT * 8), group = item / (NT * 8)
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1u;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 23))) break;
-        uint8_t* st = gbase + s * C::STAGE;
+    // ---------------------------------------------------------------- activation reorder + group sums
+    const int tok = lane & 7, grp = lane >> 3;     // this lane: token lane % 8 of group lane / 8
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (kb / S) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 23))) break;
+      uint8_t* st = gbase + s * kStage;
+      uint8_t* row = st + kWBytes + grp * kXSub + tok * 128;
+      // all eight units are loaded before the first store, so the loads overlap
+      uint4 vu[8];
 #pragma unroll
-        for (int it = 0; it < NT; ++it) {
-          const int item = lane + 32 * it;
-          const int tok = item % (NT * 8), grp = item / (NT * 8);
-          uint8_t* row = st + kWBytes + grp * C::XSUB + tok * 128;
-          // all eight units are loaded before the first store, so the loads overlap
-          uint4 vu[8];
+      for (int u = 0; u < 8; ++u) vu[u] = *reinterpret_cast<const uint4*>(row + ((u ^ tok) << 4));
+      float sum = 0.f;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) vu[u] = *reinterpret_cast<const uint4*>(row + ((u ^ (tok & 7)) << 4));
-          float sum = 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            uint4* up = reinterpret_cast<uint4*>(row + ((u ^ (tok & 7)) << 4));
-            const uint4 v = vu[u];
-            const float a0 = bf16lo_to_f32(v.x) + bf16hi_to_f32(v.x), a1 = bf16lo_to_f32(v.y) + bf16hi_to_f32(v.y);
-            const float a2 = bf16lo_to_f32(v.z) + bf16hi_to_f32(v.z), a3 = bf16lo_to_f32(v.w) + bf16hi_to_f32(v.w);
-            sum += (a0 + a1) + (a2 + a3);
-            uint4 n;
-            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.x) : "r"(v.x), "r"(v.z));   // (k0, k4)
-            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.y) : "r"(v.x), "r"(v.z));   // (k1, k5)
-            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.z) : "r"(v.y), "r"(v.w));   // (k2, k6)
-            asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.w) : "r"(v.y), "r"(v.w));   // (k3, k7)
-            *up = n;
-          }
-          reinterpret_cast<float*>(st + C::OFF_SX)[grp * (NT * 8) + tok] = sum;
-        }
-        fence_proxy_async_smem();                  // the next TMA into this stage comes after these stores
-        mbar_arrive(ready(s));                     // release: this lane's stores are visible to the consumers
+      for (int u = 0; u < 8; ++u) {
+        const uint4 v = vu[u];
+        const float a0 = bf16lo_to_f32(v.x) + bf16hi_to_f32(v.x), a1 = bf16lo_to_f32(v.y) + bf16hi_to_f32(v.y);
+        const float a2 = bf16lo_to_f32(v.z) + bf16hi_to_f32(v.z), a3 = bf16lo_to_f32(v.w) + bf16hi_to_f32(v.w);
+        sum += (a0 + a1) + (a2 + a3);
+        uint4 n;
+        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.x) : "r"(v.x), "r"(v.z));   // (k0, k4)
+        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.y) : "r"(v.x), "r"(v.z));   // (k1, k5)
+        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(n.z) : "r"(v.y), "r"(v.w));   // (k2, k6)
+        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(n.w) : "r"(v.y), "r"(v.w));   // (k3, k7)
+        *reinterpret_cast<uint4*>(row + ((u ^ tok) << 4)) = n;
       }
+      reinterpret_cast<float*>(st + kOffSx)[grp * 8 + tok] = sum;
+      fence_proxy_async_smem();                    // the next TMA into this stage comes after these stores
+      mbar_arrive(ready(s));                       // release: this lane's stores are visible to the consumers
     }
   } else {
     // ---------------------------------------------------------------- dequantize + mma.sync
     const int g = lane >> 2, q = lane & 3;
     const uint32_t magic = static_cast<uint32_t>(abort_flag[1]);   // 0x43004300, opaque to the compiler
+    float tot[4] = {0.f, 0.f, 0.f, 0.f};           // this lane's sums (D fragment layout)
     const int rg = warp * 16 + g;                  // this lane's weight rows: rg and rg + 8
     const int gpr = p.K / kGroup;                  // groups per weight row
     const int na = min(n0 + rg, p.N - 1), nb = min(n0 + rg + 8, p.N - 1);   // clamped for the loads
@@ -228,7 +192,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     for (int grp = 0; grp < 4; ++grp)
       woff[grp] = static_cast<uint32_t>(lrow * 128) +
                   ((static_cast<uint32_t>(2 * grp + (lane >> 4)) ^ static_cast<uint32_t>(lane & 7)) << 4);
-    // activation unit of this lane in a sub-tile (token row g of each 8-token tile), per 32-K step
+    // activation unit of this lane in a sub-tile (token row g), per 32-K step
     const uint32_t xoff0 = static_cast<uint32_t>(g * 128) + ((static_cast<uint32_t>(q) ^ static_cast<uint32_t>(g)) << 4);
     const uint32_t xoff1 = static_cast<uint32_t>(g * 128) + ((static_cast<uint32_t>(4 + q) ^ static_cast<uint32_t>(g)) << 4);
 
@@ -249,9 +213,9 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         const int kk = min(kb + 2, nkb - 1);
         pb[0] = __ldg(sa + kk); pb[1] = __ldg(sb_ + kk); pb[2] = __ldg(za + kk); pb[3] = __ldg(zb + kk);
       }
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(C::PREP ? ready(s) : full(s), ph, abort_flag, 22))) break;
-      const uint32_t wst = base + s * C::STAGE;
-      const float* sxs = reinterpret_cast<const float*>(gbase + s * C::STAGE + C::OFF_SX);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(ready(s), ph, abort_flag, 22))) break;
+      const uint32_t wst = base + s * kStage;
+      const float* sxs = reinterpret_cast<const float*>(gbase + s * kStage + kOffSx);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
         const uint32_t w0 = grp < 2 ? cur[0].x : cur[0].y, w1 = grp < 2 ? cur[1].x : cur[1].y;
@@ -263,60 +227,28 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
         uint32_t wq[4];                            // {row g, row g+8} x {32-K step 0, 1}
         ldmatrix_x4(wst + woff[grp], wq[0], wq[1], wq[2], wq[3]);
-        const uint32_t xsub = wst + kWBytes + grp * C::XSUB;
-        float ga[NT][4];
+        const uint32_t xsub = wst + kWBytes + grp * kXSub;
+        float ga[4];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+          // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
           const uint32_t wg = wq[2 * half], wh = wq[2 * half + 1];
-          uint32_t A[2][4];
-          if constexpr (C::PREP) {
-            // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
-            const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
-            A[0][0] = nib04(wg, magic);       A[0][1] = nib04(wh, magic);
-            A[0][2] = nib04(wg4, magic);      A[0][3] = nib04(wh4, magic);
-            A[1][0] = nib04(wg >> 8, magic);  A[1][1] = nib04(wh >> 8, magic);
-            A[1][2] = nib04(wg4 >> 8, magic); A[1][3] = nib04(wh4 >> 8, magic);
-          } else {
-            // pair b (real K elements 8q + 2b, 8q + 2b + 1) = byte b of w (low and high nibble)
-            const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
-            const uint32_t zzg = pack_bf16x2(zg, zg), zzh = pack_bf16x2(zh, zh);
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-              const uint32_t sel0 = static_cast<uint32_t>(2 * ks) | (static_cast<uint32_t>(4 + 2 * ks) << 8);
-              const uint32_t sel1 = static_cast<uint32_t>(2 * ks + 1) | (static_cast<uint32_t>(5 + 2 * ks) << 8);
-              A[ks][0] = bf16x2_sub(nib_pair(wg, wg4, sel0), zzg);
-              A[ks][1] = bf16x2_sub(nib_pair(wh, wh4, sel0), zzh);
-              A[ks][2] = bf16x2_sub(nib_pair(wg, wg4, sel1), zzg);
-              A[ks][3] = bf16x2_sub(nib_pair(wh, wh4, sel1), zzh);
-            }
-          }
-          const uint32_t xa = xsub + (half ? xoff1 : xoff0);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            uint32_t x0, x1, x2, x3;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(xa + j * 1024));
-            if (half == 0) mma16816_zero_c(ga[j], A[0][0], A[0][1], A[0][2], A[0][3], x0, x1);
-            else mma16816(ga[j], A[0][0], A[0][1], A[0][2], A[0][3], x0, x1);
-            mma16816(ga[j], A[1][0], A[1][1], A[1][2], A[1][3], x2, x3);
-          }
+          const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
+          uint32_t x0, x1, x2, x3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(xsub + (half ? xoff1 : xoff0)));
+          const uint32_t a0 = nib04(wg, magic), a1 = nib04(wh, magic), a2 = nib04(wg4, magic), a3 = nib04(wh4, magic);
+          if (half == 0) mma16816_zero_c(ga, a0, a1, a2, a3, x0, x1);
+          else mma16816(ga, a0, a1, a2, a3, x0, x1);
+          mma16816(ga, nib04(wg >> 8, magic), nib04(wh >> 8, magic), nib04(wg4 >> 8, magic), nib04(wh4 >> 8, magic),
+                   x2, x3);
         }
         // D fragment: c0 (row g, token 2q), c1 (row g, token 2q+1), c2/c3 the same for row g+8
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if constexpr (C::PREP) {
-            const float2 sx = *reinterpret_cast<const float2*>(sxs + grp * (NT * 8) + 8 * j + 2 * q);
-            tot[j][0] = fmaf(sg, fmaf(-zg, sx.x, ga[j][0]), tot[j][0]);
-            tot[j][1] = fmaf(sg, fmaf(-zg, sx.y, ga[j][1]), tot[j][1]);
-            tot[j][2] = fmaf(sh, fmaf(-zh, sx.x, ga[j][2]), tot[j][2]);
-            tot[j][3] = fmaf(sh, fmaf(-zh, sx.y, ga[j][3]), tot[j][3]);
-          } else {
-            tot[j][0] = fmaf(sg, ga[j][0], tot[j][0]);
-            tot[j][1] = fmaf(sg, ga[j][1], tot[j][1]);
-            tot[j][2] = fmaf(sh, ga[j][2], tot[j][2]);
-            tot[j][3] = fmaf(sh, ga[j][3], tot[j][3]);
-          }
-        }
+        const float2 sx = *reinterpret_cast<const float2*>(sxs + grp * 8 + 2 * q);
+        tot[0] = fmaf(sg, fmaf(-zg, sx.x, ga[0]), tot[0]);
+        tot[1] = fmaf(sg, fmaf(-zg, sx.y, ga[1]), tot[1]);
+        tot[2] = fmaf(sh, fmaf(-zh, sx.x, ga[2]), tot[2]);
+        tot[3] = fmaf(sh, fmaf(-zh, sx.y, ga[3]), tot[3]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_relaxed(empty(s));   // this warp is done with the stage
@@ -325,17 +257,14 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     const int ra = n0 + rg, rb = ra + 8;
     const float ba = (p.bias && ra < p.N) ? __bfloat162float(p.bias[ra]) : 0.f;
     const float bb = (p.bias && rb < p.N) ? __bfloat162float(p.bias[rb]) : 0.f;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int t0 = 8 * j + 2 * q, t1 = t0 + 1;
-      if (t0 < p.M) {
-        if (ra < p.N) p.Y[static_cast<size_t>(t0) * p.N + ra] = __float2bfloat16_rn(tot[j][0] + ba);
-        if (rb < p.N) p.Y[static_cast<size_t>(t0) * p.N + rb] = __float2bfloat16_rn(tot[j][2] + bb);
-      }
-      if (t1 < p.M) {
-        if (ra < p.N) p.Y[static_cast<size_t>(t1) * p.N + ra] = __float2bfloat16_rn(tot[j][1] + ba);
-        if (rb < p.N) p.Y[static_cast<size_t>(t1) * p.N + rb] = __float2bfloat16_rn(tot[j][3] + bb);
-      }
+    const int t0 = 2 * q, t1 = t0 + 1;
+    if (t0 < p.M) {
+      if (ra < p.N) p.Y[static_cast<size_t>(t0) * p.N + ra] = __float2bfloat16_rn(tot[0] + ba);
+      if (rb < p.N) p.Y[static_cast<size_t>(t0) * p.N + rb] = __float2bfloat16_rn(tot[2] + bb);
+    }
+    if (t1 < p.M) {
+      if (ra < p.N) p.Y[static_cast<size_t>(t1) * p.N + ra] = __float2bfloat16_rn(tot[1] + ba);
+      if (rb < p.N) p.Y[static_cast<size_t>(t1) * p.N + rb] = __float2bfloat16_rn(tot[3] + bb);
     }
   }
   __syncthreads();

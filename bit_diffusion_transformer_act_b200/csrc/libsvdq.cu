@@ -307,7 +307,7 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   } while (0)
 
   if (tx == 8) {
-    SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<1>, k3::Cfg<1>::SMEM, k3::Cfg<1>::THREADS, p);
+    SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel, k3::kSmem, k3::kThreads, p);
   } else {
     namespace k4 = svdq::k4;
     k4::Params q;
