@@ -10,19 +10,21 @@
 // by a pair of CTAs (a 2-CTA cluster) with the pair-wide tensor-core MMA
 // (tcgen05 cta_group::2, M = 256): CTA r holds A rows [128 r, 128 r + 128) and B
 // rows [BN/2 r, BN/2 r + BN/2) of the tile, so each SM stages half of B and the
-// pair reads every operand byte from L2 once.  192 threads per CTA:
+// pair reads every operand byte from L2 once.  320 threads per CTA:
 //   warp 0  TMA producer (both CTAs): code tiles of A and B (128-byte swizzle,
 //           256 K per stage), their E4M3 scale atoms, and, as one extra stage per
 //           tile, the low-rank tiles (bf16 [U/g_a hi | lo] in the A slot, (L2/g_w)^T
 //           in the B slot).  Completion of both CTAs' copies is counted on the
-//           leader's full barrier.
+//           leader's full barrier of the stage's issue group (two stages, or the
+//           tile's odd one).
 //   warp 1  tensor memory (both CTAs, pair allocation); in the leader one thread
 //           issues the scale copies (tcgen05.cp, shared -> tensor memory in both
 //           CTAs), the block-scaled MMAs (kind::mxf4nvf4, block16, K = 64) into a
 //           double-buffered fp32 accumulator, and the four bf16 low-rank MMAs
 //           (K = 16); commits release the stage in both CTAs and publish the
-//           accumulator to both epilogues.  Two stages are issued per wait, which
-//           halves the per-stage synchronisation cost of the issuing thread.
+//           accumulator to both epilogues.  One barrier wait covers a group of two
+//           stages: a wait costs the issuing thread about as much as a quarter of a
+//           stage's tensor work, and the issuing thread is the mainloop's limit.
 //   warps 2-9  epilogue (both CTAs): two warps per tensor-memory lane quarter (32
 //           accumulator rows), each taking every other 32-column chunk; tcgen05.ld in a
 //           three-register-set rotation, y = alpha acc + b (one fma, bias staged in
@@ -73,7 +75,12 @@ struct Cfg {
   static constexpr uint32_t SFB_OFF = 4 * (BK / 64);            // B's columns after A's within a region
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;              // full, empty, acc_full[2], acc_empty[2], drain
+  // One full barrier per MMA-issue group (two stages, or one at a tile's end): the issuing
+  // thread waits once per group.  The producer reuses a slot only after the MMAs of the stage
+  // STAGES back have completed, and those STAGES + 1 stages span at most STAGES + 1 groups, so
+  // with NBF > STAGES no barrier is posted for a group while an earlier group still owns it.
+  static constexpr int NBF = 8;
+  static constexpr int NUM_BARS = NBF + STAGES + 5;            // full[NBF], empty, acc_full[2], acc_empty[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;  // per epilogue warp: the tile's bias (BN bf16)
   static constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 32 bf16
@@ -81,6 +88,7 @@ struct Cfg {
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
   static_assert(TM_SF + 2 * SF_COLS <= TMEM_COLS, "tensor memory overflow");
+  static_assert(NBF > STAGES, "a full barrier is reused only after its group was consumed");
   static_assert(!OVERLAP || (ACC1 % 32 == 0 && ACC1 > 0), "overlap is a whole number of epilogue chunks");
   static_assert(STAGE_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1 KB alignment of swizzled tiles");
   static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit the stage slots");
@@ -154,11 +162,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint8_t* gbase = smem_raw + (base - raw);
 
   const uint32_t bars = base + C::OFF_BAR;
-  auto full = [&](int s) { return bars + 8u * s; };
-  auto empty = [&](int s) { return bars + 8u * (S + s); };
-  auto acc_full = [&](int b) { return bars + 8u * (2 * S + b); };
-  auto acc_empty = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
-  const uint32_t drain = bars + 8u * (2 * S + 4);
+  constexpr int NBF = C::NBF;
+  auto full = [&](uint32_t it) { return bars + 8u * (it % NBF); };   // group `it` of the MMA issue order
+  auto empty = [&](int s) { return bars + 8u * (NBF + s); };
+  auto acc_full = [&](int b) { return bars + 8u * (NBF + S + b); };
+  auto acc_empty = [&](int b) { return bars + 8u * (NBF + S + 2 + b); };
+  const uint32_t drain = bars + 8u * (NBF + S + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 4);
 
@@ -172,7 +181,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int nkb = (p.K + BK - 1) / BK;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+    for (int i = 0; i < NBF; ++i) mbar_init(full(i), 2);    // the leader's two arrivals per group
+    for (int s = 0; s < S; ++s) mbar_init(empty(s), 1);
     for (int b = 0; b < 2; ++b) { mbar_init(acc_full(b), 1); mbar_init(acc_empty(b), 2 * kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -199,7 +209,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   if (warp == 0) {
     {
       // ------------------------------------------------------------------ producer (whole warp, one lane issues)
-      uint32_t g = 0;
+      uint32_t g = 0, it = 0;                      // stage and issue-group counters
       bool ok = true;
       for (int t = pair; ok && t < p.tiles; t += npairs) {
         const int mt = t / p.tiles_n, nt = t % p.tiles_n;
@@ -207,30 +217,37 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int n0 = nt * BN;
         const int bn0 = n0 + static_cast<int>(cta) * C::BN_HALF;   // this CTA's B rows
         const int rb = m0 / 128, nb = n0 / 128;
-        for (int kb = 0; kb <= nkb; ++kb) {                        // kb == nkb: the low-rank stage
-          const int s = g % S;
-          const uint32_t ph = (g / S) & 1u;
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 1))) { ok = false; break; }
-          const uint32_t fb = map_to_cta(full(s), 0);
-          const uint32_t sb = base + s * C::STAGE_BYTES;
-          if (elect_one()) {
-          if (kb < nkb) {
-            if (leader) mbar_arrive_expect_tx(full(s), C::TX_MAIN);
-            tma_load_2d_pair(sb, &tmA, kb * (BK / 2), m0, fb);
-            tma_load_2d_pair(sb + C::A_BYTES, &tmB, kb * (BK / 2), bn0, fb);
-            tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES, &tmSFA, 0, rb * natoms + kb * (BK / 64), fb);
+        for (int kb0 = 0; ok && kb0 <= nkb; ++it) {                 // kb == nkb: the low-rank stage
+          const int cnt = kb0 + 1 < nkb ? 2 : 1;                    // the MMA warp's grouping
+          const uint32_t fbar = full(it);
+          const uint32_t fb = map_to_cta(fbar, 0);
+          for (int c = 0; c < cnt; ++c) {
+            const int kb = kb0 + c;
+            const int s = g % S;
+            const uint32_t ph = (g / S) & 1u;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 1))) { ok = false; break; }
+            const uint32_t sb = base + s * C::STAGE_BYTES;
+            if (elect_one()) {
+              if (kb < nkb) {
+                if (leader) mbar_arrive_expect_tx(fbar, C::TX_MAIN);
+                tma_load_2d_pair(sb, &tmA, kb * (BK / 2), m0, fb);
+                tma_load_2d_pair(sb + C::A_BYTES, &tmB, kb * (BK / 2), bn0, fb);
+                tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES, &tmSFA, 0, rb * natoms + kb * (BK / 64), fb);
 #pragma unroll
-            for (int a = 0; a < C::SFB_ATOMS; ++a)
-              tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES + C::SFA_BYTES + a * (BK / 64) * 512, &tmSFB, 0,
-                               (nb + a) * natoms + kb * (BK / 64), fb);
-          } else {
-            if (leader) mbar_arrive_expect_tx(full(s), C::TX_LOWRANK);
-            tma_load_2d_pair(sb, &tmU, 0, m0, fb);
-            tma_load_2d_pair(sb + C::A_BYTES, &tmL2, 0, bn0, fb);
+                for (int a = 0; a < C::SFB_ATOMS; ++a)
+                  tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES + C::SFA_BYTES + a * (BK / 64) * 512, &tmSFB, 0,
+                                   (nb + a) * natoms + kb * (BK / 64), fb);
+              } else {
+                if (leader) mbar_arrive_expect_tx(fbar, C::TX_LOWRANK);
+                tma_load_2d_pair(sb, &tmU, 0, m0, fb);
+                tma_load_2d_pair(sb + C::A_BYTES, &tmL2, 0, bn0, fb);
+              }
+              if (cnt == 1 && leader) mbar_arrive(fbar);          // a one-stage group's second arrival
+            }
+            __syncwarp();
+            ++g;
           }
-          }
-          __syncwarp();
-          ++g;
+          kb0 += cnt;
         }
       }
     }
@@ -246,7 +263,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       constexpr uint32_t kHiSw64 = smem_desc_hi(512, 4);        // K-major, 64-byte swizzle
       constexpr uint32_t kHiSf = smem_desc_hi(128, 0);          // scale atoms: 8 rows x 16 B groups
       constexpr uint32_t kLbo = 1u << 16;
-      uint32_t g = 0;
+      uint32_t g = 0, it = 0;                      // stage and issue-group counters
       int i = 0;
       bool ok = true;
       for (int t = pair; ok && t < p.tiles; t += npairs, ++i) {
@@ -258,12 +275,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         tc_fence_after();
         const uint32_t dacc = tmem + static_cast<uint32_t>(b * C::ACC1);
         const uint32_t sfb_shift = static_cast<uint32_t>(((nt * BN) % 128) / 32);
-        // two 256-K stages per iteration (one wait, one elect), the tile's odd stage alone
-        for (int kb = 0; kb <= nkb;) {
+        // two 256-K stages per group (one barrier wait, one elect), the tile's odd stage alone
+        for (int kb = 0; kb <= nkb; ++it) {
           const int cnt = kb + 1 < nkb ? 2 : 1;
-          bool okw = mbar_wait_bounded(full(g % S), (g / S) & 1u, abort_flag, 3);
-          if (cnt == 2) okw = okw && mbar_wait_bounded(full((g + 1) % S), ((g + 1) / S) & 1u, abort_flag, 3);
-          if (!__all_sync(0xFFFFFFFFu, okw)) { ok = false; break; }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(it), (it / NBF) & 1u, abort_flag, 3))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           if (elect_one()) {
             for (int c = 0; c < cnt; ++c) {
