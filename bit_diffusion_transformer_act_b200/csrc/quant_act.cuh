@@ -24,11 +24,15 @@
 //              maxima, the E4M3 scales and E2M1 codes, and stores 16 code bytes and
 //              2 scale bytes straight to global memory.
 // A stage is free again when the eight quantizer warps have read it and the MMAs
-// that read it have completed (tcgen05.commit).  At the end, warps 2-5 (one per
-// tensor-memory lane quarter) read U = hi + lo, the cluster sums the slices, and
-// U / g_a is written split into bf16 hi + lo, the operand layout of the GEMM's
-// low-rank MMA.  Every mbarrier wait is bounded; a wait that runs out records
-// SVDQ_ERR_TIMEOUT in the device status word and the CTA winds down.
+// that read it have completed (tcgen05.commit).  At the end, warps 0, 1, 10 and 11
+// (one per tensor-memory lane quarter; none of them stores to global memory) read
+// U = hi + lo into shared memory, the cluster sums the slices, and U / g_a is written
+// split into bf16 hi + lo, the operand layout of the GEMM's low-rank MMA.  Only those
+// four warps arrive at the cluster barrier with release semantics (the quantizers'
+// pending code stores need not complete first), and the barrier that keeps shared
+// memory alive until the peers have read it is relaxed.  Every mbarrier wait is
+// bounded; a wait that runs out records SVDQ_ERR_TIMEOUT in the device status word
+// and the CTA winds down.
 //
 // Rounding.  amax/6 is formed by a Markstein-corrected multiplication by the
 // rounded reciprocal of 6 (P. Markstein's correction: with y = RN(1/b) and
@@ -57,7 +61,8 @@ constexpr int kRows = 128;                // rows per CTA (one 128-row scale blo
 constexpr int kChunk = 64;                // K columns per pipeline stage
 constexpr int kRank = 32;
 constexpr int kQuantWarps = 8;
-constexpr int kThreads = (2 + kQuantWarps) * 32;
+constexpr int kReadWarp0 = 2 + kQuantWarps;   // warps 10, 11: tensor-memory lane quarters 2, 3 of the U read-out
+constexpr int kThreads = (4 + kQuantWarps) * 32;
 constexpr int kStages = 4;
 constexpr int kMaxSlice = 2048;           // longest K slice (columns) held as fp32 smoothing factors
 constexpr int kXBytes = kRows * kChunk * 2;          // 16 KB
@@ -177,9 +182,9 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp >= 2) {
+  if (warp >= 2 && warp < kReadWarp0) {
     // the quantizers fetch the smoothing factors while the first tiles are in flight
-    for (int i = tid - 64; i < klen; i += kThreads - 64) smooth[i] = -__bfloat162float(p.smooth[kbeg + i]);
+    for (int i = tid - 64; i < klen; i += kQuantWarps * 32) smooth[i] = -__bfloat162float(p.smooth[kbeg + i]);
     asm volatile("bar.sync 1, %0;" ::"n"(kQuantWarps * 32) : "memory");   // quantizer warps only
   }
 
@@ -220,7 +225,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
       }
       __syncwarp();
     }
-  } else {
+  } else if (warp < kReadWarp0) {
     // ---------------------------------------------------------------- quantizers
     const int qt = tid - 64;                      // 0..255
     const int r = qt >> 1;                        // row of the chunk
@@ -270,7 +275,10 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   // ---------------------------------------------------------------- U = hi + lo, summed over the cluster
   __syncthreads();                                 // every stage has been consumed: reuse them for U
   float* upart = reinterpret_cast<float*>(gbase); // [128][32] fp32, 16-byte pieces rotated by the row
-  if (warp >= 2 && warp < 6) {
+  // Read out by warps 0, 1, 10 and 11 (lane quarters 0-3), which store nothing to global
+  // memory: their release arrival below does not wait for the quantizers' code stores.
+  const bool reader = warp < 2 || warp >= kReadWarp0;
+  if (reader) {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     float u[32];
@@ -294,7 +302,9 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   }
   const int ks = p.kslices;
   tc_fence_before();
-  cluster_sync_all();                              // partials of every slice in shared memory
+  if (reader) cluster_arrive_release();            // partials of every slice in shared memory
+  else cluster_arrive_relaxed();
+  cluster_wait_acquire();
   const uint32_t crank = cluster_ctarank();
   const int rpc = kRows / ks;                      // rows finished by this CTA
   for (int i = tid; i < rpc * 8; i += kThreads) {  // one 4-column piece of one row per thread
@@ -337,7 +347,10 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
       while (global_timer_ns() - t0 < 2000000ull) { }
     }
   }
-  cluster_sync_all();                              // the other CTAs are done reading this CTA's partials
+  // the other CTAs are done reading this CTA's partials (their loads have returned: nothing
+  // to order, so a relaxed arrival)
+  cluster_arrive_relaxed();
+  cluster_wait_acquire();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc<kTmemCols>(tmem);
