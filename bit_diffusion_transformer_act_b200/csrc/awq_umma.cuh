@@ -8,20 +8,23 @@
 //
 // Design (sm_100a).  At M = 64 the product has as many tensor-core flops as there
 // are weight bytes to stream, more than mma.sync sustains; here a CTA owns 128
-// weight rows and all T (16, 32 or 64) token columns, and the weights are the A
-// operand of tcgen05.mma (kind::f16, M = 128, N = T, K = 16) with the fp32
-// accumulator in tensor memory.  448 threads:
+// weight rows and all T (16, 32 or 64) token columns, and the dequantized weights are
+// the A operand of tcgen05.mma (kind::f16, M = 128, N = T, K = 16), held in tensor
+// memory (row n in lane n, two consecutive K per 32-bit column), with the fp32
+// accumulators in tensor memory too.  Keeping A out of shared memory matters: a bf16 A
+// written to and read back from shared memory costs four times the packed weight bytes
+// twice, more shared-memory bandwidth than the MMAs' own B reads.  448 threads:
 //   warp 0     TMA producer: per 256-K stage the 128 x 128-byte weight-code tile and
 //              the tokens' activations as four 64-column sub-tiles (128-byte swizzle,
 //              rows past M read as zeros) -- the MMA's B operand as they land.
-//   warps 2-9  dequantizers: two threads per weight row; per group of 64 K a thread
-//              turns 16 of the row's code bytes into bf16 q - z (128 + q by bit placement,
-//              one packed subtraction of 128 + z: exact) and writes them into the MMA's
-//              K-major 128-byte-swizzled A layout, one stage's four groups (64 KB) per
-//              unit, two units in rotation.
-//   warp 1     tensor memory and the MMA issue: per unit (four groups) sixteen MMAs into
-//              four of eight T-column accumulators (one tcgen05.commit frees the A unit,
-//              one publishes the four accumulators, one releases the stage) -- the issuing
+//   warps 2-9  dequantizers, two per tensor-memory lane quarter: a thread owns one weight
+//              row (its lane) and half of every group; it turns its 16 code bytes of a
+//              group into bf16 q - z (128 + q by bit placement, one packed subtraction of
+//              128 + z: exact) and writes them as 16 columns of its lane (tcgen05.st);
+//              units of four groups (two at T = 64), two units in rotation.
+//   warp 1     tensor memory and the MMA issue: per unit four MMAs per group, each into
+//              its own T-column accumulator (one tcgen05.commit frees the A unit, one
+//              publishes the unit's accumulators, one releases the stage) -- the issuing
 //              thread's waits and commits are per unit, its cost when per group.
 //   warps 10-13 epilogue: a thread owns one accumulator row; per group it reads the
 //              T partial sums (tcgen05.ld) and adds s[n, g] times them to fp32
@@ -40,9 +43,9 @@ constexpr int kRows = 128;                 // weight rows per CTA = MMA M
 constexpr int kChunk = 256;                // K per stage
 constexpr int kGroup = 64;
 constexpr int kWBytes = kRows * 128;       // packed weight codes of one stage
-constexpr int kASub = kRows * 128;         // one dequantized group: 128 rows x 64 K bf16
+constexpr int kACols = kGroup / 2;         // tensor-memory columns of one dequantized group (bf16 pairs)
 constexpr int kABufs = 2;
-constexpr int kDeqWarps = 8;               // two threads per weight row (half a group each)
+constexpr int kDeqWarps = 8;               // two per lane quarter (half a group each)
 constexpr int kEpiWarp0 = 2 + kDeqWarps;
 constexpr int kThreads = (kEpiWarp0 + 4) * 32;
 
@@ -52,20 +55,21 @@ struct Cfg {
   static constexpr int XSUB = T * 128;                      // one 64-K activation sub-tile
   static constexpr int STAGE = kWBytes + 4 * XSUB;
   // groups per A unit (the MMA warp's step): a whole stage, or half of one at T = 64 where
-  // two 64 KB units would leave room for only two stages
+  // the accumulators take more tensor memory
   static constexpr int UG = T == 64 ? 2 : 4;
-  static constexpr int ABYTES = UG * kASub;
-  static constexpr int STAGES = T == 64 ? 3 : (T == 32 ? 3 : 4);
-  static constexpr int OFF_A = STAGES * STAGE;
-  static constexpr int OFF_BAR = OFF_A + kABufs * ABYTES;
-  static constexpr int DBUFS = 8;                           // accumulators in tensor memory (T columns each)
+  static constexpr int STAGES = T == 64 ? 4 : (T == 32 ? 6 : 8);
+  static constexpr int OFF_BAR = STAGES * STAGE;
+  static constexpr int DBUFS = T == 64 ? 4 : 8;             // accumulators in tensor memory (T columns each)
   static constexpr int DPAIRS = DBUFS / UG;                 // handed over a unit at a time
   static constexpr int NUM_BARS = 2 * STAGES + 2 * kABufs + 2 * DPAIRS + 1;   // + drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr int TMEM_COLS = DBUFS * T;               // 128, 256 or 512: a power of two
-  static_assert(STAGE % 1024 == 0 && OFF_A % 1024 == 0, "1 KB alignment of swizzled tiles");
-  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static constexpr int A_COL0 = DBUFS * T;                  // tensor memory: accumulators, then the A units
+  static constexpr int TMEM_COLS = 512;
+  static_assert(A_COL0 + kABufs * UG * kACols <= TMEM_COLS, "tensor memory");
+  static_assert(DPAIRS >= 2, "accumulators double-buffered per unit");
+  static_assert(STAGE % 1024 == 0, "1 KB alignment of swizzled tiles");
+  static_assert(SMEM <= 227 * 1024 && SMEM > 116 * 1024, "shared memory: one CTA (and one 512-column allocation) per SM");
 };
 
 struct Params {
@@ -206,13 +210,12 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
         for (int gi = 0; gi < C::UG; ++gi) {
           const int grp = (u * C::UG + gi) & 3;
-          const uint32_t a_lo = ((base + C::OFF_A + a * C::ABYTES + gi * kASub) >> 4) | kLbo;
+          const uint32_t a_t = tmem + static_cast<uint32_t>(C::A_COL0 + (a * C::UG + gi) * kACols);
           const uint32_t b_lo = ((base + s * C::STAGE + kWBytes + grp * C::XSUB) >> 4) | kLbo;
           const uint32_t dacc = tmem + static_cast<uint32_t>((C::UG * dp + gi) * T);
 #pragma unroll
-          for (int j = 0; j < kGroup / 16; ++j)
-            umma_bf16(dacc, make_desc(a_lo + j * 2, kHiSw128), make_desc(b_lo + j * 2, kHiSw128), idesc,
-                      j != 0 ? 1u : 0u);
+          for (int j = 0; j < kGroup / 16; ++j)       // K = 16: 8 columns of A, 32 bytes of B
+            umma_bf16_ta(dacc, a_t + j * 8, make_desc(b_lo + j * 2, kHiSw128), idesc, j != 0 ? 1u : 0u);
         }
         tc_commit(afree(a));
         tc_commit(dfull(dp));
@@ -222,10 +225,11 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     }
   } else if (warp < kEpiWarp0) {
     // ---------------------------------------------------------------- dequantizers
-    const int dt = threadIdx.x - 64;
-    const int r = dt & (kRows - 1);                // weight row of the tile
-    const int h = dt >> 7;                         // half of each group: code bytes 16 h .. 16 h + 15
+    const int dq = warp & 3;                       // tensor-memory lane quarter of this warp
+    const int r = dq * 32 + lane;                  // weight row of the tile = tensor-memory lane
+    const int h = (warp - 2) >> 2;                 // half of each group: code bytes 16 h .. 16 h + 15
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(dq * 32) << 16) + static_cast<uint32_t>(C::A_COL0 + h * 16);
     const uint32_t magic = static_cast<uint32_t>(abort_flag[1]);   // 0x43004300, opaque to the compiler
     const uint2* zrow = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
     uint2 zn = __ldg(zrow);                        // zeros of the 4 groups of the next stage
@@ -256,19 +260,20 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
           const float z = ((grp & 1) ? bf16hi_to_f32(zw) : bf16lo_to_f32(zw)) + 128.f;
           const uint32_t zz = pack_bf16x2(z, z);
           const uint32_t cw[4] = {c[gi].x, c[gi].y, c[gi].z, c[gi].w};
-          const uint32_t arow = base + C::OFF_A + a * C::ABYTES + gi * kASub + r * 128;
+          // column 4 v + t of this half: K elements 32 h + 8 v + 2 t and + 1 (code byte t of word v)
+          uint32_t o[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {             // A unit 4 h + v: K 8(4h + v) .. + 7 = code bytes of word v
+          for (int v = 0; v < 4; ++v) {
             const uint32_t w = cw[v], w4 = w >> 4;
-            const uint32_t o0 = deq_pair(w, w4, 0x0400u, zz, magic), o1 = deq_pair(w, w4, 0x0501u, zz, magic);
-            const uint32_t o2 = deq_pair(w, w4, 0x0602u, zz, magic), o3 = deq_pair(w, w4, 0x0703u, zz, magic);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         ::"r"(arow + ((static_cast<uint32_t>(4 * h + v) ^ rsw) << 4)), "r"(o0), "r"(o1), "r"(o2),
-                           "r"(o3)
-                         : "memory");
+            o[4 * v + 0] = deq_pair(w, w4, 0x0400u, zz, magic);
+            o[4 * v + 1] = deq_pair(w, w4, 0x0501u, zz, magic);
+            o[4 * v + 2] = deq_pair(w, w4, 0x0602u, zz, magic);
+            o[4 * v + 3] = deq_pair(w, w4, 0x0703u, zz, magic);
           }
+          tmem_st_32x32b_x16(tlane + static_cast<uint32_t>((a * C::UG + gi) * kACols), o);
         }
-        fence_proxy_async_smem();                  // the tensor core reads the tile through the async proxy
+        tmem_wait_st();                            // the stores are in tensor memory ...
+        tc_fence_before();                         // ... and ordered before the arrival
         __syncwarp();
         if (lane == 0) mbar_arrive(afull(a));
       }
