@@ -13,7 +13,7 @@
 // memory (row n in lane n, two consecutive K per 32-bit column), with the fp32
 // accumulators in tensor memory too.  Keeping A out of shared memory matters: a bf16 A
 // written to and read back from shared memory costs four times the packed weight bytes
-// twice, more shared-memory bandwidth than the MMAs' own B reads.  448 threads:
+// twice, more shared-memory bandwidth than the MMAs' own B reads.  480 threads:
 //   warp 0     TMA producer: per 256-K stage the 128 x 128-byte weight-code tile and
 //              the tokens' activations as four 64-column sub-tiles (128-byte swizzle,
 //              rows past M read as zeros) -- the MMA's B operand as they land.
@@ -22,10 +22,11 @@
 //              group into bf16 q - z (128 + q by bit placement, one packed subtraction of
 //              128 + z: exact) and writes them as 16 columns of its lane (tcgen05.st);
 //              units of four groups (two at T = 64), two units in rotation.
-//   warp 1     tensor memory and the MMA issue: per unit four MMAs per group, each into
-//              its own T-column accumulator (one tcgen05.commit frees the A unit, one
-//              publishes the unit's accumulators, one releases the stage) -- the issuing
-//              thread's waits and commits are per unit, its cost when per group.
+//   warps 1, 14  the MMA issue (warp 1 also owns the tensor-memory allocation), even and
+//              odd units in alternation: per unit four MMAs per group, each group into its
+//              own T-column accumulator; one tcgen05.commit frees the A unit, one publishes
+//              the unit's accumulators, one releases the unit's reads of the stage.  A single
+//              issuing thread -- its barrier waits and 8-16 MMAs per unit -- was the limit.
 //   warps 10-13 epilogue: a thread owns one accumulator row; per group it reads the
 //              T partial sums (tcgen05.ld) and adds s[n, g] times them to fp32
 //              registers, handing accumulators back four at a time; at the end + b, bf16
@@ -47,7 +48,8 @@ constexpr int kACols = kGroup / 2;         // tensor-memory columns of one dequa
 constexpr int kABufs = 2;
 constexpr int kDeqWarps = 8;               // two per lane quarter (half a group each)
 constexpr int kEpiWarp0 = 2 + kDeqWarps;
-constexpr int kThreads = (kEpiWarp0 + 4) * 32;
+constexpr int kMmaWarp2 = kEpiWarp0 + 4;   // the second MMA-issuing warp (odd units)
+constexpr int kThreads = (kMmaWarp2 + 1) * 32;
 
 template <int T>
 struct Cfg {
@@ -150,10 +152,11 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   const int gpr = p.K / kGroup;                    // groups per weight row
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), kDeqWarps + 1); }
+    // a stage is free once the dequantizers have its code bytes and every unit's MMAs are done
+    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), kDeqWarps + 4 / C::UG); }
     for (int a = 0; a < kABufs; ++a) { mbar_init(afull(a), kDeqWarps); mbar_init(afree(a), 1); }
     for (int d = 0; d < DP; ++d) { mbar_init(dfull(d), 1); mbar_init(dfree(d), 4); }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);                           // both MMA-issuing warps
     *abort_flag = 0;
     abort_flag[1] = 0x43004300;                    // the dequantization constant, read back as a register
     fence_mbar_init();
@@ -193,12 +196,12 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       }
       __syncwarp();
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kMmaWarp2) {
     // ---------------------------------------------------------------- MMA issue (one elected lane)
     constexpr uint32_t kHiSw128 = smem_desc_hi(1024, 2);      // K-major, 128-byte swizzle, 8-row groups
     constexpr uint32_t kLbo = 1u << 16;
     const uint32_t idesc = idesc_awq<T>();
-    for (int u = 0; u < nunits; ++u) {
+    for (int u = warp == 1 ? 0 : 1; u < nunits; u += 2) {   // two issuing warps, alternate units
       const int kb = u * C::UG / 4;
       const int s = kb % S, a = u % kABufs, dp = u % DP;
       bool ok = mbar_wait_bounded(full(s), (kb / S) & 1u, abort_flag, 32);
@@ -219,7 +222,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
         tc_commit(afree(a));
         tc_commit(dfull(dp));
-        if (((u + 1) * C::UG) % 4 == 0) tc_commit(empty(s));   // the stage's last unit
+        tc_commit(empty(s));                       // this unit's reads of the stage
       }
       __syncwarp();
     }
@@ -335,7 +338,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   __syncthreads();
   if (*abort_flag) {
     // a wait ran out: let the MMAs and copies already issued finish before the memory goes away
-    if (warp == 1) {
+    if (warp == 1 || warp == kMmaWarp2) {
       if (elect_one()) tc_commit(drain);
       __syncwarp();
       mbar_wait_bounded(drain, 0, nullptr, 38);
