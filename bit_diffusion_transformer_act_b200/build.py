@@ -12,7 +12,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libsvdq.so")
 SOURCES = ["libsvdq.cu", "host_pack.cpp"]
-DEPS = SOURCES + ["ptx.cuh", "quant_act.cuh", "gemm_nvfp4.cuh", "awq_w4a16.cuh", "layout.h",
+DEPS = SOURCES + ["ptx.cuh", "quant_act.cuh", "gemm_nvfp4.cuh", "awq_w4a16.cuh", "awq_umma.cuh", "layout.h",
                   os.path.join("..", "..", "include", "svdq.h")]
 
 NVCC_FLAGS = [

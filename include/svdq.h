@@ -152,7 +152,11 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
 
 /* ---------------------------------------------------------------- AWQ W4A16 */
 
-/* Kernel 3: y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.
+/* y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.  M <= 8 runs the
+ * mma.sync kernel (kernel 3), 9 <= M <= 64 the tcgen05 kernel (kernel 4, 16, 32 or 64
+ * token columns).  Both form every product exactly and scale each group's fp32 sum by s
+ * once; kernel 4 multiplies (q - z) x, kernel 3 forms s (sum (128 + q) x - (128 + z) sum x),
+ * so the two differ only in fp32 rounding.
  *   X        device bf16 [M, K]
  *   qweight  device u8 [N, K/2], element 2i of a row in the low nibble
  *   scales   device bf16 [N, K/64]
@@ -160,8 +164,7 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
  *   bias     device bf16 [N] or NULL
  *   Y        device bf16 [M, N] out
  * 1 <= M <= 64 (or M == 0), N % 64 == 0, K % 256 == 0; pointers 16-byte
- * aligned.  The products (q - z) x are exact and each group's partial sum is
- * scaled by s in fp32.  Asynchronous on `stream`. */
+ * aligned.  Asynchronous on `stream`. */
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales,
                      const void* zeros, const void* bias, int M, int N, int K,
                      void* Y, void* stream);
