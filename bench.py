@@ -34,14 +34,15 @@ SVDQ_SHAPE = (4096, 3072, 3072)              # M, K, N: DiT attention projection
 AWQ_K, AWQ_N, AWQ_MS = 3072, 18432, (1, 2, 4, 8, 16, 32, 64)
 RANK = 32
 NSETS = 8                                    # rotating copies (> 2x L2 per cycle)
+NREP = 3                                     # passes over the copies per CUDA-graph batch (24 launches)
 FP4_OVER_BF16 = 4.0                          # nominal dense ratio (9 / 2.25 PFLOP/s)
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=384)       # 16 graph batches of 24
+    ap.add_argument("--warmup", type=int, default=24)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly (for profilers)")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -265,7 +266,8 @@ def run_ours(args, world, rank, local):
         else:
             wl.awq(P, i, int(name[3:]))
 
-    # one graph per kernel kind covering the NSETS rotating copies, plus single-set graphs for remainders
+    # one graph per kernel kind: NREP passes over the NSETS rotating copies (a batch of 24 launches),
+    # plus single-set graphs for remainders
     with torch.cuda.stream(stream):
         for i in range(NSETS):                       # eager warm-up (sets attributes, loads modules)
             for n in names:
@@ -277,8 +279,9 @@ def run_ours(args, world, rank, local):
         for n in names:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                for i in range(NSETS):
-                    launch(n, i)
+                for _ in range(NREP):
+                    for i in range(NSETS):
+                        launch(n, i)
             graphs[n] = g
             singles[n] = []
             for i in range(NSETS):
@@ -292,20 +295,20 @@ def run_ours(args, world, rank, local):
         """Runs nsteps steps on `stream`; appends (name, start, end, launches) event records."""
         done = 0
         while done < nsteps:
-            chunk = min(NSETS, nsteps - done)
+            chunk = min(NSETS * NREP, nsteps - done)
             for n in names:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                if use_graph and chunk == NSETS:
+                if use_graph and chunk == NSETS * NREP:
                     graphs[n].replay()
                 elif use_graph:
                     for i in range(chunk):
-                        singles[n][i].replay()
+                        singles[n][i % NSETS].replay()
                 else:
                     with torch.cuda.stream(stream):
                         for i in range(chunk):
-                            launch(n, i)
+                            launch(n, i % NSETS)
                 e1.record(stream)
                 if events is not None:
                     events.append((n, e0, e1, chunk))
@@ -372,7 +375,7 @@ def run_ours(args, world, rank, local):
             "svdq": {"M": SVDQ_SHAPE[0], "K": SVDQ_SHAPE[1], "N": SVDQ_SHAPE[2], "rank": RANK, "group": 16},
             "awq": {"M": list(AWQ_MS), "K": AWQ_K, "N": AWQ_N, "group": 64},
             "l2": "inputs, weights and outputs rotate over 8 resident copies (> 2x L2 per cycle); no flush",
-            "launch": "CUDA graphs of 8 steps per kernel" if use_graph else "eager",
+            "launch": "CUDA graphs of 24 launches per kernel (3 passes over the 8 copies)" if use_graph else "eager",
             "parallelism": "replicas x%d" % world,
             "seed": 0,
         },
