@@ -3,6 +3,8 @@
 The compute path is libsvdq.so (hand-written CUDA for sm_100a behind a C ABI,
 ``include/svdq.h``); this package is its ctypes binding.  Importing fails if
 the library has not been built (``python -m bit_diffusion_transformer_act_b200.build``).
+``torch_ops`` registers the device calls as ``torch.ops.svdq.*`` custom operators (with
+fake implementations for tracing) and provides the nn.Module layers.
 """
 
 from .ops import (  # noqa: F401
@@ -22,3 +24,4 @@ from .ops import (  # noqa: F401
     SvdqW4A4Linear,
     AwqW4A16Linear,
 )
+from .torch_ops import AwqLinear, SvdqLinear, swap_linears  # noqa: F401,E402
