@@ -89,6 +89,12 @@ def barrier(world):
         dist.barrier()
 
 
+def job_rate(world, steps, units_per_step, slowest_ms):
+    """Whole-job throughput in units per second: the units all ranks processed (each rank ran
+    `steps` steps of `units_per_step`) over the slowest rank's device time."""
+    return world * steps * units_per_step / (slowest_ms * 1e-3)
+
+
 def allreduce_max(x, world):
     if world == 1:
         return x
@@ -344,17 +350,17 @@ def run_ours(args, world, rank, local):
     if status:
         raise RuntimeError("device status %d after the timed region" % status)
 
-    value = world * args.steps * svdq_flops() / (svdq_ms_max * 1e-3) / 1e12
+    value = job_rate(world, args.steps, svdq_flops(), svdq_ms_max) / 1e12
     fp4_peak = FP4_OVER_BF16 * peaks["bf16_tflops"]
     k2_tflops = svdq_flops() / (avg_ms["k2"] * 1e-3) / 1e12
     k1_gbs = k1_bytes() / (avg_ms["k1"] * 1e-3) / 1e9
     awq_per_m = {}
     for m in AWQ_MS:
         gbs = awq_bytes(m) / (avg_ms["awq%d" % m] * 1e-3) / 1e9
-        agg = world * args.steps * awq_bytes(m) / (awq_ms_max[m] * 1e-3) / 1e9
+        agg = job_rate(world, args.steps, awq_bytes(m), awq_ms_max[m]) / 1e9
         awq_per_m[str(m)] = {"us": avg_ms["awq%d" % m] * 1e3, "gbs": gbs, "gbs_all_ranks": agg,
                              "frac_hbm": gbs / peaks["hbm_gbs"]}
-    awq_all = world * args.steps * sum(awq_bytes(m) for m in AWQ_MS) / (sum(awq_ms_max.values()) * 1e-3) / 1e9
+    awq_all = job_rate(world, args.steps, sum(awq_bytes(m) for m in AWQ_MS), sum(awq_ms_max.values())) / 1e9
 
     result = {
         "metric": METRIC,
