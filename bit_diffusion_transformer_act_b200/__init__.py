@@ -2,7 +2,7 @@
 
 The compute path is libsvdq.so (hand-written CUDA for sm_100a behind a C ABI,
 ``include/svdq.h``); this package is its ctypes binding.  Importing fails if
-the library has not been built (``python -m bit_diffusion_transformer_act_b200.build``).
+the library has not been built (``python bit_diffusion_transformer_act_b200/build.py``).
 ``torch_ops`` registers the device calls as ``torch.ops.svdq.*`` custom operators (with
 fake implementations for tracing) and provides the nn.Module layers.
 """
@@ -21,6 +21,9 @@ from .ops import (  # noqa: F401
     svdq_quantize_act_lowrank_down,
     svdq_w4a4_nvfp4_linear,
     awq_w4a16_linear,
+    svdq_act_amax,
+    svdq_quantize_act_lowrank_down_dyn,
+    svdq_w4a4_nvfp4_linear_dyn,
     SvdqW4A4Linear,
     AwqW4A16Linear,
 )

@@ -1,6 +1,6 @@
 """Builds libsvdq.so in-tree for sm_100a with nvcc (no GPU needed to build).
 
-    python -m bit_diffusion_transformer_act_b200.build [--force]
+    python bit_diffusion_transformer_act_b200/build.py [--force]
 """
 
 import os
@@ -12,7 +12,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libsvdq.so")
 SOURCES = ["libsvdq.cu", "host_pack.cpp"]
-DEPS = SOURCES + ["ptx.cuh", "quant_act.cuh", "gemm_nvfp4.cuh", "awq_w4a16.cuh", "awq_umma.cuh", "layout.h",
+DEPS = SOURCES + ["ptx.cuh", "quant_act.cuh", "gemm_nvfp4.cuh", "awq_w4a16.cuh", "awq_umma.cuh", "act_amax.cuh", "layout.h",
                   os.path.join("..", "..", "include", "svdq.h")]
 
 NVCC_FLAGS = [

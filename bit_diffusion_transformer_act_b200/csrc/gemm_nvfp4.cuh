@@ -36,6 +36,7 @@
 // flight are drained (bounded), tensor memory is freed and the kernel returns.
 #pragma once
 
+#include "act_amax.cuh"
 #include "ptx.cuh"
 
 namespace svdq {
@@ -104,7 +105,9 @@ struct Params {
   int M, N, K;
   int tiles_n;                     // N / BN
   int tiles;                       // ceil(M / 256) * tiles_n
-  float alpha;
+  float alpha;                     // g_a g_w
+  const unsigned int* amax;        // or, if not null, g_a from this amax word (kernel 5) ...
+  float w_scale;                   // ... times g_w
 };
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
@@ -337,6 +340,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter .. +31
     const int ew = warp - 2;
+    const float alpha = p.amax ? act_scale_from_amax(__uint_as_float(*p.amax)) * p.w_scale : p.alpha;
     const int eh = ew >> 2;                        // this warp takes every other chunk, starting at eh
     constexpr int NCW = C::NCH / 2;                // chunks per warp per tile
     uint8_t* sbias = gbase + C::OFF_BIAS + ew * 512;
@@ -383,7 +387,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int c = chunk(jj);
         if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
-        epilogue_stage32(r, reinterpret_cast<const uint4*>(sbias + c * 64), p.alpha, stage_row, sw);
+        epilogue_stage32(r, reinterpret_cast<const uint4*>(sbias + c * 64), alpha, stage_row, sw);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

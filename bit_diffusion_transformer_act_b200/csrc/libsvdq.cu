@@ -12,6 +12,7 @@
 #include "../../include/svdq.h"
 #include "layout.h"
 #include "ptx.cuh"
+#include "act_amax.cuh"
 #include "quant_act.cuh"
 #include "gemm_nvfp4.cuh"
 #include "awq_w4a16.cuh"
@@ -107,11 +108,14 @@ int launch_status() {
 
 extern "C" {
 
-int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
-                                   int rank, float act_global_scale, void* act_codes, void* act_scales,
-                                   void* lowrank_act, void* stream) {
+// Kernel 1 with the activation scale given (act_amax null) or formed on the device from the
+// amax word of kernel 5.
+static int quantize_impl(const void* X, const void* smooth_inv, const void* packed_w, int M, int K, int rank,
+                         float act_global_scale, const void* act_amax, void* act_codes, void* act_scales,
+                         void* lowrank_act, void* stream) {
   if (M < 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
-  if (!is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (!act_amax && !is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (act_amax && (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
   if (rank != svdq::kRank || K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;                       // empty batch: nothing to read or write
   if (!X || !smooth_inv || !packed_w || !act_codes || !act_scales || !lowrank_act) return SVDQ_ERR_INVALID_ARG;
@@ -130,8 +134,9 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   p.ucat = static_cast<__nv_bfloat16*>(lowrank_act);
   p.M = M;
   p.K = K;
-  p.g = act_global_scale;
-  p.inv_g = 1.0f / act_global_scale;   // exact: a power of two
+  p.g = act_amax ? 1.0f : act_global_scale;
+  p.inv_g = 1.0f / p.g;                // exact: a power of two
+  p.amax = static_cast<const unsigned int*>(act_amax);
 
   const int rowblocks = (M + 127) / 128;               // 128-row CTAs covering the scale padding
   const int kgroups = K / 64;
@@ -176,11 +181,31 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const 
   return launch_status();
 }
 
-int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act,
-                           float act_global_scale, const void* packed_w, float w_global_scale, int M, int N, int K,
-                           int rank, void* Y, void* stream) {
+int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                   int rank, float act_global_scale, void* act_codes, void* act_scales,
+                                   void* lowrank_act, void* stream) {
+  return quantize_impl(X, smooth_inv, packed_w, M, K, rank, act_global_scale, nullptr, act_codes, act_scales,
+                       lowrank_act, stream);
+}
+
+int svdq_quantize_act_lowrank_down_dyn(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                       int rank, const void* act_amax, void* act_codes, void* act_scales,
+                                       void* lowrank_act, void* stream) {
+  if (!act_amax) return SVDQ_ERR_INVALID_ARG;
+  return quantize_impl(X, smooth_inv, packed_w, M, K, rank, 1.0f, act_amax, act_codes, act_scales, lowrank_act,
+                       stream);
+}
+
+// Kernel 2 with the activation scale given (act_amax null) or formed on the device from the
+// amax word of kernel 5.
+static int linear_impl(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                       float act_global_scale, const void* act_amax, const void* packed_w, float w_global_scale,
+                       int M, int N, int K, int rank, void* Y, void* stream) {
   if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
-  if (!is_pow2_scale(act_global_scale) || !is_pow2_scale(w_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_scale(w_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (!act_amax && !is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
+  if (act_amax && (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
+  if (act_amax) act_global_scale = 1.0f;
   if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
@@ -205,6 +230,8 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   p.tiles_n = N / BN;
   p.tiles = ((M + 255) / 256) * p.tiles_n;
   p.alpha = static_cast<float>(alpha);
+  p.amax = static_cast<const unsigned int*>(act_amax);
+  p.w_scale = w_global_scale;
 
   const int natoms = K / 64;
   const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
@@ -252,6 +279,56 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const 
   else if (BN == 256) SVDQ_GEMM_LAUNCH(256);
   else SVDQ_GEMM_LAUNCH(128);
 #undef SVDQ_GEMM_LAUNCH
+  return launch_status();
+}
+
+int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                           float act_global_scale, const void* packed_w, float w_global_scale, int M, int N, int K,
+                           int rank, void* Y, void* stream) {
+  return linear_impl(act_codes, act_scales, lowrank_act, act_global_scale, nullptr, packed_w, w_global_scale, M, N,
+                     K, rank, Y, stream);
+}
+
+int svdq_w4a4_nvfp4_linear_dyn(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                               const void* act_amax, const void* packed_w, float w_global_scale, int M, int N, int K,
+                               int rank, void* Y, void* stream) {
+  if (!act_amax) return SVDQ_ERR_INVALID_ARG;
+  return linear_impl(act_codes, act_scales, lowrank_act, 1.0f, act_amax, packed_w, w_global_scale, M, N, K, rank, Y,
+                     stream);
+}
+
+int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream) {
+  if (M < 0 || K <= 0 || K % 64 != 0) return SVDQ_ERR_INVALID_ARG;
+  if (!act_amax || (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
+  if (M > 0 && (!X || !smooth_inv || !aligned16(X) || !aligned16(smooth_inv))) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(act_amax, 0, sizeof(unsigned int), s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  if (M == 0) return SVDQ_OK;                       // amax of an empty batch: 0 (g = 1)
+  namespace k5 = svdq::k5;
+  const size_t nvec = static_cast<size_t>(M) * (K / 8);
+  const size_t want = (nvec + k5::kThreads - 1) / k5::kThreads;
+  const int blocks = static_cast<int>(std::min<size_t>(want, static_cast<size_t>(sm_count(dev)) * 8));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks, 1, 1);
+  cfg.blockDim = dim3(k5::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k5::act_amax_kernel, static_cast<const __nv_bfloat16*>(X),
+                         static_cast<const __nv_bfloat16*>(smooth_inv), M, K,
+                         static_cast<unsigned int*>(act_amax)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
   return launch_status();
 }
 

@@ -52,6 +52,7 @@
 // nearest as its scalar counterpart.
 #pragma once
 
+#include "act_amax.cuh"
 #include "ptx.cuh"
 
 namespace svdq {
@@ -79,6 +80,7 @@ struct Params {
   int kslices;                     // cluster size along K
   float g;                         // per-tensor scale (power of two)
   float inv_g;
+  const unsigned int* amax;        // or, if not null, g from this amax word (kernel 5) at run time
 };
 
 // Shared memory (1024-byte aligned base): stages | smooth slice (fp32) | barriers.
@@ -177,6 +179,11 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   }
   if (warp == 1) tmem_alloc<kTmemCols>(smem_addr(tmem_slot));
   grid_dependency_wait();                          // X and the outputs may belong to the previous kernel
+  float g = p.g, inv_g = p.inv_g;                  // the per-tensor scale: given, or from the batch's amax
+  if (p.amax) {
+    g = act_scale_from_amax(__uint_as_float(*p.amax));
+    inv_g = 1.0f / g;                              // exact: a power of two
+  }
   grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -260,7 +267,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
           for (int w = 0; w < 4; ++w)
             nx[hh * 4 + w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(xw[w]), bf16hi_to_f32(xw[w])), sp[w]);
         }
-        sc2 |= quantize_group(nx, p.g, p.inv_g, cb[gq]) << (8 * gq);
+        sc2 |= quantize_group(nx, g, inv_g, cb[gq]) << (8 * gq);
       }
       // the tile has been read: release it to the producer (with the MMA's commit)
       __syncwarp();
@@ -321,7 +328,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
       if (src < ks) { sum.x += v[src].x; sum.y += v[src].y; sum.z += v[src].z; sum.w += v[src].w; }
     const int mm = m0 + rr;
     if (mm < p.M) {
-      const float uu[4] = {sum.x * p.inv_g, sum.y * p.inv_g, sum.z * p.inv_g, sum.w * p.inv_g};  // exact
+      const float uu[4] = {sum.x * inv_g, sum.y * inv_g, sum.z * inv_g, sum.w * inv_g};  // exact
       uint32_t hw[2], lw[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {

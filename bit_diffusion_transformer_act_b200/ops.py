@@ -28,7 +28,7 @@ class SvdqError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libsvdq.so not built at {LIB_PATH}; run `python -m bit_diffusion_transformer_act_b200.build`")
+        raise ImportError(f"libsvdq.so not built at {LIB_PATH}; run `python bit_diffusion_transformer_act_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
@@ -40,6 +40,9 @@ def _load():
         "svdq_quantize_act_lowrank_down": ([vp, vp, vp, i, i, i, f, vp, vp, vp, vp], i),
         "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
         "awq_w4a16_linear": ([vp, vp, vp, vp, vp, i, i, i, vp, vp], i),
+        "svdq_act_amax": ([vp, vp, i, i, vp, vp], i),
+        "svdq_quantize_act_lowrank_down_dyn": ([vp, vp, vp, i, i, i, vp, vp, vp, vp, vp], i),
+        "svdq_w4a4_nvfp4_linear_dyn": ([vp, vp, vp, vp, vp, f, i, i, i, i, vp, vp], i),
         "svdq_unswizzle_scales": ([vp, i, i, vp], i),
         "svdq_swizzle_scales": ([vp, i, i, vp], i),
         "svdq_device_status": ([i], i),
@@ -54,7 +57,8 @@ def _load():
 LIB = _load()
 EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes", "svdq_pack_weights",
             "svdq_act_scale_bytes", "svdq_quantize_act_lowrank_down", "svdq_w4a4_nvfp4_linear",
-            "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status")
+            "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status",
+            "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn")
 
 
 def _check(fn, st):
@@ -182,6 +186,53 @@ def svdq_w4a4_nvfp4_linear(act_codes, act_scales, lowrank_act, act_global_scale,
                                     float(act_global_scale), _ptr(packed_w), float(w_global_scale),
                                     M, N, K, rank, _ptr(Y), _stream())
     _check("svdq_w4a4_nvfp4_linear", st)
+    return Y
+
+
+def svdq_act_amax(X, smooth_inv, act_amax=None):
+    """Returns a cuda uint32 [1] holding the bits of max |X smooth_inv| (the dynamic scale's input)."""
+    M, K = X.shape
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    if act_amax is None:
+        act_amax = torch.empty((1,), dtype=torch.int32, device=X.device)
+    st = LIB.svdq_act_amax(_ptr(X), _ptr(smooth_inv), M, K, _ptr(act_amax), _stream())
+    _check("svdq_act_amax", st)
+    return act_amax
+
+
+def svdq_quantize_act_lowrank_down_dyn(X, smooth_inv, packed_w, act_amax, rank=RANK,
+                                       act_codes=None, act_scales=None, lowrank_act=None):
+    """As svdq_quantize_act_lowrank_down with g_a formed on the device from act_amax."""
+    M, K = X.shape
+    dev = X.device
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    if act_codes is None:
+        act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    if act_scales is None:
+        act_scales = torch.empty((svdq_act_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+    if lowrank_act is None:
+        lowrank_act = torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev)
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    st = LIB.svdq_quantize_act_lowrank_down_dyn(_ptr(X), _ptr(smooth_inv), _ptr(packed_w), M, K, rank,
+                                                _ptr(act_amax), _ptr(act_codes), _ptr(act_scales),
+                                                _ptr(lowrank_act), _stream())
+    _check("svdq_quantize_act_lowrank_down_dyn", st)
+    return act_codes, act_scales, lowrank_act
+
+
+def svdq_w4a4_nvfp4_linear_dyn(act_codes, act_scales, lowrank_act, act_amax, packed_w, w_global_scale,
+                               M, N, K, rank=RANK, Y=None):
+    """As svdq_w4a4_nvfp4_linear with g_a formed on the device from act_amax."""
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    st = LIB.svdq_w4a4_nvfp4_linear_dyn(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act), _ptr(act_amax),
+                                        _ptr(packed_w), float(w_global_scale), M, N, K, rank, _ptr(Y), _stream())
+    _check("svdq_w4a4_nvfp4_linear_dyn", st)
     return Y
 
 

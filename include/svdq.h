@@ -150,6 +150,31 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
                            const void* packed_w, float w_global_scale,
                            int M, int N, int K, int rank, void* Y, void* stream);
 
+/* -------------------------------------------- dynamic per-tensor activation scale */
+
+/* Kernel 5: the variant of the W4A4 layer whose activation scale g_a comes from the batch
+ * (max |X smooth_inv| over the whole tensor) instead of from calibration.
+ * "Nunchaku Lite" docs, "Supported quantization types" (svdq_w4a4 / nvfp4 / group 16); the
+ * per-tensor scale rule: g_a = the smallest power of two with g_a * 6 * 448 >= amax, 1 for
+ * amax = 0.
+ *
+ * svdq_act_amax clears the caller's 4-byte device word act_amax on `stream` and folds
+ * amax = max |X[m,k] smooth_inv[k]| into it as the bits of a non-negative float (the products
+ * are exact in fp32, so the word is exact).  X device bf16 [M, K], smooth_inv device bf16 [K];
+ * M >= 0 (M = 0 leaves 0), K % 64 == 0, X and smooth_inv 16-byte aligned, act_amax 4-byte aligned.
+ *
+ * svdq_quantize_act_lowrank_down_dyn and svdq_w4a4_nvfp4_linear_dyn are the calls of kernels 1
+ * and 2 with g_a read from act_amax on the device (after the previous kernel of the stream has
+ * finished) instead of passed in: the same outputs as the static calls given that g_a, and
+ * lowrank_act holds U / g_a of that g_a.  Other arguments and errors as the static calls. */
+int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream);
+int svdq_quantize_act_lowrank_down_dyn(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                       int rank, const void* act_amax, void* act_codes, void* act_scales,
+                                       void* lowrank_act, void* stream);
+int svdq_w4a4_nvfp4_linear_dyn(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                               const void* act_amax, const void* packed_w, float w_global_scale, int M, int N, int K,
+                               int rank, void* Y, void* stream);
+
 /* ---------------------------------------------------------------- AWQ W4A16 */
 
 /* y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.  M <= 8 runs the

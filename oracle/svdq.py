@@ -14,7 +14,8 @@ types": svdq_w4a4 / nvfp4 / group 16; "NunchakuLiteQuantizationConfig": rank 32)
 with R [N, K] the residual weight, L1 [K, r], L2 [r, N] the bfloat16 low-rank
 factors, b [N] the bias, and Q the NVFP4 quantizer of ``oracle.nvfp4``.  The
 activation per-tensor scale g_a is supplied by the caller (static calibration,
-a power of two); the weight per-tensor scale g_w comes from amax(R).  The
+a power of two), or in the dynamic variant taken from the batch's own amax of X_hat
+(``dynamic_act_scale``); the weight per-tensor scale g_w comes from amax(R).  The
 low-rank intermediate X_hat @ L1 is kept in float64 (not rounded).
 """
 
@@ -33,6 +34,15 @@ def smooth(X, smooth_inv):
 def quantize_activations(X, smooth_inv, g_a):
     """NVFP4 codes [M, K] and E4M3 scales [M, K/16] of X_hat with per-tensor scale g_a."""
     return nvfp4.quantize(smooth(X, smooth_inv), g_a)
+
+
+def dynamic_act_scale(X, smooth_inv):
+    """The dynamic variant's activation per-tensor scale: the per-tensor scale rule
+    (``nvfp4.global_scale``) applied to the batch's own amax of X_hat instead of a calibrated
+    one ("Nunchaku Lite" docs, "Supported quantization types": a per-tensor scale with the
+    per-16 block scales)."""
+    Xh = smooth(X, smooth_inv)
+    return nvfp4.global_scale(np.max(np.abs(Xh)) if Xh.size else 0.0)
 
 
 def quantize_weights(R):

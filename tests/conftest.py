@@ -8,6 +8,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_library():
+    """Compiles libsvdq.so if it is missing or stale, before any test imports the package
+    (importing the package loads the library).  The builder is loaded from its file so that
+    this needs no package import."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_svdq_build", os.path.join(ROOT, "bit_diffusion_transformer_act_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs an sm_100a GPU (B200) and the built CUDA library")
     config.addinivalue_line("markers", "slow: full-size CPU work (oracle on large shapes)")

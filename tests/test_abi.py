@@ -10,10 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_diffusion_transformer_act_b200 import build as _build
-
-_build.build()
-import bit_diffusion_transformer_act_b200 as P  # noqa: E402
+import bit_diffusion_transformer_act_b200 as P  # noqa: E402  (conftest has built the library)
 
 from parity_util import swizzled_offset, unswizzle  # noqa: E402
 

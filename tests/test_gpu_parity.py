@@ -225,3 +225,62 @@ def test_awq_adaln_full_size(P, awq_full, M):
     Y = _run_awq(P, sub)
     check_output(Y, a.X[:M].astype(np.float64) @ deq.T)
     assert P.svdq_device_status() == 0
+
+
+# ---------------------------------------------------------------- dynamic activation scale (kernel 5)
+
+def _run_svdq_dyn(P, X, smooth, packed, g_w, N):
+    M, K = X.shape
+    Xd, sd = _bf16_dev(X), _bf16_dev(smooth)
+    amax = P.svdq_act_amax(Xd, sd)
+    codes, scales, U = P.svdq_quantize_act_lowrank_down_dyn(Xd, sd, packed, amax)
+    Y = P.svdq_w4a4_nvfp4_linear_dyn(codes, scales, U, amax, packed, g_w, M, N, K)
+    torch.cuda.synchronize()
+    a = float(amax.view(torch.float32).cpu().item())
+    return a, codes, scales, U, Y
+
+
+def test_dynamic_scale_amax_is_exact_and_layer_matches_the_oracle(P):
+    w = synth.svdq_workload(256, 512, 512)
+    packed, gw = _pack(P, w)
+    a, codes, scales, U, Y = _run_svdq_dyn(P, w.X, w.smooth_inv, packed, gw, 512)
+    assert a == np.max(np.abs(svdq.smooth(w.X, w.smooth_inv)))          # bit-exact amax
+    g = svdq.dynamic_act_scale(w.X, w.smooth_inv)
+    Uc = U.float().cpu().numpy().astype(np.float64)
+    _check_act(codes.cpu().numpy(), scales.cpu().numpy(), g * (Uc[:, :32] + Uc[:, 32:]), w.X, w.smooth_inv, w.L1, g)
+    check_output(Y.float().cpu().numpy(), svdq.forward(w.X, w.smooth_inv, w.R, w.L1, w.L2, w.bias, g))
+    # the same kernels with that scale passed in: identical outputs
+    cs, ss, us, ys = _run_svdq(P, w.X, w.smooth_inv, packed, g, gw, 512)
+    assert np.array_equal(cs, codes.cpu().numpy()) and np.array_equal(ss, scales.cpu().numpy())
+    assert np.array_equal(ys, Y.float().cpu().numpy())
+    assert P.svdq_device_status() == 0
+
+
+@pytest.mark.parametrize("factor", [0.0, 2.0 ** 12, 2.0 ** -9])
+def test_dynamic_scale_zero_and_extreme_batches(P, factor):
+    w = synth.svdq_workload(128, 256, 256)
+    packed, gw = _pack(P, w)
+    X = synth.to_bf16(w.X * factor)
+    a, codes, scales, U, Y = _run_svdq_dyn(P, X, w.smooth_inv, packed, gw, 256)
+    g = svdq.dynamic_act_scale(X, w.smooth_inv)
+    assert a == np.max(np.abs(svdq.smooth(X, w.smooth_inv)))
+    cx, sx = svdq.quantize_activations(X, w.smooth_inv, g)
+    assert np.array_equal(codes.cpu().numpy(), nvfp4.pack_nibbles(cx))
+    assert np.array_equal(unswizzle(scales.cpu().numpy(), 128, 256)[:128], sx)
+    check_output(Y.float().cpu().numpy(), svdq.forward(X, w.smooth_inv, w.R, w.L1, w.L2, w.bias, g))
+
+
+def test_dynamic_scale_full_attention_layer(P):
+    M, K, N = 4096, 3072, 3072
+    w = synth.svdq_workload(M, K, N)
+    packed, gw = _pack(P, w)
+    a, codes, scales, U, Y = _run_svdq_dyn(P, w.X, w.smooth_inv, packed, gw, N)
+    assert a == np.max(np.abs(svdq.smooth(w.X, w.smooth_inv)))
+    g = svdq.dynamic_act_scale(w.X, w.smooth_inv)
+    cx, sx = svdq.quantize_activations(w.X, w.smooth_inv, g)
+    assert np.array_equal(codes.cpu().numpy(), nvfp4.pack_nibbles(cx))
+    assert np.array_equal(unswizzle(scales.cpu().numpy(), M, K)[:M], sx)
+    rows = np.sort(np.random.default_rng(12).choice(M, size=256, replace=False))
+    check_output(Y.float().cpu().numpy()[rows],
+                 svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, g))
+    assert P.svdq_device_status() == 0

@@ -161,3 +161,31 @@ def test_synthetic_workload_close_to_unquantized_layer():
     y = svdq.forward(w.X, w.smooth_inv, w.R, w.L1, w.L2, w.bias, w.g_a)
     ref = w.X.astype(np.float64) @ w.W.astype(np.float64).T + w.bias
     assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.05
+
+
+# ---------------------------------------------------------------- the dynamic activation scale
+
+def test_dynamic_scale_closed_forms():
+    # amax of X_hat exactly 6 * 448 = 2688 -> g = 1; one ulp above -> 2; half of it -> 1/2
+    s = np.ones(64)
+    X = np.zeros((3, 64))
+    X[1, 5] = -2688.0
+    assert svdq.dynamic_act_scale(X, s) == 1.0
+    X[1, 5] = np.nextafter(2688.0, np.inf)
+    assert svdq.dynamic_act_scale(X, s) == 2.0
+    X[1, 5] = 1344.0
+    assert svdq.dynamic_act_scale(X, s) == 0.5
+    X[1, 5] = 1344.0 + 2.0 ** -20
+    assert svdq.dynamic_act_scale(X, s) == 1.0
+    assert svdq.dynamic_act_scale(np.zeros((2, 64)), s) == 1.0
+
+
+def test_dynamic_scale_uses_the_smoothed_activations_and_scales_exactly():
+    rng = np.random.default_rng(11)
+    X = synth.to_bf16(rng.standard_normal((16, 128)) * 3.0)
+    s = synth.to_bf16(np.exp2(rng.integers(-3, 4, size=128)).astype(np.float64))   # powers of two
+    amax = np.max(np.abs(X * s[None, :]))
+    g = svdq.dynamic_act_scale(X, s)
+    assert g * 2688.0 >= amax > g * 1344.0 and np.log2(g) == int(np.log2(g))
+    for k in (-3, 5):                       # an exact power-of-two rescale of X rescales g exactly
+        assert svdq.dynamic_act_scale(X * 2.0 ** k, s) == g * 2.0 ** k

@@ -3,10 +3,7 @@
 import numpy as np
 import pytest
 
-from bit_diffusion_transformer_act_b200 import build as _build
-
-_build.build()
-import bit_diffusion_transformer_act_b200 as P  # noqa: E402
+import bit_diffusion_transformer_act_b200 as P  # noqa: E402  (conftest has built the library)
 
 from oracle import nvfp4, svdq  # noqa: E402
 import synth  # noqa: E402
