@@ -240,7 +240,7 @@ class Workload:
                 "scales": torch.empty((P.svdq_act_scale_bytes(M, K),), dtype=torch.uint8, device=dev),
                 "U": torch.empty((M, 2 * RANK), dtype=torch.bfloat16, device=dev),
                 "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
-                "amax": torch.zeros((1,), dtype=torch.int32, device=dev),
+                "amax": torch.zeros((4,), dtype=torch.int32, device=dev),
             })
         a = synth.awq_workload(max(AWQ_MS), AWQ_K, AWQ_N)
         ax = bf16_dev(a.X, dev)

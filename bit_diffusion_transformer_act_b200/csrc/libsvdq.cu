@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <numeric>
 #include <cmath>
 #include <mutex>
 
@@ -299,20 +300,27 @@ int svdq_w4a4_nvfp4_linear_dyn(const void* act_codes, const void* act_scales, co
 
 int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream) {
   if (M < 0 || K <= 0 || K % 64 != 0) return SVDQ_ERR_INVALID_ARG;
-  if (!act_amax || (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
+  if (!act_amax || !aligned16(act_amax)) return SVDQ_ERR_INVALID_ARG;
   if (M > 0 && (!X || !smooth_inv || !aligned16(X) || !aligned16(smooth_inv))) return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(act_amax, 0, sizeof(unsigned int), s) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return SVDQ_ERR_CUDA;
+  if (M == 0) {                                     // amax of an empty batch: 0 (g = 1)
+    if (cudaMemsetAsync(act_amax, 0, sizeof(unsigned int), s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    return SVDQ_OK;
   }
-  if (M == 0) return SVDQ_OK;                       // amax of an empty batch: 0 (g = 1)
   namespace k5 = svdq::k5;
-  const size_t nvec = static_cast<size_t>(M) * (K / 8);
+  // a multiple of q blocks, so that the grid's thread count is a multiple of the row's K / 8
+  // units (the kernel keeps one column per thread); up to 8 blocks per SM
+  const int kv = K / 8;
+  const int q = kv / std::gcd(kv, k5::kThreads);
+  const size_t nvec = static_cast<size_t>(M) * kv;
   const size_t want = (nvec + k5::kThreads - 1) / k5::kThreads;
-  const int blocks = static_cast<int>(std::min<size_t>(want, static_cast<size_t>(sm_count(dev)) * 8));
+  const size_t cap = static_cast<size_t>(sm_count(dev)) * 8;
+  const int blocks = static_cast<int>(std::max<size_t>(q, std::min(want, cap) / q * q));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks, 1, 1);
   cfg.blockDim = dim3(k5::kThreads, 1, 1);

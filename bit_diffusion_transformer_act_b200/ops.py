@@ -190,12 +190,15 @@ def svdq_w4a4_nvfp4_linear(act_codes, act_scales, lowrank_act, act_global_scale,
 
 
 def svdq_act_amax(X, smooth_inv, act_amax=None):
-    """Returns a cuda uint32 [1] holding the bits of max |X smooth_inv| (the dynamic scale's input)."""
+    """Returns the 16-byte device buffer (int32 [4]) whose word 0 holds the bits of
+    max |X smooth_inv| (the dynamic scale's input); a buffer passed in must have been
+    zero-filled once (the call leaves words 1-3 zero)."""
     M, K = X.shape
     _require(X, torch.bfloat16, (M, K), "X")
     _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
     if act_amax is None:
-        act_amax = torch.empty((1,), dtype=torch.int32, device=X.device)
+        act_amax = torch.zeros((4,), dtype=torch.int32, device=X.device)
+    _require(act_amax, torch.int32, (4,), "act_amax")
     st = LIB.svdq_act_amax(_ptr(X), _ptr(smooth_inv), M, K, _ptr(act_amax), _stream())
     _check("svdq_act_amax", st)
     return act_amax

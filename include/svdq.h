@@ -158,13 +158,15 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
  * per-tensor scale rule: g_a = the smallest power of two with g_a * 6 * 448 >= amax, 1 for
  * amax = 0.
  *
- * svdq_act_amax clears the caller's 4-byte device word act_amax on `stream` and folds
- * amax = max |X[m,k] smooth_inv[k]| into it as the bits of a non-negative float (the products
- * are exact in fp32, so the word is exact).  X device bf16 [M, K], smooth_inv device bf16 [K];
- * M >= 0 (M = 0 leaves 0), K % 64 == 0, X and smooth_inv 16-byte aligned, act_amax 4-byte aligned.
+ * svdq_act_amax writes amax = max |X[m,k] smooth_inv[k]| into word 0 of act_amax as the bits
+ * of a non-negative float (the products are exact in fp32, so the word is exact).  act_amax is
+ * a 16-byte device buffer that the caller zero-fills once, at allocation; each call leaves
+ * words 1-3 zero again (there is no clearing pass per call, and graph replays find it clean).
+ * X device bf16 [M, K], smooth_inv device bf16 [K]; M >= 0 (M = 0 writes 0), K % 64 == 0;
+ * X, smooth_inv and act_amax 16-byte aligned.  Calls sharing one act_amax must be stream-ordered.
  *
  * svdq_quantize_act_lowrank_down_dyn and svdq_w4a4_nvfp4_linear_dyn are the calls of kernels 1
- * and 2 with g_a read from act_amax on the device (after the previous kernel of the stream has
+ * and 2 with g_a read from word 0 of act_amax on the device (after the previous kernel of the stream has
  * finished) instead of passed in: the same outputs as the static calls given that g_a, and
  * lowrank_act holds U / g_a of that g_a.  Other arguments and errors as the static calls. */
 int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream);

@@ -236,7 +236,9 @@ def _run_svdq_dyn(P, X, smooth, packed, g_w, N):
     codes, scales, U = P.svdq_quantize_act_lowrank_down_dyn(Xd, sd, packed, amax)
     Y = P.svdq_w4a4_nvfp4_linear_dyn(codes, scales, U, amax, packed, g_w, M, N, K)
     torch.cuda.synchronize()
-    a = float(amax.view(torch.float32).cpu().item())
+    words = amax.cpu()
+    assert words[1] == 0 and words[2] == 0                              # left clean for the next call
+    a = float(words[:1].view(torch.float32).item())
     return a, codes, scales, U, Y
 
 
@@ -284,3 +286,35 @@ def test_dynamic_scale_full_attention_layer(P):
     check_output(Y.float().cpu().numpy()[rows],
                  svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, g))
     assert P.svdq_device_status() == 0
+
+
+def test_dynamic_scale_buffer_is_reused_cleanly_eager_and_in_graphs(P):
+    w = synth.svdq_workload(128, 256, 256)
+    s = _bf16_dev(w.smooth_inv)
+    buf = torch.zeros(4, dtype=torch.int32, device="cuda")
+    big, small = synth.to_bf16(w.X * 64.0), w.X
+
+    def amax_ref(X):
+        return np.max(np.abs(svdq.smooth(X, w.smooth_inv)))
+
+    def read():
+        torch.cuda.synchronize()
+        words = buf.cpu()
+        assert words[1] == 0 and words[2] == 0
+        return float(words[:1].view(torch.float32).item())
+
+    for X in (big, small, big, small):                     # a smaller batch after a larger one
+        P.svdq_act_amax(_bf16_dev(X), s, buf)
+        assert read() == amax_ref(X)
+    Xg = _bf16_dev(big)
+    g = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        P.svdq_act_amax(Xg, s, buf)                         # warm-up on the capture stream
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        P.svdq_act_amax(Xg, s, buf)
+    for X in (big, small, big):
+        Xg.copy_(_bf16_dev(X))
+        g.replay()
+        assert read() == amax_ref(X)
