@@ -87,6 +87,28 @@ def test_gpu_entry_points_reject_bad_arguments_before_any_device_work():
     assert L.awq_w4a16_linear(None, None, None, None, None, 0, 64, 256, None, None) == 0
 
 
+def test_dynamic_scale_entry_points_reject_bad_arguments_before_any_device_work():
+    L = P.LIB
+    odd2 = ctypes.c_void_p((1 << 20) + 2)
+    odd8 = ctypes.c_void_p((1 << 20) + 8)
+    # svdq_act_amax: the 16-byte amax buffer, K % 64, M >= 0, inputs present when M > 0
+    assert L.svdq_act_amax(FAKE, FAKE, 4, 64, None, None) == 1
+    assert L.svdq_act_amax(FAKE, FAKE, 4, 64, odd8, None) == 1
+    assert L.svdq_act_amax(FAKE, FAKE, 4, 96, FAKE, None) == 1
+    assert L.svdq_act_amax(FAKE, FAKE, -1, 64, FAKE, None) == 1
+    assert L.svdq_act_amax(None, FAKE, 4, 64, FAKE, None) == 1
+    # the *_dyn calls need the amax word (4-byte aligned); the static calls' checks apply otherwise
+    assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 64, 32, None, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 64, 32, odd2, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 96, 32, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, None, FAKE, 1.0, 4, 128, 64, 32, FAKE, None) == 1
+    assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, FAKE, FAKE, 0.3, 4, 128, 64, 32, FAKE, None) == 1
+    assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, FAKE, FAKE, 1.0, 4, 192, 64, 32, FAKE, None) == 2
+    # an empty batch is valid and needs no device
+    assert L.svdq_quantize_act_lowrank_down_dyn(None, None, None, 0, 64, 32, FAKE, None, None, None, None) == 0
+    assert L.svdq_w4a4_nvfp4_linear_dyn(None, None, None, FAKE, None, 1.0, 0, 128, 64, 32, None, None) == 0
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_a_device_reports_a_cuda_error():
     assert P.LIB.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 4
