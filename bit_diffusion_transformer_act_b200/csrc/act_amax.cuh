@@ -23,14 +23,23 @@
 namespace svdq {
 
 // Smallest power of two g with g * 2688 >= amax (2688 = 6 * 448), 1 for amax = 0.  Every
-// product g * 2688 is exact (2688 = 21 * 2^7), so the comparisons decide exactly.
+// product g * 2688 is exact (2688 = 21 * 2^7; an overflow to +inf compares correctly), so
+// the comparisons decide exactly.  The first guess from the rounded quotient is off by at
+// most one power of two, so two bounded correction steps each way suffice, and the function
+// ends for every input: NaN gives 1, +inf (an infinite activation) the largest power of two,
+// and amax below 2688 * 2^-126 (not supported) a wrong but finite scale.
 __device__ __forceinline__ float act_scale_from_amax(float amax) {
   if (!(amax > 0.f)) return 1.f;
+  if (isinf(amax)) return 0x1p127f;
   int e;
-  (void)frexpf(amax / 2688.f, &e);                 // a first guess within a factor of two
+  (void)frexpf(amax / 2688.f, &e);                 // amax / 2688 in [2^(e-1), 2^e), up to rounding
   float g = ldexpf(1.f, e);
-  while (g * 2688.f < amax) g *= 2.f;
-  while (g * (0.5f * 2688.f) >= amax) g *= 0.5f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (g * 2688.f < amax) g *= 2.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (g * (0.5f * 2688.f) >= amax) g *= 0.5f;
   return g;
 }
 
