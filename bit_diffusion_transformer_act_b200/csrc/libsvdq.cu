@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <numeric>
 #include <cmath>
 #include <mutex>
@@ -31,20 +32,23 @@ bool is_pow2_scale(float g) {
   return std::frexp(static_cast<double>(g), &e) == 0.5;
 }
 
-// Current device, checked to be compute capability 10.0 (cached per device).
+// Current device, checked to be compute capability 10.0 (cached per device; the caches of
+// this file are atomics, so calls from several host threads are safe).
 int current_device_ok(int* dev_out) {
-  static int cc_major[kMaxDevices], cc_minor[kMaxDevices];
-  static bool known[kMaxDevices];
+  static std::atomic<int> cc[kMaxDevices];         // 0: not yet known, else 100 major + minor + 1
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;
-  if (!known[dev]) {
-    if (cudaDeviceGetAttribute(&cc_major[dev], cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&cc_minor[dev], cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+  int v = cc[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return SVDQ_ERR_CUDA;
-    known[dev] = true;
+    v = 100 * major + minor + 1;
+    cc[dev].store(v, std::memory_order_release);
   }
-  if (cc_major[dev] != 10 || cc_minor[dev] != 0) return SVDQ_ERR_ARCH;
+  if (v != 100 * 10 + 0 + 1) return SVDQ_ERR_ARCH;
   *dev_out = dev;
   return SVDQ_OK;
 }
@@ -82,22 +86,23 @@ bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem
 // Raises the dynamic shared-memory limit of one kernel, once per device.
 template <auto Kernel>
 bool set_smem_once(int bytes, int dev) {
-  static bool done[kMaxDevices];
-  if (done[dev]) return true;
+  static std::atomic<bool> done[kMaxDevices];
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  // two threads may both get here: the attribute call is idempotent
   if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
-  done[dev] = true;
+  done[dev].store(true, std::memory_order_release);
   return true;
 }
 
 // Number of SMs of a device (cached).
 int sm_count(int dev) {
-  static int count[kMaxDevices];
-  if (count[dev] == 0) {
-    int c = 0;
+  static std::atomic<int> count[kMaxDevices];
+  int c = count[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-    count[dev] = c;
+    count[dev].store(c, std::memory_order_relaxed);
   }
-  return count[dev];
+  return c;
 }
 
 int launch_status() {
