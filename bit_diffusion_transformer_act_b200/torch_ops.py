@@ -114,6 +114,17 @@ class SvdqLinear(nn.Module):
                                              self.w_global_scale, self.out_features, self.rank)
         return y.reshape(*lead, self.out_features)
 
+    def get_extra_state(self):
+        # the per-tensor scales and sizes travel with state_dict() next to the buffers
+        return {"in_features": self.in_features, "out_features": self.out_features, "rank": self.rank,
+                "act_global_scale": self.act_global_scale, "w_global_scale": self.w_global_scale}
+
+    def set_extra_state(self, state):
+        self.in_features, self.out_features = int(state["in_features"]), int(state["out_features"])
+        self.rank = int(state["rank"])
+        self.act_global_scale = float(state["act_global_scale"])
+        self.w_global_scale = float(state["w_global_scale"])
+
     def extra_repr(self) -> str:
         return f"in_features={self.in_features}, out_features={self.out_features}, rank={self.rank}, nvfp4"
 

@@ -68,3 +68,14 @@ def test_swap_linears_replaces_selected_layers():
     assert names == ["0", "2.0", "2.1"]
     assert isinstance(model[0], T.AwqLinear) and isinstance(model[2][1], T.AwqLinear)
     assert isinstance(model[2][0], nn.Linear)
+
+
+def test_svdq_layer_state_dict_round_trip_keeps_the_scales():
+    a = T.SvdqLinear(512, 256, 32, torch.arange(1024, dtype=torch.int32).to(torch.uint8),
+                     torch.ones(512, dtype=torch.bfloat16), 0.5, 0.25)
+    b = T.SvdqLinear(64, 128, 32, torch.zeros(1024, dtype=torch.uint8), torch.zeros(512, dtype=torch.bfloat16),
+                     1.0, 1.0)
+    b.load_state_dict(a.state_dict())
+    assert (b.in_features, b.out_features, b.rank) == (512, 256, 32)
+    assert (b.act_global_scale, b.w_global_scale) == (0.5, 0.25)
+    assert torch.equal(b.packed_w, a.packed_w) and torch.equal(b.smooth_inv, a.smooth_inv)
