@@ -14,6 +14,8 @@ Everything is plain NumPy in float64, written from the definitions:
 * ``svdq``     the SVDQuant forward  y = Q4(X diag(lambda)^-1) Q4(R)^T
   + (X diag(lambda)^-1 L1) L2 + b.
 * ``awq``      the AWQ-style W4A16 group-64 dequantize-then-matmul forward.
+* ``qkv_epilogue``  the QKV projection's epilogue (per-head RMSNorm and RoPE of q and k),
+  the definition a fused epilogue kernel is to match.
 
 Sources: "Nunchaku Lite" (Hugging Face Diffusers documentation), section
 "Supported quantization types" (method table: svdq_w4a4 / nvfp4 / group 16,
