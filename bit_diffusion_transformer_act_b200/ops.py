@@ -78,12 +78,28 @@ def _np_ptr(a):
     return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
 
 
+def _on_device(t, name):
+    """Device calls take raw pointers: a host tensor (or one on another GPU) would be read as
+    device memory, so it is refused here, before the call."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index is not None and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
+
+
 def _require(t, dtype, shape, name):
     if not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected {dtype} tensor of shape {tuple(shape)}, got "
                          f"{getattr(t, 'dtype', type(t))} {tuple(getattr(t, 'shape', ()))}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    _on_device(t, name)
+
+
+def _require_blob(t, name, min_bytes=0):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_contiguous() or t.numel() < min_bytes:
+        raise ValueError(f"{name}: expected a contiguous uint8 tensor of at least {min_bytes} bytes")
+    _on_device(t, name)
 
 
 # ---------------------------------------------------------------- host side
@@ -160,6 +176,7 @@ def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, ra
     dev = X.device
     _require(X, torch.bfloat16, (M, K), "X")
     _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    _require_blob(packed_w, "packed_w")
     if act_codes is None:
         act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
     if act_scales is None:
@@ -179,6 +196,10 @@ def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, ra
 def svdq_w4a4_nvfp4_linear(act_codes, act_scales, lowrank_act, act_global_scale, packed_w, w_global_scale,
                            M, N, K, rank=RANK, Y=None):
     """Returns Y bf16 [M, N] = bf16(g_a g_w Q(X_hat) Q(R)^T + lowrank_act L2 + b)."""
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    _require_blob(packed_w, "packed_w", svdq_packed_weight_bytes(N, K, rank))
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
     _require(Y, torch.bfloat16, (M, N), "Y")
@@ -211,6 +232,8 @@ def svdq_quantize_act_lowrank_down_dyn(X, smooth_inv, packed_w, act_amax, rank=R
     dev = X.device
     _require(X, torch.bfloat16, (M, K), "X")
     _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    _require_blob(packed_w, "packed_w")
+    _require(act_amax, torch.int32, (4,), "act_amax")
     if act_codes is None:
         act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
     if act_scales is None:
@@ -230,6 +253,11 @@ def svdq_quantize_act_lowrank_down_dyn(X, smooth_inv, packed_w, act_amax, rank=R
 def svdq_w4a4_nvfp4_linear_dyn(act_codes, act_scales, lowrank_act, act_amax, packed_w, w_global_scale,
                                M, N, K, rank=RANK, Y=None):
     """As svdq_w4a4_nvfp4_linear with g_a formed on the device from act_amax."""
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    _require(act_amax, torch.int32, (4,), "act_amax")
+    _require_blob(packed_w, "packed_w", svdq_packed_weight_bytes(N, K, rank))
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
     _require(Y, torch.bfloat16, (M, N), "Y")

@@ -124,3 +124,27 @@ def test_swizzle_helpers_follow_the_documented_layout():
         assert np.array_equal(P.svdq_unswizzle_scales(sw, rows, K), plain)
     # one byte placed by hand: row 37 (lane 5 of quarter 1), group 6 (atom 1, slot 2), K = 128
     assert swizzled_offset(37, 6, 128) == 512 + 5 * 16 + 1 * 4 + 2
+
+
+def test_python_wrappers_refuse_host_tensors_before_calling_the_library():
+    # device calls take raw pointers: a host tensor must never reach a kernel
+    X = torch.zeros((4, 64), dtype=torch.bfloat16)
+    s = torch.zeros((64,), dtype=torch.bfloat16)
+    blob = torch.zeros((P.svdq_packed_weight_bytes(128, 64),), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P.svdq_quantize_act_lowrank_down(X, s, blob, 1.0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P.svdq_act_amax(X, s)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P.awq_w4a16_linear(X, torch.zeros((64, 32), dtype=torch.uint8), torch.zeros((64, 1), dtype=torch.bfloat16),
+                           torch.zeros((64, 1), dtype=torch.bfloat16))
+    codes = torch.zeros((4, 32), dtype=torch.uint8)
+    scales = torch.zeros((P.svdq_act_scale_bytes(4, 64),), dtype=torch.uint8)
+    low = torch.zeros((4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P.svdq_w4a4_nvfp4_linear(codes, scales, low, 1.0, blob, 1.0, 4, 128, 64)
+    # the guards' own checks (size and shape come before the device check)
+    with pytest.raises(ValueError, match="at least"):                  # a blob too short for N, K
+        P.ops._require_blob(blob[:100], "packed_w", P.svdq_packed_weight_bytes(128, 64))
+    with pytest.raises(ValueError, match="expected"):                  # codes of the wrong shape
+        P.ops._require(codes[:, :16], torch.uint8, (4, 32), "act_codes")
