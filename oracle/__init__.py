@@ -16,6 +16,8 @@ Everything is plain NumPy in float64, written from the definitions:
 * ``awq``      the AWQ-style W4A16 group-64 dequantize-then-matmul forward.
 * ``qkv_epilogue``  the QKV projection's epilogue (per-head RMSNorm and RoPE of q and k),
   the definition a fused epilogue kernel is to match.
+* ``mlp_epilogue``  the MLP up-projection's epilogue: GELU of the stored output, then the
+  down projection's activation pass (NVFP4 codes, scales, low-rank U) on the hidden state.
 
 Sources: "Nunchaku Lite" (Hugging Face Diffusers documentation), section
 "Supported quantization types" (method table: svdq_w4a4 / nvfp4 / group 16,

@@ -1,0 +1,42 @@
+"""Pins of the MLP epilogue oracle (GELU, then the down projection's activation pass)."""
+
+import math
+
+import numpy as np
+
+from oracle import mlp_epilogue as E
+from oracle import nvfp4, svdq
+import synth
+
+
+def test_gelu_closed_forms_exclude_the_tanh_approximation():
+    assert E.gelu(0.0) == 0.0
+    assert abs(E.gelu(1.0) - 0.8413447460685429) < 1e-15                 # Phi(1); tanh form gives 0.84119
+    assert abs(E.gelu(-1.0) + 0.15865525393145707) < 1e-15
+    assert E.gelu(10.0) == 10.0
+    x = np.linspace(-6, 6, 97)
+    assert np.allclose(E.gelu(x) - E.gelu(-x), x, rtol=0, atol=1e-14)     # x Phi(x) + x Phi(-x) = x
+
+
+def test_hidden_state_rounds_before_and_after_gelu():
+    y = np.array([1.0 + 2.0 ** -10])                                      # not a bf16 value
+    # bf16(y) = 1 -> GELU = 0.84134... -> bf16 0.83984375; without the first rounding it would be 0.84375
+    assert E.hidden_state(y)[0] == 0.83984375
+    assert E.hidden_state(np.array([0.0, -20.0, 20.0])).tolist() == [0.0, -0.0, 20.0]
+
+
+def test_requantize_applies_the_down_projection_smoothing_and_scale():
+    rng = np.random.default_rng(5)
+    M, F = 16, 256
+    y = synth.to_bf16(rng.standard_normal((M, F)) * 2.0)
+    L1 = synth.to_bf16(rng.standard_normal((F, 32)) * 0.1)
+    h = E.hidden_state(y)
+    s1 = np.ones(F)
+    g = nvfp4.global_scale(np.max(np.abs(h)))
+    c1, sc1, u1 = E.gelu_requantize(y, s1, g, L1)
+    # smoothing by 2^3 with the per-tensor scale times 2^3: the same codes and scales, U times 8
+    c8, sc8, u8 = E.gelu_requantize(y, s1 * 8.0, g * 8.0, L1)
+    assert np.array_equal(c1, c8) and np.array_equal(sc1, sc8)
+    assert np.allclose(u8, 8.0 * u1, rtol=1e-15)
+    cx, sx = svdq.quantize_activations(h, s1, g)
+    assert np.array_equal(c1, cx) and np.array_equal(sc1, sx)
