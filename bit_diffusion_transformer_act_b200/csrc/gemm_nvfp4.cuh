@@ -340,7 +340,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter .. +31
     const int ew = warp - 2;
-    const float alpha = p.amax ? act_scale_from_amax(__uint_as_float(*p.amax)) * p.w_scale : p.alpha;
+    float alpha = p.alpha;
+    if (p.amax) {
+      // the host checks g_a g_w for the static call; here it is formed on the device, so a
+      // product outside [2^-126, 2^126] is clamped and reported instead of refused
+      alpha = act_scale_from_amax(__uint_as_float(*p.amax)) * p.w_scale;
+      if (!(alpha >= 0x1p-126f && alpha <= 0x1p126f)) {
+        if (pair == 0 && threadIdx.x == 64) atomicOr(&g_device_status, 2u);
+        alpha = fminf(fmaxf(alpha, 0x1p-126f), 0x1p126f);
+      }
+    }
     const int eh = ew >> 2;                        // this warp takes every other chunk, starting at eh
     constexpr int NCW = C::NCH / 2;                // chunks per warp per tile
     uint8_t* sbias = gbase + C::OFF_BIAS + ew * 512;

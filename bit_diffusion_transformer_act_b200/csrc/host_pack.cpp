@@ -98,6 +98,7 @@ const char* svdq_status_string(int status) {
     case SVDQ_ERR_ARCH: return "device is not sm_100 (B200)";
     case SVDQ_ERR_CUDA: return "CUDA error";
     case SVDQ_ERR_TIMEOUT: return "kernel wait timed out";
+    case SVDQ_ERR_SCALE_RANGE: return "device-side scale product out of range (clamped)";
     default: return "unknown status";
   }
 }

@@ -424,7 +424,8 @@ int svdq_device_status(int clear) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(svdq::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SVDQ_ERR_CUDA;
   }
-  return (v & 1u) ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+  if (v & 1u) return SVDQ_ERR_TIMEOUT;
+  return (v & 2u) ? SVDQ_ERR_SCALE_RANGE : SVDQ_OK;
 }
 
 }  // extern "C"

@@ -11,7 +11,8 @@
 namespace svdq {
 
 // Device status word of this library (per device).  Bit 0: a bounded wait ran
-// out.  Higher bits record which wait site gave up first (for diagnostics).
+// out.  Bit 1: a scale product formed on the device was out of range and was
+// clamped.  Bits 8-15 record which wait site gave up (for diagnostics).
 __device__ unsigned int g_device_status = 0;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.

@@ -17,7 +17,7 @@ from .build import LIB_PATH
 RANK = 32
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device is not sm_100 (B200)",
-           4: "CUDA error", 5: "kernel wait timed out"}
+           4: "CUDA error", 5: "kernel wait timed out", 6: "device-side scale product out of range (clamped)"}
 
 
 class SvdqError(RuntimeError):
@@ -94,6 +94,14 @@ def _require(t, dtype, shape, name):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     _on_device(t, name)
+
+
+def _l1_section_end(K, rank):
+    """Bytes of the packed blob that the activation kernel reads: the 1 KB header and the
+    low-rank down factor section that follows it (two bf16 [rank, K] parts, hi and lo).  The C
+    call has no size argument, so this is the only guard against a blob that is too short
+    (or packed for a smaller K)."""
+    return 1024 + 4 * rank * K
 
 
 def _require_blob(t, name, min_bytes=0):
@@ -174,9 +182,9 @@ def svdq_quantize_act_lowrank_down(X, smooth_inv, packed_w, act_global_scale, ra
     lowrank_act bf16 [M, 2r] holding U / g_a as a high part then a low part)."""
     M, K = X.shape
     dev = X.device
+    _require_blob(packed_w, "packed_w", _l1_section_end(K, rank))
     _require(X, torch.bfloat16, (M, K), "X")
     _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
-    _require_blob(packed_w, "packed_w")
     if act_codes is None:
         act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
     if act_scales is None:
@@ -230,9 +238,9 @@ def svdq_quantize_act_lowrank_down_dyn(X, smooth_inv, packed_w, act_amax, rank=R
     """As svdq_quantize_act_lowrank_down with g_a formed on the device from act_amax."""
     M, K = X.shape
     dev = X.device
+    _require_blob(packed_w, "packed_w", _l1_section_end(K, rank))
     _require(X, torch.bfloat16, (M, K), "X")
     _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
-    _require_blob(packed_w, "packed_w")
     _require(act_amax, torch.int32, (4,), "act_amax")
     if act_codes is None:
         act_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)

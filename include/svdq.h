@@ -62,7 +62,8 @@ typedef enum {
   SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* a dimension outside the supported tiling */
   SVDQ_ERR_ARCH = 3,               /* current device is not compute capability 10.0 (B200) */
   SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or a launch failed */
-  SVDQ_ERR_TIMEOUT = 5             /* a kernel gave up on a bounded wait (see svdq_device_status) */
+  SVDQ_ERR_TIMEOUT = 5,            /* a kernel gave up on a bounded wait (see svdq_device_status) */
+  SVDQ_ERR_SCALE_RANGE = 6         /* a device-side g_a g_w left [2^-126, 2^126] (see svdq_device_status) */
 } svdq_status;
 
 /* Fixed parameters of the method table ("Supported quantization types"). */
@@ -168,7 +169,11 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
  * svdq_quantize_act_lowrank_down_dyn and svdq_w4a4_nvfp4_linear_dyn are the calls of kernels 1
  * and 2 with g_a read from word 0 of act_amax on the device (after the previous kernel of the stream has
  * finished) instead of passed in: the same outputs as the static calls given that g_a, and
- * lowrank_act holds U / g_a of that g_a.  Other arguments and errors as the static calls. */
+ * lowrank_act holds U / g_a of that g_a.  Other arguments and errors as the static calls, with one
+ * exception: the static call refuses a product g_a g_w outside [2^-126, 2^126] on the host, and the
+ * dynamic call, which forms it on the device, clamps it to that range instead and records
+ * SVDQ_ERR_SCALE_RANGE in the device status word (svdq_device_status), so the outputs are finite
+ * but wrong for such a batch.  (An infinite amax gives g_a = 2^127.) */
 int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream);
 int svdq_quantize_act_lowrank_down_dyn(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
                                        int rank, const void* act_amax, void* act_codes, void* act_scales,
@@ -204,8 +209,10 @@ int svdq_unswizzle_scales(const void* swizzled, int rows, int K, uint8_t* out);
 int svdq_swizzle_scales(const uint8_t* plain, int rows, int K, void* swizzled);
 
 /* Reads (and with clear != 0, resets) the device-side status word of the
- * current device that kernels set when a bounded wait runs out.  Returns
- * SVDQ_OK or SVDQ_ERR_TIMEOUT; SVDQ_ERR_CUDA if the read itself failed.
+ * current device that kernels set when a bounded wait runs out or a dynamic
+ * scale product is out of range.  Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (which
+ * wins when both happened) or SVDQ_ERR_SCALE_RANGE; SVDQ_ERR_CUDA if the read
+ * itself failed.
  * This call synchronizes the device; it is meant for tests and diagnostics. */
 int svdq_device_status(int clear);
 

@@ -31,8 +31,15 @@ def gelu(x):
 
 
 def hidden_state(y_up):
-    """h = bf16(GELU(bf16(y))): the hidden state as the unfused pipeline stores it (GELU of the
-    stored bf16 output, taken to fp32 -- where the pipeline computes it -- and stored as bf16)."""
+    """h = bf16(GELU(bf16(y))): the hidden state as the unfused pipeline stores it -- the up
+    projection's output rounded to bf16, its GELU evaluated here in float64 (essentially exact)
+    and rounded once to bf16.
+
+    A kernel that evaluates GELU in fp32 (a few ulp of error) rounds to the same bf16 value
+    except where the exact GELU lies within that error of a bf16 rounding midpoint, and there it
+    may land one bf16 ulp away.  The contract a fused kernel is held to is therefore stated on
+    its own intermediate values: its h is within one bf16 ulp of hidden_state(its own bf16 y),
+    and its codes and scales equal quantize_activations of its own h bit for bit."""
     return bf16_round(gelu(bf16_round(np.asarray(y_up, dtype=np.float64))))
 
 

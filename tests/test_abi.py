@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for s in range(6):
+    for s in range(7):
         assert P.LIB.svdq_status_string(s)
     assert P.LIB.svdq_status_string(99) == b"unknown status"
     assert P.LIB.svdq_abi_version() == 2
@@ -143,6 +143,19 @@ def test_python_wrappers_refuse_host_tensors_before_calling_the_library():
     low = torch.zeros((4, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         P.svdq_w4a4_nvfp4_linear(codes, scales, low, 1.0, blob, 1.0, 4, 128, 64)
+    # the activation calls read the blob's header and low-rank section (1 KB + 4 rank K bytes):
+    # a shorter blob is refused before any device call, in both the static and dynamic wrappers
+    short = torch.zeros((1024 + 4 * 32 * 64 - 16,), dtype=torch.uint8)
+    amax = torch.zeros((4,), dtype=torch.int32)
+    with pytest.raises(ValueError, match="at least 9216 bytes"):
+        P.svdq_quantize_act_lowrank_down(X, s, short, 1.0)
+    with pytest.raises(ValueError, match="at least 9216 bytes"):
+        P.svdq_quantize_act_lowrank_down_dyn(X, s, short, amax)
+    wide = torch.zeros((4, 128), dtype=torch.bfloat16)              # K = 128 needs 17408 bytes
+    with pytest.raises(ValueError, match="at least 17408 bytes"):
+        P.svdq_quantize_act_lowrank_down(wide, torch.zeros((128,), dtype=torch.bfloat16), blob[:9216], 1.0)
+    with pytest.raises(ValueError, match="CUDA tensor"):                # long enough: the device check follows
+        P.svdq_quantize_act_lowrank_down_dyn(X, s, short[:0].new_zeros(9216), amax)
     # the guards' own checks (size and shape come before the device check)
     with pytest.raises(ValueError, match="at least"):                  # a blob too short for N, K
         P.ops._require_blob(blob[:100], "packed_w", P.svdq_packed_weight_bytes(128, 64))

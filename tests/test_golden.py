@@ -1,5 +1,6 @@
-"""The oracle reproduces the fixtures under tests/golden/ (regression guard; see the README
-there -- these are not pins, the pins are the test_oracle_* tests).  Codes, scales and the
+"""The oracle reproduces the fixtures under tests/golden/ (a regression guard against unintended
+change of the oracle, written by make_golden.py from the oracle and the seeded generator only --
+these are not pins, the pins are the test_oracle_* tests).  Codes, scales and the
 per-tensor scales must match exactly; float64 outputs to 1e-12 relative (a matmul's last
 bits depend on the BLAS build)."""
 

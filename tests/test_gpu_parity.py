@@ -141,11 +141,25 @@ def test_repeat_calls_are_deterministic(P):
 
 # ---------------------------------------------------------------- full-size layers (sampled outputs)
 
+def sample_rows(M, seed, extra=128):
+    """Rows of a full-size output to check against the oracle: one random row from every
+    128-row half of every 256-row M tile (each CTA of a pair, each tile), the last row (the M
+    tail), and `extra` more random rows."""
+    rng = np.random.default_rng(seed)
+    rows = {int(rng.integers(lo, min(M, lo + 128))) for lo in range(0, M, 128)}
+    rows.add(M - 1)
+    rows.update(int(r) for r in rng.choice(M, size=min(M, extra), replace=False))
+    return np.array(sorted(rows))
+
+
 FULL = [
     ("attention 4096x3072->3072", 4096, 3072, 3072, False),
     ("mlp-up 4608x3072->12288", 4608, 3072, 12288, False),
     ("mlp-down 4608x12288->3072 (gelu)", 4608, 12288, 3072, True),
     ("qkv 64x3072->9216", 64, 3072, 9216, False),
+    ("qkv 256x3072->9216", 256, 3072, 9216, False),
+    ("qkv 1024x3072->9216", 1024, 3072, 9216, False),
+    ("qkv 4608x3072->9216", 4608, 3072, 9216, False),
     ("qkv 18432x3072->9216", 18432, 3072, 9216, False),
     # N not a multiple of 256: 192- and 128-wide output tiles, several per CTA pair
     ("192-wide tiles 8192x1024->1152", 8192, 1024, 1152, False),
@@ -158,8 +172,7 @@ def test_full_size_layer(P, name, M, K, N, gelu):
     w = synth.svdq_workload(M, K, N, gelu_input=gelu)
     packed, gw = _pack(P, w)
     codes, scales, U, Y = _run_svdq(P, w.X, w.smooth_inv, packed, w.g_a, gw, N)
-    rng = np.random.default_rng(11)
-    rows = np.sort(rng.choice(M, size=min(M, 256), replace=False))
+    rows = sample_rows(M, 11)
     # activation codes and scales: every row (bit-exact), low-rank on the sampled rows
     cx, sx = svdq.quantize_activations(w.X, w.smooth_inv, w.g_a)
     assert np.array_equal(codes, nvfp4.pack_nibbles(cx))
@@ -282,9 +295,39 @@ def test_dynamic_scale_full_attention_layer(P):
     cx, sx = svdq.quantize_activations(w.X, w.smooth_inv, g)
     assert np.array_equal(codes.cpu().numpy(), nvfp4.pack_nibbles(cx))
     assert np.array_equal(unswizzle(scales.cpu().numpy(), M, K)[:M], sx)
-    rows = np.sort(np.random.default_rng(12).choice(M, size=256, replace=False))
+    rows = sample_rows(M, 12)
     check_output(Y.float().cpu().numpy()[rows],
                  svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, g))
+    assert P.svdq_device_status() == 0
+
+
+def test_dynamic_scale_product_out_of_range_is_clamped_and_reported(P):
+    # g_a g_w formed on the device above 2^126: the GEMM clamps it and records the range status
+    # (the static call refuses such a product on the host).  X holds one 2^127 (amax = 2^127,
+    # g_a = 2^116) and R values near 2^22 (g_w = 2^11): the product is 2^127.
+    rng = np.random.default_rng(5)
+    M, K, N = 128, 256, 128
+    X = synth.to_bf16(rng.standard_normal((M, K)))
+    X[3, 17] = 2.0 ** 127
+    smooth = np.ones(K, np.float32)
+    R = (rng.standard_normal((N, K)) * 2.0 ** 20).astype(np.float32)
+    L1 = np.zeros((K, 32), np.float32)
+    L2 = np.zeros((32, N), np.float32)
+    blob, gw = P.svdq_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2), None, synth.bf16_bits(smooth))
+    assert gw == 2.0 ** 11
+    assert P.svdq_device_status() == 0
+    a, *_ = _run_svdq_dyn(P, X, smooth, torch.from_numpy(blob).cuda(), gw, N)
+    assert a == 2.0 ** 127
+    assert P.svdq_device_status(clear=True) == 6
+    assert P.svdq_device_status() == 0                                  # cleared
+    with pytest.raises(P.SvdqError):                                    # the static call refuses it
+        P.svdq_w4a4_nvfp4_linear(*P.svdq_quantize_act_lowrank_down(_bf16_dev(X), _bf16_dev(smooth),
+                                                                   torch.from_numpy(blob).cuda(), 2.0 ** 116),
+                                 2.0 ** 116, torch.from_numpy(blob).cuda(), gw, M, N, K)
+    # an in-range batch afterwards runs clean
+    w = synth.svdq_workload(128, 256, 256)
+    packed, gw2 = _pack(P, w)
+    _run_svdq_dyn(P, w.X, w.smooth_inv, packed, gw2, 256)
     assert P.svdq_device_status() == 0
 
 

@@ -40,3 +40,47 @@ def test_requantize_applies_the_down_projection_smoothing_and_scale():
     assert np.allclose(u8, 8.0 * u1, rtol=1e-15)
     cx, sx = svdq.quantize_activations(h, s1, g)
     assert np.array_equal(c1, cx) and np.array_equal(sc1, sx)
+
+
+def _gelu_decimal(x, digits=60):
+    """x Phi(x) from the Maclaurin series of erf in `digits`-digit decimal arithmetic (an
+    evaluation independent of math.erf, accurate far beyond float64 for |x| <= 8)."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = digits
+    X = Decimal(x)
+    # pi to 64 digits (a constant of mathematics)
+    pi = Decimal("3.141592653589793238462643383279502884197169399375105820974944592")
+    z = X / Decimal(2).sqrt()
+    term, total, n = z, z, 0
+    while True:
+        n += 1
+        term = -term * z * z / n
+        add = term / (2 * n + 1)
+        total += add
+        if abs(add) < Decimal(10) ** -(digits - 5):
+            break
+    erf = 2 * total / pi.sqrt()
+    return X * (1 + erf) / 2
+
+
+def test_hidden_state_rounds_the_exact_gelu_at_its_nearest_bf16_midpoint():
+    # Among all bf16 y with 2^-4 <= |y| <= 4, take the one whose GELU lies closest (relative) to
+    # a bf16 rounding midpoint: there an fp32 evaluation may round either way, and the oracle
+    # must take the side the exact value is on.
+    from decimal import Decimal
+    mags = np.array([m * 2.0 ** e for e in range(-4, 2) for m in np.arange(128, 256) / 128.0] + [4.0])
+    ys = np.concatenate([mags, -mags])
+    g = E.gelu(ys)
+    ulp = np.exp2(np.floor(np.log2(np.abs(g))) - 7)
+    frac = np.abs(g) / ulp - np.floor(np.abs(g) / ulp)
+    dist = np.abs(frac - 0.5) * ulp / np.abs(g)           # relative distance to the nearest midpoint
+    i = int(np.argmin(dist))
+    assert dist[i] < 2.0 ** -18                           # within reach of fp32 evaluation error
+    exact = _gelu_decimal(float(ys[i]))
+    lo = math.floor(abs(g[i]) / ulp[i]) * ulp[i]
+    mid = Decimal(lo) + Decimal(ulp[i]) / 2
+    up = abs(exact) > mid                                 # the side of the midpoint the exact value is on
+    expect = math.copysign(lo + ulp[i] if up else lo, g[i])
+    assert E.hidden_state(np.array([ys[i]]))[0] == expect
+    # and float64 agrees with the 60-digit evaluation to well below the distance
+    assert abs(Decimal(float(g[i])) - exact) < Decimal(float(dist[i] * abs(g[i]))) / 1000
