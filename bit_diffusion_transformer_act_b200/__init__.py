@@ -22,6 +22,7 @@ from .ops import (  # noqa: F401
     svdq_w4a4_nvfp4_linear,
     awq_w4a16_linear,
     svdq_act_amax,
+    svdq_act_amax_noalloc,
     svdq_quantize_act_lowrank_down_dyn,
     svdq_w4a4_nvfp4_linear_dyn,
     SvdqW4A4Linear,

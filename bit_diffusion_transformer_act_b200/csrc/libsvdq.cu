@@ -20,9 +20,17 @@
 #include "awq_w4a16.cuh"
 #include "awq_umma.cuh"
 
+// Scratch of svdq_act_amax_noalloc: kernel 5's result word, partial maximum and block
+// counter, for callers that cannot allocate device memory.  Every GPU that loads this
+// library holds these 256 bytes until the process exits; all calls on a device share them.
+static __device__ __align__(256) unsigned int g_amax_noalloc_scratch[64];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr size_t kAmaxScratchWords = 3;       // words of g_amax_noalloc_scratch kernel 5 uses
+static_assert(kAmaxScratchWords * sizeof(unsigned int) <= sizeof(g_amax_noalloc_scratch),
+              "kernel 5 needs three words whatever M and K are");
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -103,6 +111,25 @@ int sm_count(int dev) {
     count[dev].store(c, std::memory_order_relaxed);
   }
   return c;
+}
+
+// Device address of g_amax_noalloc_scratch on device `dev` (which must be current).  In host
+// code the array's name only stands for it: the address comes from cudaGetSymbolAddress, asked
+// once per device (by the first call on that device) and cached.
+int amax_noalloc_scratch(int dev, unsigned int** out) {
+  static std::atomic<uintptr_t> addr[kMaxDevices];
+  uintptr_t a = addr[dev].load(std::memory_order_acquire);
+  if (a == 0) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_amax_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    a = reinterpret_cast<uintptr_t>(p);
+    addr[dev].store(a, std::memory_order_release);   // two threads may both get here: same value
+  }
+  *out = reinterpret_cast<unsigned int*>(a);
+  return SVDQ_OK;
 }
 
 int launch_status() {
@@ -343,6 +370,45 @@ int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act
     return SVDQ_ERR_CUDA;
   }
   return launch_status();
+}
+
+// Kernel 5 with its scratch words in g_amax_noalloc_scratch instead of a caller buffer: the
+// scratch is cleared, the kernel runs on it, and its result word is copied to `amax`.  Nothing
+// is allocated.  Calls that overlap on the GPU share the scratch and race.
+int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, void* amax, void* stream) {
+  if (M < 0 || K <= 0 || K % 64 != 0) return SVDQ_ERR_INVALID_ARG;
+  if (!amax || (reinterpret_cast<uintptr_t>(amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
+  if (M > 0 && (!X || !smooth_inv || !aligned16(X) || !aligned16(smooth_inv))) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  unsigned int* scratch = nullptr;
+  if (int st = amax_noalloc_scratch(dev, &scratch)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the kernel expects its partial maximum and block counter at zero; it leaves them so, but a
+  // call is not to depend on what an earlier one left behind
+  if (cudaMemsetAsync(scratch, 0, kAmaxScratchWords * sizeof(unsigned int), s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  if (M > 0) {
+    namespace k5 = svdq::k5;
+    const int kv = K / 8;
+    const int q = kv / std::gcd(kv, k5::kThreads);
+    const size_t nvec = static_cast<size_t>(M) * kv;
+    const size_t want = (nvec + k5::kThreads - 1) / k5::kThreads;
+    const size_t cap = static_cast<size_t>(sm_count(dev)) * 8;
+    const int blocks = static_cast<int>(std::max<size_t>(q, std::min(want, cap) / q * q));
+    k5::act_amax_kernel<<<blocks, k5::kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X),
+                                                         static_cast<const __nv_bfloat16*>(smooth_inv), M, K,
+                                                         scratch);
+    if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+  }
+  // word 0: the result (0 for an empty batch, from the clearing above)
+  if (cudaMemcpyAsync(amax, scratch, sizeof(unsigned int), cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
 }
 
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, const void* zeros, const void* bias,

@@ -41,6 +41,7 @@ def _load():
         "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
         "awq_w4a16_linear": ([vp, vp, vp, vp, vp, i, i, i, vp, vp], i),
         "svdq_act_amax": ([vp, vp, i, i, vp, vp], i),
+        "svdq_act_amax_noalloc": ([vp, vp, i, i, vp, vp], i),
         "svdq_quantize_act_lowrank_down_dyn": ([vp, vp, vp, i, i, i, vp, vp, vp, vp, vp], i),
         "svdq_w4a4_nvfp4_linear_dyn": ([vp, vp, vp, vp, vp, f, i, i, i, i, vp, vp], i),
         "svdq_unswizzle_scales": ([vp, i, i, vp], i),
@@ -58,7 +59,8 @@ LIB = _load()
 EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes", "svdq_pack_weights",
             "svdq_act_scale_bytes", "svdq_quantize_act_lowrank_down", "svdq_w4a4_nvfp4_linear",
             "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status",
-            "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn")
+            "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn",
+            "svdq_act_amax_noalloc")
 
 
 def _check(fn, st):
@@ -231,6 +233,19 @@ def svdq_act_amax(X, smooth_inv, act_amax=None):
     st = LIB.svdq_act_amax(_ptr(X), _ptr(smooth_inv), M, K, _ptr(act_amax), _stream())
     _check("svdq_act_amax", st)
     return act_amax
+
+
+def svdq_act_amax_noalloc(X, smooth_inv, amax):
+    """max |X smooth_inv| into `amax` (a float32 [1] CUDA tensor), through the C call that
+    allocates nothing (its scratch is the library's own static array; calls must not overlap
+    on the GPU)."""
+    M, K = X.shape
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    _require(amax, torch.float32, (1,), "amax")
+    st = LIB.svdq_act_amax_noalloc(_ptr(X), _ptr(smooth_inv), M, K, _ptr(amax), _stream())
+    _check("svdq_act_amax_noalloc", st)
+    return amax
 
 
 def svdq_quantize_act_lowrank_down_dyn(X, smooth_inv, packed_w, act_amax, rank=RANK,

@@ -182,6 +182,30 @@ int svdq_w4a4_nvfp4_linear_dyn(const void* act_codes, const void* act_scales, co
                                const void* act_amax, const void* packed_w, float w_global_scale, int M, int N, int K,
                                int rank, void* Y, void* stream);
 
+/* The amax of svdq_act_amax for callers that cannot allocate device memory -- code that runs
+ * where cudaMalloc is not allowed or not wanted: inside an inference engine or plugin whose
+ * memory is planned up front by the host application, in a real-time path that must not call
+ * into the allocator, or under a caching allocator that does not own this library's buffers.
+ * The pages describe no such call; it is a convenience of this library with no counterpart
+ * there.
+ *
+ * Writes max |X[m,k] smooth_inv[k]| (the bits of a non-negative float, exact, as svdq_act_amax
+ * writes into its word 0) to the 4-byte device word `amax`, which the caller passes like any
+ * other output; M = 0 writes 0.  The kernel's scratch (its result, partial maximum and block
+ * counter: three 32-bit words, whatever M and K are) lives in a 256-byte array that the
+ * library holds on every GPU that loads it, until the process exits; since no M or K needs
+ * more than those three words, no size is refused for want of scratch.  The call clears the
+ * scratch before its kernel, then copies the result out; it calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - The first call on a device looks up the array's device address there (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array: calls whose work overlaps on the GPU (other
+ *     streams, or other host threads, without ordering between them) race and give wrong
+ *     results.  Order them on one stream.
+ * X device bf16 [M, K], smooth_inv device bf16 [K]; M >= 0, K % 64 == 0; X and smooth_inv
+ * 16-byte aligned, amax 4-byte aligned.  Errors as svdq_act_amax.  Asynchronous on `stream`. */
+int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, void* amax, void* stream);
+
 /* ---------------------------------------------------------------- AWQ W4A16 */
 
 /* y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.  M <= 8 runs the

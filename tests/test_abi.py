@@ -97,6 +97,13 @@ def test_dynamic_scale_entry_points_reject_bad_arguments_before_any_device_work(
     assert L.svdq_act_amax(FAKE, FAKE, 4, 96, FAKE, None) == 1
     assert L.svdq_act_amax(FAKE, FAKE, -1, 64, FAKE, None) == 1
     assert L.svdq_act_amax(None, FAKE, 4, 64, FAKE, None) == 1
+    # svdq_act_amax_noalloc: a 4-byte-aligned result word, the same size and input checks
+    assert L.svdq_act_amax_noalloc(FAKE, FAKE, 4, 64, None, None) == 1
+    assert L.svdq_act_amax_noalloc(FAKE, FAKE, 4, 64, odd2, None) == 1
+    assert L.svdq_act_amax_noalloc(FAKE, FAKE, 4, 96, FAKE, None) == 1
+    assert L.svdq_act_amax_noalloc(FAKE, FAKE, -1, 64, FAKE, None) == 1
+    assert L.svdq_act_amax_noalloc(None, FAKE, 4, 64, FAKE, None) == 1
+    assert L.svdq_act_amax_noalloc(FAKE, odd8, 4, 64, FAKE, None) == 1
     # the *_dyn calls need the amax word (4-byte aligned); the static calls' checks apply otherwise
     assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 64, 32, None, FAKE, FAKE, FAKE, None) == 1
     assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 64, 32, odd2, FAKE, FAKE, FAKE, None) == 1
