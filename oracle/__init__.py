@@ -14,6 +14,8 @@ Everything is plain NumPy in float64, written from the definitions:
 * ``svdq``     the SVDQuant forward  y = Q4(X diag(lambda)^-1) Q4(R)^T
   + (X diag(lambda)^-1 L1) L2 + b.
 * ``awq``      the AWQ-style W4A16 group-64 dequantize-then-matmul forward.
+* ``int4``     the svdq_w4a4 int4 / group-64 row: signed 4-bit codes with a bf16 scale
+  (amax / 7, rounded once) per 64 K elements on both operands, the same low-rank branch.
 * ``qkv_epilogue``  the QKV projection's epilogue (per-head RMSNorm and RoPE of q and k),
   the definition a fused epilogue kernel is to match.
 * ``mlp_epilogue``  the MLP up-projection's epilogue: GELU of the stored output, then the
@@ -37,4 +39,4 @@ No worked numeric example exists on the pages, so parity with the pages' own
 kernels is unpinned beyond those invariants.
 """
 
-from . import formats, nvfp4, svdq, awq  # noqa: F401
+from . import formats, nvfp4, svdq, awq, int4  # noqa: F401
