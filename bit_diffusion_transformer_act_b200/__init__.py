@@ -20,6 +20,9 @@ from .ops import (  # noqa: F401
     svdq_device_status,
     svdq_quantize_act_lowrank_down,
     svdq_w4a4_nvfp4_linear,
+    svdq_w4a4_nvfp4_linear_qkv,
+    svdq_w4a4_nvfp4_linear_gelu_quant,
+    svdq_gelu_quant_workspace_bytes,
     awq_w4a16_linear,
     svdq_act_amax,
     svdq_act_amax_noalloc,

@@ -47,9 +47,10 @@ constexpr int BK = 256;                    // K elements per pipeline stage
 constexpr int kEpiWarps = 8;                // two per tensor-memory lane quarter
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 
-template <int BN>
+template <int BN, bool QKV = false>
 struct Cfg {
   static_assert(BN == 128 || BN == 192 || BN == 256, "tile width");
+  static_assert(!QKV || BN != 192, "the QKV epilogue's tiles hold whole 128-column heads");
   static constexpr int BN_HALF = BN / 2;                       // B rows staged by each CTA
   static constexpr int SFB_ATOMS = BN == 128 ? 1 : 2;          // 128-row scale blocks spanned by a tile
   static constexpr int A_BYTES = BM * BK / 2;
@@ -84,7 +85,9 @@ struct Cfg {
   static constexpr int NUM_BARS = NBF + STAGES + 5;            // full[NBF], empty, acc_full[2], acc_empty[2], drain
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;  // per epilogue warp: the tile's bias (BN bf16)
-  static constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * 512 + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 32 bf16
+  static constexpr int OFF_NW = OFF_BIAS + kEpiWarps * 512;    // QKV epilogue, per epilogue warp: q and k norm weights
+  static constexpr int NW_BYTES = QKV ? kEpiWarps * 512 : 0;
+  static constexpr int OFF_STAGE = (OFF_NW + NW_BYTES + 1023) / 1024 * 1024;  // per epilogue warp: 32 x 32 bf16
   static constexpr int SMEM_BYTES = OFF_STAGE + kEpiWarps * 2048 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TX_MAIN = 2u * STAGE_BYTES;        // bytes landing per stage, both CTAs
   static constexpr uint32_t TX_LOWRANK = 2u * (UCAT_BYTES + L2_BYTES);
@@ -108,6 +111,14 @@ struct Params {
   float alpha;                     // g_a g_w
   const unsigned int* amax;        // or, if not null, g_a from this amax word (kernel 5) ...
   float w_scale;                   // ... times g_w
+  // QKV epilogue (the kQkv instantiation): q, k, v thirds of `third` columns each (heads x 128);
+  // q and k RMS-normalised per 128-column head and rotated by RoPE
+  const __nv_bfloat16* norm_wq;    // [128]
+  const __nv_bfloat16* norm_wk;    // [128]
+  const float* rope_cos;           // [64, M]: cos of the angle of pair i (dims 2i, 2i + 1) of token m at [i][m]
+  const float* rope_sin;           // [64, M]
+  float eps;
+  int third;
 };
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
@@ -151,13 +162,13 @@ __device__ __forceinline__ void epilogue_stage32(const uint32_t (&r)[32], const 
                  : "memory");
 }
 
-template <int BN>
+template <int BN, bool kQkv = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
                   const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, kQkv>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -357,6 +368,160 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const uint32_t stage_row = stage_tile + lane * 64;                      // this lane's staging row
     const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
     int i = 0;
+    if constexpr (kQkv) {
+      // ---------------------------------------------------------------- QKV epilogue
+      // A warp owns one 128-column head of its 32 rows (BN = 256: the tile's head eh; BN = 128:
+      // the tile's one head, taken by the eh = 0 warps while their partners only hand the
+      // accumulator back), so RMSNorm's sum of squares and RoPE's pairs stay in one thread.
+      // Two passes over the head's four 32-column chunks of tensor memory: the sum of squares,
+      // then one chunk at a time (norm weight, rotation, bf16 into the warp's staging tile, one
+      // TMA store) with the next chunk's cos / sin loads in flight -- 32 accumulator registers
+      // live instead of 128.  The tables are pair-major, so a warp's load of one pair covers
+      // its 32 consecutive tokens in one 128-byte line.
+      uint8_t* snw = gbase + C::OFF_NW + ew * 512;                          // q weights, then k weights
+      {
+        const __nv_bfloat16* src = lane < 16 ? p.norm_wq : p.norm_wk;
+        *reinterpret_cast<uint4*>(snw + lane * 16) = __ldg(reinterpret_cast<const uint4*>(src) + (lane & 15));
+        __syncwarp();
+      }
+      const bool active = BN == 256 || eh == 0;
+      const int hcol = BN == 256 ? eh * 128 : 0;                            // the head's first tile column
+      for (int t = pair; t < p.tiles; t += npairs, ++i) {
+        const int mt = t / p.tiles_n, nt = t % p.tiles_n;
+        const int m0 = mt * 256 + static_cast<int>(cta) * BM + quarter * 32;
+        const int n0 = nt * BN;
+        const int b = i & 1;
+        const int ab = C::ACC_STAGES == 2 ? b : 0;
+        const int use = C::ACC_STAGES == 2 ? (i >> 1) : i;
+        const int part = (n0 + hcol) / p.third;    // 0 q, 1 k, 2 v (a tile never straddles two)
+        const bool live = active && m0 < p.M;      // warp-uniform
+        const int m = min(m0 + lane, p.M - 1);
+        // Order of the head's four chunks in the second pass, and the point of release.  With
+        // overlapping buffers (BN = 256) the next tile overwrites buffer 0's columns ACC1..255
+        // (head 1's chunks 1-3) or buffer 1's first 256 - ACC1 columns (head 0's chunks 0-2):
+        // the warp holding them reads those first and hands the accumulator back once they
+        // are in registers; the other warp hands it back after the first pass.  With two
+        // separate buffers (BN = 128) the accumulator is handed back after the last read.
+        const bool shared = BN == 256 && ((b == 0 && eh == 1) || (b == 1 && eh == 0));
+        const int first = (BN == 256 && b == 0 && eh == 1) ? 1 : 0;
+        auto chunk_of = [&](int jj) { return (first + jj) & 3; };
+        const int rel_after = BN == 256 ? (shared ? 2 : -1) : 3;   // pass-2 position after whose read to release
+        if (lane < BN / 8)
+          *reinterpret_cast<uint4*>(sbias + lane * 16) = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
+        __syncwarp();
+        // the rotation tables of the first chunk do not depend on the accumulator
+        float tc[16], ts[16];
+        const float* ccol = p.rope_cos + m;        // pair i of token m at [i * M + m]
+        const float* scol = p.rope_sin + m;
+        auto load_tables = [&](int j, float (&c)[16], float (&sn)[16]) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            c[x] = __ldg(ccol + static_cast<size_t>(16 * j + x) * p.M);
+            sn[x] = __ldg(scol + static_cast<size_t>(16 * j + x) * p.M);
+          }
+        };
+        if (live && part < 2) load_tables(chunk_of(0), tc, ts);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(ab), use & 1, abort_flag, 4))) break;
+        tc_fence_after();
+        const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                              static_cast<uint32_t>(b * C::ACC1 + hcol);
+        auto release = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(map_to_cta(acc_empty(ab), 0));
+        };
+        if (!live) {
+          release();
+          continue;
+        }
+        const uint4* bh = reinterpret_cast<const uint4*>(sbias + hcol * 2);
+        // y = alpha acc + b for 32 columns (chunk j of the head), in place
+        auto affine = [&](uint32_t (&r)[32], int j) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 bv = bh[j * 4 + q];
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int k = q * 8 + w * 2;
+              r[k] = __float_as_uint(fmaf(alpha, __uint_as_float(r[k]), bf16lo_to_f32(bw[w])));
+              r[k + 1] = __float_as_uint(fmaf(alpha, __uint_as_float(r[k + 1]), bf16hi_to_f32(bw[w])));
+            }
+          }
+        };
+        // first pass (q and k): the head's sum of squares, two chunks at a time
+        float rinv = 1.f;
+        if (part < 2) {
+          float ss = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            uint32_t A[32], B[32];
+            tmem_ld_32x32b_x32(trow + 32u * j, A);
+            tmem_ld_32x32b_x32(trow + 32u * (j + 1), B);
+            tmem_wait_ld_regs(A);
+            tmem_wait_ld_regs(B);
+            affine(A, j);
+            affine(B, j + 1);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              ss = fmaf(__uint_as_float(A[k]), __uint_as_float(A[k]), ss);
+              ss = fmaf(__uint_as_float(B[k]), __uint_as_float(B[k]), ss);
+            }
+          }
+          rinv = rsqrtf(ss * (1.0f / 128.0f) + p.eps);
+        }
+        if (rel_after < 0) release();
+        const uint32_t* wn = reinterpret_cast<const uint32_t*>(snw + (part == 1 ? 256 : 0));
+        // second pass: one chunk at a time, the next chunk's tables in flight meanwhile
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = chunk_of(jj);
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + 32u * j, r);
+          float nc[16], ns[16];
+          if (part < 2 && jj + 1 < 4) load_tables(chunk_of(jj + 1), nc, ns);
+          tmem_wait_ld_regs(r);
+          if (jj == rel_after) release();
+          affine(r, j);
+          if (part < 2) {
+            // RMSNorm weight, then the rotation of pairs 16 j .. 16 j + 15
+#pragma unroll
+            for (int pr = 0; pr < 16; ++pr) {
+              const uint32_t ww = wn[16 * j + pr];                            // weights of dims 2 pr, 2 pr + 1
+              const float x0 = __uint_as_float(r[2 * pr]) * rinv * bf16lo_to_f32(ww);
+              const float x1 = __uint_as_float(r[2 * pr + 1]) * rinv * bf16hi_to_f32(ww);
+              r[2 * pr] = __float_as_uint(fmaf(x0, tc[pr], -x1 * ts[pr]));
+              r[2 * pr + 1] = __float_as_uint(fmaf(x0, ts[pr], x1 * tc[pr]));
+            }
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              tc[x] = nc[x];
+              ts[x] = ns[x];
+            }
+          }
+          // bf16 into the staging tile (once the previous store from it has read it), one TMA store
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          {
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = pack_bf16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                           ::"r"(stage_row + ((static_cast<uint32_t>(q) ^ sw) << 4)), "r"(o[q * 4]), "r"(o[q * 4 + 1]),
+                             "r"(o[q * 4 + 2]), "r"(o[q * 4 + 3])
+                           : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, stage_tile, n0 + hcol + 32 * j, m0);
+            bulk_commit_group();
+          }
+        }
+      }
+    } else
     for (int t = pair; t < p.tiles; t += npairs, ++i) {
       const int mt = t / p.tiles_n, nt = t % p.tiles_n;
       const int m0 = mt * 256 + static_cast<int>(cta) * BM + quarter * 32;   // this warp's first row

@@ -19,6 +19,7 @@
 #include "gemm_nvfp4.cuh"
 #include "awq_w4a16.cuh"
 #include "awq_umma.cuh"
+#include "gemm_gelu_quant.cuh"
 
 // Scratch of svdq_act_amax_noalloc: kernel 5's result word, partial maximum and block
 // counter, for callers that cannot allocate device memory.  Every GPU that loads this
@@ -229,11 +230,22 @@ int svdq_quantize_act_lowrank_down_dyn(const void* X, const void* smooth_inv, co
                        stream);
 }
 
+// The QKV epilogue's extra arguments (svdq_w4a4_nvfp4_linear_qkv).
+struct QkvArgs {
+  int heads;
+  const void* norm_wq;
+  const void* norm_wk;
+  float eps;
+  const void* rope_cos;
+  const void* rope_sin;
+};
+
 // Kernel 2 with the activation scale given (act_amax null) or formed on the device from the
-// amax word of kernel 5.
+// amax word of kernel 5; with qkv non-null, the instantiation whose epilogue normalises and
+// rotates q and k.
 static int linear_impl(const void* act_codes, const void* act_scales, const void* lowrank_act,
                        float act_global_scale, const void* act_amax, const void* packed_w, float w_global_scale,
-                       int M, int N, int K, int rank, void* Y, void* stream) {
+                       int M, int N, int K, int rank, void* Y, void* stream, const QkvArgs* qkv = nullptr) {
   if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_scale(w_global_scale)) return SVDQ_ERR_INVALID_ARG;
   if (!act_amax && !is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
@@ -253,7 +265,19 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   namespace k2 = svdq::k2;
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
-  const int BN = (N % 256 == 0) ? 256 : (N % 192 == 0 ? 192 : 128);
+  // Output tile width: the widest that divides N, unless at this M its tiles would leave CTA
+  // pairs idle (few rows: the kernel is bound by streaming the weights, and every pair should
+  // stream its share) -- then the width giving the most tiles up to one per pair.
+  const int mtiles = (M + 255) / 256;
+  const int npairs = sm_count(dev) / 2;
+  int BN = (N % 256 == 0) ? 256 : (N % 192 == 0 ? 192 : 128);
+  if (qkv) BN = ((N / 3) % 256 == 0) ? 256 : 128;      // whole heads per tile, q/k/v thirds never straddled
+  if (mtiles * (N / BN) < npairs) {
+    for (int bn : {192, 128}) {
+      if (qkv && bn == 192) continue;
+      if (bn < BN && N % bn == 0 && mtiles * (N / bn) <= npairs && mtiles * (N / bn) > mtiles * (N / BN)) BN = bn;
+    }
+  }
   k2::Params p;
   p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
@@ -265,6 +289,18 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   p.alpha = static_cast<float>(alpha);
   p.amax = static_cast<const unsigned int*>(act_amax);
   p.w_scale = w_global_scale;
+  p.norm_wq = p.norm_wk = nullptr;
+  p.rope_cos = p.rope_sin = nullptr;
+  p.eps = 0.f;
+  p.third = N;
+  if (qkv) {
+    p.norm_wq = static_cast<const __nv_bfloat16*>(qkv->norm_wq);
+    p.norm_wk = static_cast<const __nv_bfloat16*>(qkv->norm_wk);
+    p.rope_cos = static_cast<const float*>(qkv->rope_cos);
+    p.rope_sin = static_cast<const float*>(qkv->rope_sin);
+    p.eps = qkv->eps;
+    p.third = N / 3;
+  }
 
   const int natoms = K / 64;
   const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
@@ -288,10 +324,10 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   const int pairs = std::min(p.tiles, sm_count(dev) / 2);
   const dim3 grid(2 * pairs, 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-#define SVDQ_GEMM_LAUNCH(BN_)                                                                       \
+#define SVDQ_GEMM_LAUNCH(BN_, QKV_)                                                                 \
   do {                                                                                              \
-    const int smem = k2::Cfg<BN_>::SMEM_BYTES;                                                      \
-    if (!set_smem_once<k2::nvfp4_gemm_kernel<BN_>>(smem, dev)) return SVDQ_ERR_CUDA;                \
+    const int smem = k2::Cfg<BN_, QKV_>::SMEM_BYTES;                                                \
+    if (!set_smem_once<k2::nvfp4_gemm_kernel<BN_, QKV_>>(smem, dev)) return SVDQ_ERR_CUDA;          \
     cudaLaunchConfig_t cfg = {};                                                                    \
     cfg.gridDim = grid;                                                                             \
     cfg.blockDim = dim3(k2::kThreads, 1, 1);                                                        \
@@ -302,15 +338,22 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
     attr[0].val.programmaticStreamSerializationAllowed = 1;                                         \
     cfg.attrs = attr;                                                                               \
     cfg.numAttrs = 1;                                                                               \
-    if (cudaLaunchKernelEx(&cfg, k2::nvfp4_gemm_kernel<BN_>, tA, tB, tSFA, tSFB, tU, tL2, tY, p) !=  \
+    if (cudaLaunchKernelEx(&cfg, k2::nvfp4_gemm_kernel<BN_, QKV_>, tA, tB, tSFA, tSFB, tU, tL2, tY, p) != \
         cudaSuccess) {                                                                              \
       (void)cudaGetLastError();                                                                     \
       return SVDQ_ERR_CUDA;                                                                         \
     }                                                                                               \
   } while (0)
-  if (BN == 192) SVDQ_GEMM_LAUNCH(192);
-  else if (BN == 256) SVDQ_GEMM_LAUNCH(256);
-  else SVDQ_GEMM_LAUNCH(128);
+  if (qkv) {
+    if (BN == 256) SVDQ_GEMM_LAUNCH(256, true);
+    else SVDQ_GEMM_LAUNCH(128, true);
+  } else if (BN == 192) {
+    SVDQ_GEMM_LAUNCH(192, false);
+  } else if (BN == 256) {
+    SVDQ_GEMM_LAUNCH(256, false);
+  } else {
+    SVDQ_GEMM_LAUNCH(128, false);
+  }
 #undef SVDQ_GEMM_LAUNCH
   return launch_status();
 }
@@ -328,6 +371,145 @@ int svdq_w4a4_nvfp4_linear_dyn(const void* act_codes, const void* act_scales, co
   if (!act_amax) return SVDQ_ERR_INVALID_ARG;
   return linear_impl(act_codes, act_scales, lowrank_act, 1.0f, act_amax, packed_w, w_global_scale, M, N, K, rank, Y,
                      stream);
+}
+
+int svdq_w4a4_nvfp4_linear_qkv(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                               float act_global_scale, const void* packed_w, float w_global_scale, int M, int N,
+                               int K, int rank, int heads, int head_dim, const void* norm_wq, const void* norm_wk,
+                               float eps, const void* rope_cos, const void* rope_sin, void* Y, void* stream) {
+  if (heads <= 0 || head_dim <= 0 || !(eps >= 0.f) || !std::isfinite(eps)) return SVDQ_ERR_INVALID_ARG;
+  if (head_dim != 128 || N != 3 * heads * head_dim) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M > 0) {
+    if (!norm_wq || !norm_wk || !rope_cos || !rope_sin) return SVDQ_ERR_INVALID_ARG;
+    if (!aligned16(norm_wq) || !aligned16(norm_wk) || !aligned16(rope_cos) || !aligned16(rope_sin))
+      return SVDQ_ERR_INVALID_ARG;
+  }
+  const QkvArgs q{heads, norm_wq, norm_wk, eps, rope_cos, rope_sin};
+  return linear_impl(act_codes, act_scales, lowrank_act, act_global_scale, nullptr, packed_w, w_global_scale, M, N,
+                     K, rank, Y, stream, &q);
+}
+
+// Tile partition of kernel 6: pairs, and the partial slots per pair (row blocks a pair's
+// contiguous range of the row-major tile order can touch).
+static void gelu_quant_partition(int M, int N, int dev, int* npairs, int* slots) {
+  const int tiles_n = N / svdq::k6::BN;
+  const int tiles = ((M + 255) / 256) * tiles_n;
+  const int P = std::max(1, std::min(tiles, sm_count(dev) / 2));
+  int sl = 1;
+  for (int p = 0; p < P; ++p) {
+    const int a = svdq::k6::range_start(p, tiles, P), b = svdq::k6::range_start(p + 1, tiles, P);
+    if (b > a) sl = std::max(sl, (b - 1) / tiles_n - a / tiles_n + 1);
+  }
+  *npairs = P;
+  *slots = sl;
+}
+
+size_t svdq_gelu_quant_workspace_bytes(int M, int N) {
+  if (M <= 0 || N <= 0 || N % 128 != 0) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  int P, slots;
+  gelu_quant_partition(M, N, dev, &P, &slots);
+  return static_cast<size_t>(P) * slots * 256 * 32 * sizeof(float);
+}
+
+int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                                      float act_global_scale, const void* packed_w, float w_global_scale, int M,
+                                      int N, int K, int rank, const void* down_smooth_inv, const void* down_packed_w,
+                                      float down_act_global_scale, void* out_codes, void* out_scales,
+                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes, void* h_out,
+                                      void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_scale(act_global_scale) || !is_pow2_scale(w_global_scale) || !is_pow2_scale(down_act_global_scale))
+    return SVDQ_ERR_INVALID_ARG;
+  if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  const double alpha = static_cast<double>(act_global_scale) * w_global_scale;
+  if (!(alpha >= 0x1p-126 && alpha <= 0x1p126)) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!act_codes || !act_scales || !lowrank_act || !packed_w || !down_smooth_inv || !down_packed_w || !out_codes ||
+      !out_scales || !out_lowrank_act || !workspace)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
+      !aligned16(down_smooth_inv) || !aligned16(down_packed_w) || !aligned16(out_codes) || !aligned16(out_scales) ||
+      !aligned16(out_lowrank_act) || !aligned16(workspace) || (h_out && !aligned16(h_out)))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  namespace k6 = svdq::k6;
+  int P, slots;
+  gelu_quant_partition(M, N, dev, &P, &slots);
+  if (workspace_bytes < static_cast<size_t>(P) * slots * 256 * 32 * sizeof(float)) return SVDQ_ERR_INVALID_ARG;
+
+  const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
+  const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
+  const svdq::BlobLayout LD = svdq::blob_layout(0, N, rank);   // the down blob's L1 section (its K is N)
+  k6::Params p;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
+  p.smooth = static_cast<const __nv_bfloat16*>(down_smooth_inv);
+  p.codes = static_cast<uint8_t*>(out_codes);
+  p.scales = static_cast<uint8_t*>(out_scales);
+  p.ws = static_cast<float*>(workspace);
+  p.h_out = static_cast<__nv_bfloat16*>(h_out);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_n = N / k6::BN;
+  p.tiles = ((M + 255) / 256) * p.tiles_n;
+  p.slots = slots;
+  p.alpha = static_cast<float>(alpha);
+  p.g = down_act_global_scale;
+  p.inv_g = 1.0f / down_act_global_scale;         // exact: a power of two
+
+  const int natoms = K / 64;
+  const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
+  const uint64_t sfb_rows = static_cast<uint64_t>(N / 128) * natoms;
+  CUtensorMap tA, tB, tSFA, tSFB, tU, tL2, tL1;
+  if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, 128, k6::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, k6::BN_HALF,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tSFA, act_scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, sfa_rows, 128, 128, k6::BK / 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap(&tSFB, blob + L.scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, sfb_rows, 128, 128, k6::BK / 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, 2 * rank, 2 * rank, k6::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, k6::BN_HALF,
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_tmap(&tL1, static_cast<const uint8_t*>(down_packed_w) + LD.l1s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                 2 * rank, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  if (!set_smem_once<k6::gemm_gelu_quant_kernel>(k6::SMEM_BYTES, dev)) return SVDQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * P, 1, 1);
+  cfg.blockDim = dim3(k6::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = k6::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k6::gemm_gelu_quant_kernel, tA, tB, tSFA, tSFB, tU, tL2, tL1, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg2 = {};
+  cfg2.gridDim = dim3((M * 8 + 255) / 256, 1, 1);
+  cfg2.blockDim = dim3(256, 1, 1);
+  cfg2.stream = s;
+  cfg2.attrs = attr;
+  cfg2.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg2, k6::u_reduce_kernel, static_cast<const float*>(workspace), M, p.tiles_n, p.tiles, P,
+                         slots, p.inv_g, static_cast<__nv_bfloat16*>(out_lowrank_act)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 int svdq_act_amax(const void* X, const void* smooth_inv, int M, int K, void* act_amax, void* stream) {

@@ -79,6 +79,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: for a barrier whose arrivals publish writes made
+// by threads of another CTA of the cluster.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Bounded wait at cluster scope (as mbar_wait_bounded; the first probe and the final successful
+// probe acquire at cluster scope).
+__device__ __noinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                       uint32_t site) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (abort && *abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_device_status, 1u | ((site & 0xFFu) << 8));
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Slow path of mbar_wait_bounded (kept out of line).
 __device__ __noinline__ bool mbar_wait_bounded_slow(uint32_t bar, uint32_t parity,
                                                     volatile int* abort, uint32_t site) {
@@ -378,6 +406,12 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t local_saddr, uint32_t ra
 // reads, and much cheaper than a cluster-scope release.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// Arrival with release at cluster scope: publishes this thread's earlier shared-memory writes
+// to a waiter (acquiring at cluster scope) in another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 // TMA tile load into this CTA's shared memory whose completion is signalled on an

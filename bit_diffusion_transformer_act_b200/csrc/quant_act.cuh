@@ -53,6 +53,7 @@
 #pragma once
 
 #include "act_amax.cuh"
+#include "nvfp4_quant.cuh"
 #include "ptx.cuh"
 
 namespace svdq {
@@ -92,51 +93,6 @@ constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
 static_assert(kRows * kRank * 4 <= kStages * kStageBytes, "partial U reuses the stages");
 static_assert(kStageBytes % 1024 == 0 && kXBytes % 1024 == 0, "1 KB alignment of swizzled tiles");
-
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
-// RN(a / 6) for a >= 0 (Markstein correction of a * RN(1/6)).
-__device__ __forceinline__ float div6(float a) {
-  const float y = 0.16666667163372039794921875f;      // RN(1/6) in binary32
-  const float q0 = a * y;
-  const float e = fmaf(-q0, 6.0f, a);
-  return fmaf(e, y, q0);
-}
-
-// Quantizes one group of 16 smoothed values given as 8 pairs of -x_hat (see the
-// rounding note above): returns the E4M3 scale code and writes 8 code bytes.
-__device__ __forceinline__ uint32_t quantize_group(const uint64_t (&nx)[8], float g, float inv_g, uint2& out) {
-  float a[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) f32x2_unpack(nx[i], a[2 * i], a[2 * i + 1]);
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; i += 2) amax = fmax3(amax, fabsf(a[i]), fabsf(a[i + 1]));
-  const uint32_t sc = cvt_e4m3x2(div6(amax) * inv_g, 0.f) & 0xFFu;
-  float S, unused;
-  e4m3x2_to_f32(sc, S, unused);
-  const float D = S * g;
-  if (D == 0.f) {
-    out = make_uint2(0u, 0u);
-    return 0u;
-  }
-  const float rn = -rcp_approx(D);
-  const uint64_t rn2 = f32x2_pack(rn, rn), D2 = f32x2_pack(D, D);
-  float q[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint64_t q0 = f32x2_mul(nx[i], rn2);            // x_hat r
-    const uint64_t e = f32x2_fma(q0, D2, nx[i]);          // q0 D - x_hat, exact
-    f32x2_unpack(f32x2_fma(e, rn2, q0), q[2 * i], q[2 * i + 1]);   // q0 - e r
-  }
-  out.x = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-  out.y = cvt_e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  return sc;
-}
 
 // kind::f16 instruction descriptor: D f32, A and B bf16, K-major, N = 64, M = 128.
 __device__ __forceinline__ uint32_t idesc_lowrank() {

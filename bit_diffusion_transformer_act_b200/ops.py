@@ -39,6 +39,10 @@ def _load():
         "svdq_act_scale_bytes": ([i, i], sz),
         "svdq_quantize_act_lowrank_down": ([vp, vp, vp, i, i, i, f, vp, vp, vp, vp], i),
         "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
+        "svdq_w4a4_nvfp4_linear_qkv": ([vp, vp, vp, f, vp, f, i, i, i, i, i, i, vp, vp, f, vp, vp, vp, vp], i),
+        "svdq_gelu_quant_workspace_bytes": ([i, i], sz),
+        "svdq_w4a4_nvfp4_linear_gelu_quant": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp, f, vp, vp, vp, vp, sz, vp, vp],
+                                              i),
         "awq_w4a16_linear": ([vp, vp, vp, vp, vp, i, i, i, vp, vp], i),
         "svdq_act_amax": ([vp, vp, i, i, vp, vp], i),
         "svdq_act_amax_noalloc": ([vp, vp, i, i, vp, vp], i),
@@ -60,7 +64,8 @@ EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes"
             "svdq_act_scale_bytes", "svdq_quantize_act_lowrank_down", "svdq_w4a4_nvfp4_linear",
             "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status",
             "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn",
-            "svdq_act_amax_noalloc")
+            "svdq_act_amax_noalloc", "svdq_w4a4_nvfp4_linear_qkv", "svdq_gelu_quant_workspace_bytes",
+            "svdq_w4a4_nvfp4_linear_gelu_quant")
 
 
 def _check(fn, st):
@@ -218,6 +223,75 @@ def svdq_w4a4_nvfp4_linear(act_codes, act_scales, lowrank_act, act_global_scale,
                                     M, N, K, rank, _ptr(Y), _stream())
     _check("svdq_w4a4_nvfp4_linear", st)
     return Y
+
+
+def svdq_w4a4_nvfp4_linear_qkv(act_codes, act_scales, lowrank_act, act_global_scale, packed_w, w_global_scale,
+                               M, N, K, heads, norm_wq, norm_wk, eps, rope_cos, rope_sin, rank=RANK, Y=None):
+    """The fused Q/K/V projection: Y bf16 [M, N = 3 heads 128] holding q, k (RMS-normalised per
+    head with norm_wq / norm_wk bf16 [128], then rotated by rope_cos / rope_sin float32 [64, M],
+    pair-major) and v."""
+    D = 128
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    _require_blob(packed_w, "packed_w", svdq_packed_weight_bytes(N, K, rank))
+    _require(norm_wq, torch.bfloat16, (D,), "norm_wq")
+    _require(norm_wk, torch.bfloat16, (D,), "norm_wk")
+    _require(rope_cos, torch.float32, (D // 2, M), "rope_cos")
+    _require(rope_sin, torch.float32, (D // 2, M), "rope_sin")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    st = LIB.svdq_w4a4_nvfp4_linear_qkv(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act),
+                                        float(act_global_scale), _ptr(packed_w), float(w_global_scale),
+                                        M, N, K, rank, heads, D, _ptr(norm_wq), _ptr(norm_wk), float(eps),
+                                        _ptr(rope_cos), _ptr(rope_sin), _ptr(Y), _stream())
+    _check("svdq_w4a4_nvfp4_linear_qkv", st)
+    return Y
+
+
+def svdq_gelu_quant_workspace_bytes(M, N):
+    return int(LIB.svdq_gelu_quant_workspace_bytes(M, N))
+
+
+def svdq_w4a4_nvfp4_linear_gelu_quant(act_codes, act_scales, lowrank_act, act_global_scale, packed_w, w_global_scale,
+                                      M, N, K, down_smooth_inv, down_packed_w, down_act_global_scale, rank=RANK,
+                                      out_codes=None, out_scales=None, out_lowrank_act=None, workspace=None,
+                                      h_out=None):
+    """The MLP up projection with GELU and the down projection's activation pass fused: returns the
+    down projection's (act_codes uint8 [M, N/2], act_scales, lowrank_act bf16 [M, 2r]) for its
+    smooth_inv (bf16 [N]), packed weights (its low-rank section is used) and g_a.  h_out (bf16
+    [M, N]), if given, also receives the hidden state."""
+    _require(act_codes, torch.uint8, (M, K // 2), "act_codes")
+    _require(act_scales, torch.uint8, (svdq_act_scale_bytes(M, K),), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    _require_blob(packed_w, "packed_w", svdq_packed_weight_bytes(N, K, rank))
+    _require(down_smooth_inv, torch.bfloat16, (N,), "down_smooth_inv")
+    _require_blob(down_packed_w, "down_packed_w", _l1_section_end(N, rank))
+    dev = act_codes.device
+    if out_codes is None:
+        out_codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    if out_scales is None:
+        out_scales = torch.empty((svdq_act_scale_bytes(M, N),), dtype=torch.uint8, device=dev)
+    if out_lowrank_act is None:
+        out_lowrank_act = torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev)
+    ws_bytes = svdq_gelu_quant_workspace_bytes(M, N)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+    _require(out_codes, torch.uint8, (M, N // 2), "out_codes")
+    _require(out_scales, torch.uint8, (svdq_act_scale_bytes(M, N),), "out_scales")
+    _require(out_lowrank_act, torch.bfloat16, (M, 2 * rank), "out_lowrank_act")
+    _require_blob(workspace, "workspace", ws_bytes)
+    if h_out is not None:
+        _require(h_out, torch.bfloat16, (M, N), "h_out")
+    st = LIB.svdq_w4a4_nvfp4_linear_gelu_quant(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act),
+                                               float(act_global_scale), _ptr(packed_w), float(w_global_scale),
+                                               M, N, K, rank, _ptr(down_smooth_inv), _ptr(down_packed_w),
+                                               float(down_act_global_scale), _ptr(out_codes), _ptr(out_scales),
+                                               _ptr(out_lowrank_act), _ptr(workspace), workspace.numel(),
+                                               _ptr(h_out), _stream())
+    _check("svdq_w4a4_nvfp4_linear_gelu_quant", st)
+    return out_codes, out_scales, out_lowrank_act
 
 
 def svdq_act_amax(X, smooth_inv, act_amax=None):

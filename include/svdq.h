@@ -151,6 +151,64 @@ int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
                            const void* packed_w, float w_global_scale,
                            int M, int N, int K, int rank, void* Y, void* stream);
 
+/* Kernel 2 for a fused Q/K/V projection, with the per-head RMSNorm of q and k and their
+ * rotary position embedding (RoPE) done in the GEMM's epilogue -- "Nunchaku Lite" docs,
+ * section on fused kernels: the original engine fuses the Q, K, V projections with RMSNorm and
+ * RoPE (its benchmark table gives the RMSNorm + RoPE epilogue 1.236x and the whole fusion
+ * 1.27x).  The pages name the operations only; the readings used:
+ *   - Y [M, N] holds q, k, v side by side, N = 3 * heads * head_dim, each third head-major
+ *     (head h at columns h * head_dim .. + head_dim - 1 of its third);
+ *   - y = g_a g_w (Q(X_hat) Q(R)^T) + lowrank_act L2 + b as in svdq_w4a4_nvfp4_linear, kept in
+ *     fp32 (not rounded to bf16 before the normalisation);
+ *   - q and k heads: x / sqrt(mean(x^2) + eps) * w, with w = norm_wq (q) or norm_wk (k), bf16
+ *     [head_dim] shared by the heads; then pair i = (x[2i], x[2i+1]) of every head of token m
+ *     rotated: (x0 c - x1 s, x0 s + x1 c) with c = rope_cos[m, i], s = rope_sin[m, i];
+ *   - v is stored as the plain layer stores it; everything is rounded to bf16 once, at the end.
+ * The cos / sin tables are inputs, fp32 and pair-major: [head_dim / 2, M], the value for pair
+ * i of token m at [i * M + m] (so that 32 consecutive tokens' values of one pair are one
+ * 128-byte line); a model's position scheme (one axis, or several as in image transformers)
+ * only changes the tables.
+ * head_dim == 128; N == 3 * heads * 128; other arguments and errors as svdq_w4a4_nvfp4_linear;
+ * norm_wq, norm_wk, rope_cos, rope_sin device pointers, 16-byte aligned; eps >= 0 finite.
+ * Asynchronous on `stream`. */
+int svdq_w4a4_nvfp4_linear_qkv(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                               float act_global_scale, const void* packed_w, float w_global_scale, int M, int N,
+                               int K, int rank, int heads, int head_dim, const void* norm_wq, const void* norm_wk,
+                               float eps, const void* rope_cos, const void* rope_sin, void* Y, void* stream);
+
+/* Kernels 6 and 7: the MLP up projection with GELU and the down projection's activation pass in
+ * its epilogue -- "Nunchaku Lite" docs, section on fused kernels: the original engine runs the
+ * MLP with a fused GELU kernel (its benchmark table gives the GELU-MLP fusion 1.06x).  The
+ * pages name the fusion only; the reading used is that it computes what the unfused pipeline
+ * computes, without the hidden state ever reaching memory:
+ *   y = bf16(g_a g_w (Q(X_hat) Q(R)^T) + lowrank_act L2 + b)        (svdq_w4a4_nvfp4_linear)
+ *   h = bf16(GELU(y)),  GELU(x) = x Phi(x) (erf form, evaluated in fp32)
+ *   out_codes, out_scales, out_lowrank_act = svdq_quantize_act_lowrank_down(h, down_smooth_inv,
+ *       down_packed_w, down_act_global_scale)   (the down projection's activation pass on h)
+ * The low-rank product U = h_hat L1 of the down projection needs every column of a row; the GEMM
+ * keeps it in tensor memory over each CTA pair's consecutive output tiles of a row block and
+ * writes one fp32 partial per (pair, row block) to `workspace`; kernel 7 sums them in a fixed
+ * order (repeat calls are bit-identical).  Against the unfused pipeline the result can differ
+ * only where fp32 GELU lands on the other side of a bf16 rounding midpoint than the exact value
+ * (h one bf16 ulp apart); codes and scales are exact for the h this call forms.
+ *   act_codes, act_scales, lowrank_act, packed_w, g's: as svdq_w4a4_nvfp4_linear (N = the MLP
+ *     width, the down projection's K)
+ *   down_smooth_inv   device bf16 [N]; down_packed_w the down projection's packed blob (only its
+ *     header and low-rank section, the first 1024 + 4 rank N bytes, are read)
+ *   down_act_global_scale  the down projection's static g_a (a power of two)
+ *   out_codes   u8 [M, N/2]; out_scales u8 [svdq_act_scale_bytes(M, N)]; out_lowrank_act bf16 [M, 2 rank]
+ *   workspace   device scratch of at least svdq_gelu_quant_workspace_bytes(M, N) bytes
+ *     (the caller allocates it; contents need no initialisation and are overwritten)
+ *   h_out       device bf16 [M, N] or NULL: if given, also receives h (for inspection)
+ * N % 128 == 0, K % 64 == 0, rank == 32; 16-byte aligned pointers.  Asynchronous on `stream`. */
+size_t svdq_gelu_quant_workspace_bytes(int M, int N);   /* for the current device; 0 if invalid */
+int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_scales, const void* lowrank_act,
+                                      float act_global_scale, const void* packed_w, float w_global_scale, int M,
+                                      int N, int K, int rank, const void* down_smooth_inv, const void* down_packed_w,
+                                      float down_act_global_scale, void* out_codes, void* out_scales,
+                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes, void* h_out,
+                                      void* stream);
+
 /* -------------------------------------------- dynamic per-tensor activation scale */
 
 /* Kernel 5: the variant of the W4A4 layer whose activation scale g_a comes from the batch

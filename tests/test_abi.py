@@ -87,6 +87,40 @@ def test_gpu_entry_points_reject_bad_arguments_before_any_device_work():
     assert L.awq_w4a16_linear(None, None, None, None, None, 0, 64, 256, None, None) == 0
 
 
+def test_qkv_entry_point_rejects_bad_arguments_before_any_device_work():
+    L = P.LIB
+    odd = ctypes.c_void_p((1 << 20) + 8)
+
+    def qkv(M=4, N=768, K=64, heads=2, D=128, eps=1e-6, wq=FAKE, cos=FAKE):
+        return L.svdq_w4a4_nvfp4_linear_qkv(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, M, N, K, 32, heads, D, wq, FAKE,
+                                            eps, cos, FAKE, FAKE, None)
+    assert qkv(D=64, N=384) == 2                       # head_dim 128 only
+    assert qkv(N=640) == 2                             # N = 3 heads head_dim
+    assert qkv(heads=0) == 1
+    assert qkv(eps=-1.0) == 1
+    assert qkv(eps=float("inf")) == 1
+    assert qkv(wq=None) == 1
+    assert qkv(cos=odd) == 1
+    assert qkv(K=96) == 2                              # the plain call's checks follow
+    assert qkv(M=0, wq=None, cos=None) == 0            # an empty batch needs neither tables nor a device
+
+
+def test_gelu_quant_entry_point_rejects_bad_arguments_before_any_device_work():
+    L = P.LIB
+
+    def call(M=4, N=256, K=64, g=1.0, gd=1.0, ws=FAKE, wsb=1 << 30, h=None, codes=FAKE):
+        return L.svdq_w4a4_nvfp4_linear_gelu_quant(FAKE, FAKE, FAKE, g, FAKE, 1.0, M, N, K, 32, FAKE, FAKE, gd,
+                                                   codes, FAKE, FAKE, ws, wsb, h, None)
+    assert call(N=192) == 2                             # N % 128
+    assert call(K=96) == 2
+    assert call(g=0.3) == 1 and call(gd=3.0) == 1       # scales must be powers of two
+    assert call(ws=None) == 1 and call(codes=None) == 1
+    assert call(h=ctypes.c_void_p((1 << 20) + 8)) == 1  # misaligned optional output
+    assert call(M=-1) == 1
+    assert call(M=0, ws=None, codes=None) == 0          # empty batch: nothing needed
+    assert P.svdq_gelu_quant_workspace_bytes(4, 200) == 0
+
+
 def test_dynamic_scale_entry_points_reject_bad_arguments_before_any_device_work():
     L = P.LIB
     odd2 = ctypes.c_void_p((1 << 20) + 2)

@@ -186,6 +186,111 @@ def test_full_size_layer(P, name, M, K, N, gelu):
     assert P.svdq_device_status() == 0
 
 
+# ---------------------------------------------------------------- fused QKV epilogue (RMSNorm + RoPE)
+
+def rope_tables(M, D):
+    """fp32 cos / sin tables [M, D/2]: token m at position m, pair i at the inverse frequency
+    10000^(-i / (D/2)) (the usual one-axis scheme; the kernel takes any tables)."""
+    ang = np.arange(M, dtype=np.float64)[:, None] * 10000.0 ** (-np.arange(D // 2) / (D // 2))[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+QKV = [
+    ("3 heads, 128-wide tiles, M tail 300x512->1152", 300, 512, 3),
+    ("2 heads, 256-wide tiles 8192x256->768", 8192, 256, 2),
+    ("qkv 64x3072->9216 (24 heads)", 64, 3072, 24),
+    ("qkv 4608x3072->9216 (24 heads)", 4608, 3072, 24),
+]
+
+
+@pytest.mark.parametrize("name,M,K,heads", QKV, ids=[q[0] for q in QKV])
+def test_qkv_rmsnorm_rope_epilogue(P, name, M, K, heads):
+    from oracle import qkv_epilogue as E
+    D, eps = 128, 1e-6
+    N = 3 * heads * D
+    w = synth.svdq_workload(M, K, N)
+    packed, gw = _pack(P, w)
+    codes, scales, U = P.svdq_quantize_act_lowrank_down(_bf16_dev(w.X), _bf16_dev(w.smooth_inv), packed, w.g_a)
+    rng = np.random.default_rng(heads + M)
+    wq = synth.to_bf16(1.0 + 0.2 * rng.standard_normal(D))
+    wk = synth.to_bf16(1.0 + 0.2 * rng.standard_normal(D))
+    cos, sin = rope_tables(M, D)
+    Y = P.svdq_w4a4_nvfp4_linear_qkv(codes, scales, U, w.g_a, packed, gw, M, N, K, heads, _bf16_dev(wq),
+                                     _bf16_dev(wk), eps, torch.from_numpy(np.ascontiguousarray(cos.T)).cuda(),
+                                     torch.from_numpy(np.ascontiguousarray(sin.T)).cuda())
+    torch.cuda.synchronize()
+    Yg = Y.float().cpu().numpy()
+    rows = sample_rows(M, 21)
+    y_ref = svdq.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias, w.g_a)
+    q, k, v = E.qkv_epilogue(y_ref, heads, wq, wk, eps, cos[rows].astype(np.float64), sin[rows].astype(np.float64))
+    HD = heads * D
+    r = len(rows)
+    check_output(Yg[rows, :HD], q.reshape(r, HD))
+    check_output(Yg[rows, HD:2 * HD], k.reshape(r, HD))
+    check_output(Yg[rows, 2 * HD:], v.reshape(r, HD))
+    if heads % 2 == 0:
+        # same tile width as the plain call: v is the plain layer's output bit for bit
+        Yp = P.svdq_w4a4_nvfp4_linear(codes, scales, U, w.g_a, packed, gw, M, N, K)
+        torch.cuda.synchronize()
+        assert np.array_equal(Yp.float().cpu().numpy()[:, 2 * HD:], Yg[:, 2 * HD:])
+    assert P.svdq_device_status() == 0
+
+
+# ---------------------------------------------------------------- fused MLP up projection (GELU + re-quantization)
+
+MLP = [
+    ("tiny 300x256->512, down ->256", 300, 256, 512, 256),
+    ("M tail and row blocks over pairs 1000x512->1536, down ->384", 1000, 512, 1536, 384),
+    ("mlp 4608x3072->12288, down ->3072", 4608, 3072, 12288, 3072),
+]
+
+
+@pytest.mark.parametrize("name,M,K,F,Nd", MLP, ids=[c[0] for c in MLP])
+def test_mlp_up_gelu_requantize_epilogue(P, name, M, K, F, Nd):
+    from oracle import mlp_epilogue as E
+    up = synth.svdq_workload(M, K, F)
+    dn = synth.svdq_workload(min(M, 512), F, Nd, gelu_input=True)   # the down layer; its X only calibrates
+    pu, gwu = _pack(P, up)
+    pd, gwd = _pack(P, dn)
+    g_dn = dn.g_a
+    codes, scales, U = P.svdq_quantize_act_lowrank_down(_bf16_dev(up.X), _bf16_dev(up.smooth_inv), pu, up.g_a)
+    sd = _bf16_dev(dn.smooth_inv)
+    h = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    c1, s1, u1 = P.svdq_w4a4_nvfp4_linear_gelu_quant(codes, scales, U, up.g_a, pu, gwu, M, F, K, sd, pd, g_dn,
+                                                     h_out=h)
+    c2, s2, u2 = P.svdq_w4a4_nvfp4_linear_gelu_quant(codes, scales, U, up.g_a, pu, gwu, M, F, K, sd, pd, g_dn)
+    torch.cuda.synchronize()
+    hg = h.float().cpu().numpy().astype(np.float64)
+    c1, s1, u1 = c1.cpu().numpy(), s1.cpu().numpy(), u1.float().cpu().numpy().astype(np.float64)
+    # without the hidden-state output, and again: the same bits
+    assert np.array_equal(c1, c2.cpu().numpy()) and np.array_equal(s1, s2.cpu().numpy())
+    assert np.array_equal(u1, u2.float().cpu().numpy())
+    # the hidden state against the oracle's (from the oracle's up projection), sampled rows
+    rows = sample_rows(M, 31)
+    y_ref = svdq.forward(up.X[rows], up.smooth_inv, up.R, up.L1, up.L2, up.bias, up.g_a)
+    check_output(hg[rows], E.hidden_state(y_ref))
+    # the down projection's activation pass on this h: codes and scales bit for bit, every row
+    cx, sx = svdq.quantize_activations(hg, dn.smooth_inv, g_dn)
+    assert np.array_equal(c1, nvfp4.pack_nibbles(cx)), np.argwhere(c1 != nvfp4.pack_nibbles(cx))[:5]
+    sg = unswizzle(s1, (M + 127) // 128 * 128, F)
+    assert np.array_equal(sg[:M], sx), np.argwhere(sg[:M] != sx)[:5]
+    assert np.all(sg[M:] == 0)
+    # U = h_hat L1 within fp32 accumulation (over the pairs' partials) and the hi + lo split
+    Hh = svdq.smooth(hg, dn.smooth_inv)
+    L1 = dn.L1.astype(np.float64)
+    U_ref = Hh @ L1
+    Ug = g_dn * (u1[:, :32] + u1[:, 32:])
+    bound = 2e-5 * (np.abs(Hh) @ np.abs(L1)) + 2.0 ** -15 * np.abs(U_ref) + 1e-30
+    assert np.all(np.abs(Ug - U_ref) <= bound), np.max(np.abs(Ug - U_ref) / bound)
+    # and the down projection run on them against the oracle's down projection of this h
+    Yd = P.svdq_w4a4_nvfp4_linear(torch.from_numpy(c1).cuda(), torch.from_numpy(s1).cuda(),
+                                  torch.from_numpy(u1.astype(np.float32)).to(torch.bfloat16).cuda(), g_dn, pd, gwd,
+                                  M, Nd, F)
+    torch.cuda.synchronize()
+    check_output(Yd.float().cpu().numpy()[rows], svdq.forward(hg[rows], dn.smooth_inv, dn.R, dn.L1, dn.L2, dn.bias, g_dn))
+    assert P.svdq_device_status() == 0
+
+
 # ---------------------------------------------------------------- AWQ W4A16
 
 def _run_awq(P, a, bias=None):
