@@ -1,24 +1,35 @@
 #!/usr/bin/env python
 """Benchmark of the SVDQuant W4A4 (NVFP4) linear layer and the AWQ W4A16 linear layer.
 
-One step is one pass of the whole hot path over one batch of synthetic input:
-  * the SVDQ W4A4 NVFP4 attention projection, M=4096, K=N=3072, rank 32, group 16
-    (kernel 1: smoothing + NVFP4 quantization + low-rank down; kernel 2: the
-    block-scaled tcgen05 GEMM with the low-rank-up/bias epilogue);
-  * the AWQ W4A16 adaLN linear, K=3072, N=18432, group 64, at M = 1, 2, 4, 8, 16, 32, 64.
-`value` is the SVDQ layer throughput in TFLOP/s (2MNK per step over the device
-time of kernels 1+2); the AWQ throughput in GB/s is reported under "awq".
+One step is one pass of the whole hot path over one batch of synthetic input, on every
+seeded configuration:
+  * the SVDQ W4A4 NVFP4 DiT attention projection, M=4096, K=N=3072, rank 32, group 16, as the
+    layer runs it (kernel 1: smoothing + NVFP4 quantization + low-rank down, chained with
+    programmatic dependent launch into kernel 2: the block-scaled tcgen05 GEMM with the
+    low-rank-up/bias epilogue), then each of its two kernels on its own;
+  * the AWQ W4A16 adaLN linear, K=3072, N=18432, group 64, at M = 1, 2, 4, 8, 16, 32, 64;
+  * the SVDQ fused-QKV sweep, K=3072, N=9216, M = 64, 256, 1024, 4608, 18432 (layer);
+  * the SVDQ DiT MLP pair: up 4608x3072->12288, down 4608x12288->3072 on GELU-shaped inputs.
+`value` is the attention layer's throughput in TFLOP/s (2MNK per step over the device time
+of its chained kernels); every other figure is reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU: the layers do not need to shard (every GPU runs its own replica),
-so N ranks run N independent replicas; `value` sums all ranks' work over the
-slowest rank's time ("scaling": "weak").  Inputs and weights are rotated over
-8 resident copies so that every step reads from HBM, not from L2.
+Timing: each segment (a layer or kernel of one configuration) is one CUDA graph holding
+exactly K launches (or K layers) over rotating resident copies of its inputs, weights and
+outputs (more than twice the L2 size per cycle, so every launch reads from HBM); CUDA events
+on the launching stream bracket every graph, and the timed region is all segments back to
+back.  The SM clock is sampled through NVML throughout the timed region.
+
+Multi-GPU: the layers do not need to shard (every GPU runs its own replica), so N ranks run N
+independent replicas; `value` sums all ranks' work over the slowest rank's time ("scaling":
+"weak").
 """
 
 import argparse
+import hashlib
 import json
+import math
 import os
 import sys
 import threading
@@ -30,26 +41,36 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 SVDQ W4A4 linear TFLOPS (% FP4 peak); AWQ W4A16 GB/s (% HBM)"
-SVDQ_SHAPE = (4096, 3072, 3072)              # M, K, N: DiT attention projection, 64x64 latent tokens
+ATTN = (4096, 3072, 3072)                    # M, K, N: DiT attention projection, 64x64 latent tokens
+QKV_K, QKV_N, QKV_MS = 3072, 9216, (64, 256, 1024, 4608, 18432)
+QKV_HEADS, QKV_FUSED_MS, QKV_EPS = 24, (64, 4608), 1e-6   # 24 heads of 128; the fused-epilogue rows
+MLP_UP = (4608, 3072, 12288)
+MLP_DOWN = (4608, 12288, 3072)
 AWQ_K, AWQ_N, AWQ_MS = 3072, 18432, (1, 2, 4, 8, 16, 32, 64)
 RANK = 32
-NSETS = 8                                    # rotating copies (> 2x L2 per cycle)
-NREP = 3                                     # passes over the copies per CUDA-graph batch (24 launches)
 FP4_OVER_BF16 = 4.0                          # nominal dense ratio (9 / 2.25 PFLOP/s)
+# Nominal dense FP4 rate of one SM per clock: one kind::mxf4nvf4 MMA of M=128 (per SM),
+# N=256, K=64 every 128 cycles.  Times the SM count and the sampled clock it gives the
+# clock-matched peak beside the measured-derived one.
+FP4_FLOP_PER_SM_CLK = 2 * 128 * 256 * 64 / 128
+GEMM_SOURCES = ("gemm_nvfp4.cuh", "ptx.cuh", "act_amax.cuh", "libsvdq.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "nvfp4_gemm_kernel_attention_4096x3072x3072_dram.txt")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=384)       # 16 graph batches of 24
-    ap.add_argument("--warmup", type=int, default=24)
+    ap.add_argument("--steps", type=int, default=48)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly (for profilers)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="one resident copy, eager launches of every kernel (for ncu captures); prints timings")
-    return ap.parse_args()
+    ap.add_argument("--case", default="attention", choices=["attention", "qkv64", "qkv4608_fused"],
+                    help="workload of --profile-case")
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -62,6 +83,30 @@ def load_peaks():
                 "source": "measured"}
     except (OSError, KeyError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_sources_sha():
+    """sha256 over the GEMM kernel's sources: a DRAM capture is valid only for the build it
+    was taken on."""
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "bit_diffusion_transformer_act_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic():
+    """DRAM bytes (read + write) per launch of the attention GEMM from the ncu capture summary,
+    or None when there is none or it was taken on other kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            kv = dict(line.split(":", 1) for line in f if ":" in line and not line.startswith("#"))
+    except OSError:
+        return None, "no capture"
+    kv = {k.strip(): v.strip() for k, v in kv.items()}
+    if kv.get("sources_sha256") != gemm_sources_sha():
+        return None, "capture taken on other kernel sources (stale)"
+    return int(kv["dram_bytes_read"]) + int(kv["dram_bytes_write"]), "ncu capture of this build, cold caches"
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -89,44 +134,6 @@ def barrier(world):
         dist.barrier()
 
 
-def time_dynamic_variant(P, wl, stream, use_graph, reps=5):
-    """The dynamic-activation-scale layer (a variant, timed after the main region): kernel 5
-    alone and the whole layer (kernels 5, 1, 2), each as CUDA-graph batches over the copies."""
-    import torch
-    out = {}
-    for name, fn in (("amax", wl.amax), ("layer", wl.dyn_layer)):
-        def batch():
-            for _ in range(NREP):
-                for i in range(NSETS):
-                    fn(P, i)
-        with torch.cuda.stream(stream):
-            batch()                                  # warm-up (eager)
-        torch.cuda.synchronize()
-        if use_graph:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                batch()
-            run = g.replay
-        else:
-            run = batch
-        best = None
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            with torch.cuda.stream(stream):
-                run()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            t = e0.elapsed_time(e1) / (NSETS * NREP)
-            best = t if best is None else min(best, t)
-        out[name + "_us"] = best * 1e3
-    M, K, N = SVDQ_SHAPE
-    out["amax_gbs"] = 2.0 * M * K / (out["amax_us"] * 1e-6) / 1e9
-    out["layer_tflops"] = svdq_flops() / (out["layer_us"] * 1e-6) / 1e12
-    out["note"] = "g_a from the batch's amax (kernel 5) instead of calibration; best of 5 graph batches of 24"
-    return out
-
-
 def job_rate(world, steps, units_per_step, slowest_ms):
     """Whole-job throughput in units per second: the units all ranks processed (each rank ran
     `steps` steps of `units_per_step`) over the slowest rank's device time."""
@@ -152,7 +159,8 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
 
 
 class ClockSampler:
-    """Samples the SM clock and the clock-event reasons of one GPU through NVML."""
+    """Samples the SM clock and the clock-event reasons of one GPU through NVML, as often as
+    NVML answers (a fraction of a millisecond), while the timed region runs."""
 
     def __init__(self, device_index):
         self.samples, self.reasons, self.max_mhz = [], 0, None
@@ -173,18 +181,22 @@ class ClockSampler:
         except Exception:
             self._h = None
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
-            except Exception:
-                pass
-            time.sleep(0.001)
+            self._sample()
+            time.sleep(0.0001)
 
     def __enter__(self):
         if self._h is not None:
+            self._sample()
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
@@ -193,47 +205,66 @@ class ClockSampler:
         if self._h is not None:
             self._stop.set()
             self._t.join()
-            self._run_once()
-
-    def _run_once(self):
-        try:
-            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
-        except Exception:
-            pass
+            self._sample()
 
     def summary(self):
         if self._h is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
         names = [n for bit, n in REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": float(np.median(self.samples)) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": float(np.min(self.samples)) if self.samples else None,
                 "reasons": names, "samples": len(self.samples)}
 
 
-# ---------------------------------------------------------------- our implementation
+# ---------------------------------------------------------------- work per configuration
 
 def bf16_dev(a, dev):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).to(dev)
 
 
-class Workload:
-    """Resident inputs, weights and outputs of one step, in NSETS rotating copies."""
+def n_sets(footprint_bytes, l2_bytes):
+    """Rotating copies so that one pass over them touches more than twice the L2 size."""
+    return int(min(16, max(2, math.ceil(2 * l2_bytes / footprint_bytes))))
 
-    def __init__(self, P, dev):
+
+def svdq_flops(M, K, N):
+    return 2.0 * M * N * K
+
+
+def k1_bytes(M, K):
+    """Kernel 1: X, smooth_inv, the packed low-rank down factor (hi + lo), codes, scales, U (hi + lo)."""
+    return 2 * M * K + 2 * K + 4 * K * RANK + M * K / 2 + M * K / 16 + 4 * M * RANK
+
+
+def k2_bytes(M, K, N):
+    """Kernel 2: codes and scales of both operands, L2, bias, U (hi + lo) and the bf16 output."""
+    return (N + M) * K * (0.5 + 1 / 16) + 2 * RANK * N + 2 * N + 4 * M * RANK + 2 * M * N
+
+
+def awq_bytes(m):
+    return AWQ_N * AWQ_K / 2 + 4 * AWQ_N * AWQ_K / 64 + 2 * m * AWQ_K + 2 * m * AWQ_N
+
+
+class SvdqCase:
+    """One SVDQ layer (M, K, N) with its weights packed once and `nsets` rotating resident
+    copies of input, weights, intermediates and output."""
+
+    def __init__(self, P, dev, w, M, l2_bytes, nsets=None):
         import torch
         import synth
-        M, K, N = SVDQ_SHAPE
-        w = synth.svdq_workload(M, K, N)
+        K, N = w.K, w.N
         blob, self.g_w = P.svdq_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2),
                                              synth.bf16_bits(w.bias), synth.bf16_bits(w.smooth_inv))
         self.g_a = w.g_a
         self.M, self.K, self.N = M, K, N
-        X = bf16_dev(w.X, dev)
         self.smooth = bf16_dev(w.smooth_inv, dev)
+        X = bf16_dev(w.X[:M], dev)
         blob_d = torch.from_numpy(blob).to(dev)
-        self.host_X = w.X                                   # for the end-to-end leg
+        per_set = blob.nbytes + k1_bytes(M, K) + 2 * M * N
+        self.nsets = nsets or n_sets(per_set, l2_bytes)
         self.sets = []
-        for _ in range(NSETS):
+        for _ in range(self.nsets):
             self.sets.append({
                 "X": X.clone(), "W": blob_d.clone(),
                 "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
@@ -242,187 +273,341 @@ class Workload:
                 "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
                 "amax": torch.zeros((4,), dtype=torch.int32, device=dev),
             })
-        a = synth.awq_workload(max(AWQ_MS), AWQ_K, AWQ_N)
-        ax = bf16_dev(a.X, dev)
-        qw = torch.from_numpy(a.qweight).to(dev)
-        sc, zr = bf16_dev(a.scales, dev), bf16_dev(a.zeros, dev)
-        self.awq_sets = []
-        for _ in range(NSETS):
-            s = {"qw": qw.clone(), "s": sc.clone(), "z": zr.clone(), "X": {}, "Y": {}}
-            for m in AWQ_MS:
-                s["X"][m] = ax[:m].clone()
-                s["Y"][m] = torch.empty((m, AWQ_N), dtype=torch.bfloat16, device=dev)
-            self.awq_sets.append(s)
 
     def k1(self, P, i):
-        s = self.sets[i]
+        s = self.sets[i % self.nsets]
         P.svdq_quantize_act_lowrank_down(s["X"], self.smooth, s["W"], self.g_a, RANK, s["codes"], s["scales"], s["U"])
 
     def k2(self, P, i):
-        s = self.sets[i]
+        s = self.sets[i % self.nsets]
         P.svdq_w4a4_nvfp4_linear(s["codes"], s["scales"], s["U"], self.g_a, s["W"], self.g_w,
                                  self.M, self.N, self.K, RANK, s["Y"])
 
+    def layer(self, P, i):
+        self.k1(P, i)
+        self.k2(P, i)
+
+    def set_qkv(self, dev, heads, eps):
+        """Norm weights and RoPE tables of a fused Q/K/V projection over this case's N."""
+        import torch
+        rng = np.random.default_rng(7)
+        D = 128
+        self.heads, self.eps = heads, eps
+        self.wq = bf16_dev(1.0 + 0.2 * rng.standard_normal(D), dev)
+        self.wk = bf16_dev(1.0 + 0.2 * rng.standard_normal(D), dev)
+        ang = np.arange(self.M)[:, None] * 10000.0 ** (-np.arange(D // 2) / (D // 2))[None, :]
+        self.cos = torch.from_numpy(np.ascontiguousarray(np.cos(ang).T, dtype=np.float32)).to(dev)   # [64, M]
+        self.sin = torch.from_numpy(np.ascontiguousarray(np.sin(ang).T, dtype=np.float32)).to(dev)
+
+    def qkv_fused(self, P, i):
+        """Kernel 1, then the GEMM whose epilogue RMS-normalises and rotates q and k."""
+        s = self.sets[i % self.nsets]
+        self.k1(P, i)
+        P.svdq_w4a4_nvfp4_linear_qkv(s["codes"], s["scales"], s["U"], self.g_a, s["W"], self.g_w, self.M, self.N,
+                                     self.K, self.heads, self.wq, self.wk, self.eps, self.cos, self.sin, Y=s["Y"])
+
+    def qkv_torch_norm_rope(self, P, i):
+        """The unfused pipeline's second half, for comparison only: RMSNorm and RoPE of q and k
+        as separate PyTorch operations on the plain layer's bf16 output (not this library)."""
+        import torch
+        s = self.sets[i % self.nsets]
+        M, HD = self.M, self.heads * 128
+        x = s["Y"][:, :2 * HD].view(M, 2, self.heads, 128).float()
+        w = torch.stack([self.wq, self.wk]).float().view(1, 2, 1, 128)
+        x = x * torch.rsqrt(x.pow(2).mean(-1, keepdim=True) + self.eps) * w
+        x0, x1 = x[..., 0::2], x[..., 1::2]
+        c, sn = self.cos.t().reshape(M, 1, 1, 64), self.sin.t().reshape(M, 1, 1, 64)
+        out = torch.stack([x0 * c - x1 * sn, x0 * sn + x1 * c], dim=-1).flatten(-2)
+        s["Y"][:, :2 * HD].copy_(out.reshape(M, 2 * HD).to(torch.bfloat16))
+
     def amax(self, P, i):
-        s = self.sets[i]
+        s = self.sets[i % self.nsets]
         P.svdq_act_amax(s["X"], self.smooth, s["amax"])
 
     def dyn_layer(self, P, i):
         """The layer with the dynamic activation scale: kernel 5, then kernels 1 and 2 reading it."""
-        s = self.sets[i]
+        s = self.sets[i % self.nsets]
         P.svdq_act_amax(s["X"], self.smooth, s["amax"])
         P.svdq_quantize_act_lowrank_down_dyn(s["X"], self.smooth, s["W"], s["amax"], RANK, s["codes"], s["scales"],
                                              s["U"])
         P.svdq_w4a4_nvfp4_linear_dyn(s["codes"], s["scales"], s["U"], s["amax"], s["W"], self.g_w,
                                      self.M, self.N, self.K, RANK, s["Y"])
 
-    def awq(self, P, i, m):
-        s = self.awq_sets[i]
+
+class MlpFused:
+    """The MLP pair with the up projection's fused epilogue (GELU + the down projection's
+    activation pass): kernel 1 on X, kernels 6 and 7, then the down projection's GEMM on their
+    outputs; buffers per rotating set of the two layers."""
+
+    def __init__(self, P, dev, up, down):
+        import torch
+        self.up, self.down = up, down
+        M, F = up.M, up.N
+        self.ws_bytes = P.svdq_gelu_quant_workspace_bytes(M, F)
+        self.nsets = min(up.nsets, down.nsets)
+        self.sets = [{"codes": torch.empty((M, F // 2), dtype=torch.uint8, device=dev),
+                      "scales": torch.empty((P.svdq_act_scale_bytes(M, F),), dtype=torch.uint8, device=dev),
+                      "U": torch.empty((M, 2 * RANK), dtype=torch.bfloat16, device=dev),
+                      "ws": torch.empty((self.ws_bytes,), dtype=torch.uint8, device=dev)} for _ in range(self.nsets)]
+
+    def up_fused(self, P, i):
+        u, d, s = self.up.sets[i % self.nsets], self.down.sets[i % self.nsets], self.sets[i % self.nsets]
+        self.up.k1(P, i % self.nsets)
+        P.svdq_w4a4_nvfp4_linear_gelu_quant(u["codes"], u["scales"], u["U"], self.up.g_a, u["W"], self.up.g_w,
+                                            self.up.M, self.up.N, self.up.K, self.down.smooth, d["W"], self.down.g_a,
+                                            RANK, s["codes"], s["scales"], s["U"], s["ws"])
+
+    def down_gemm(self, P, i):
+        d, s = self.down.sets[i % self.nsets], self.sets[i % self.nsets]
+        P.svdq_w4a4_nvfp4_linear(s["codes"], s["scales"], s["U"], self.down.g_a, d["W"], self.down.g_w,
+                                 self.down.M, self.down.N, self.down.K, RANK, d["Y"])
+
+
+class AwqCase:
+    """The AWQ adaLN weight in rotating copies, with inputs and outputs for every M."""
+
+    def __init__(self, P, dev, l2_bytes, nsets=None):
+        import torch
+        import synth
+        a = synth.awq_workload(max(AWQ_MS), AWQ_K, AWQ_N)
+        ax = bf16_dev(a.X, dev)
+        qw = torch.from_numpy(a.qweight).to(dev)
+        sc, zr = bf16_dev(a.scales, dev), bf16_dev(a.zeros, dev)
+        self.nsets = nsets or n_sets(awq_bytes(1), l2_bytes)
+        self.sets = []
+        for _ in range(self.nsets):
+            s = {"qw": qw.clone(), "s": sc.clone(), "z": zr.clone(), "X": {}, "Y": {}}
+            for m in AWQ_MS:
+                s["X"][m] = ax[:m].clone()
+                s["Y"][m] = torch.empty((m, AWQ_N), dtype=torch.bfloat16, device=dev)
+            self.sets.append(s)
+
+    def run(self, P, i, m):
+        s = self.sets[i % self.nsets]
         P.awq_w4a16_linear(s["X"][m], s["qw"], s["s"], s["z"], None, s["Y"][m])
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one nvfp4_gemm_kernel<256>
-# launch at the attention shape, from an ncu capture with cold caches (13.15 MB read = the
-# algorithmic input bytes; the bf16 output stays in L2 within the launch).  Must be
-# re-measured whenever the GEMM kernel changes.
-GEMM_DRAM_BYTES_PER_LAUNCH = 13154560
+class Workloads:
+    def __init__(self, P, dev, l2_bytes, extra=True):
+        import synth
+        self.attn = SvdqCase(P, dev, synth.svdq_workload(*ATTN), ATTN[0], l2_bytes)
+        self.awq = AwqCase(P, dev, l2_bytes)
+        self.qkv, self.mlp_up, self.mlp_down = {}, None, None
+        if extra:
+            wq = synth.svdq_workload(max(QKV_MS), QKV_K, QKV_N)      # one layer; batches are row prefixes
+            self.qkv = {m: SvdqCase(P, dev, wq, m, l2_bytes) for m in QKV_MS}
+            del wq
+            for m in QKV_FUSED_MS:
+                self.qkv[m].set_qkv(dev, QKV_HEADS, QKV_EPS)
+            self.mlp_up = SvdqCase(P, dev, synth.svdq_workload(*MLP_UP), MLP_UP[0], l2_bytes)
+            self.mlp_down = SvdqCase(P, dev, synth.svdq_workload(*MLP_DOWN, gelu_input=True), MLP_DOWN[0], l2_bytes)
+            self.mlp_fused = MlpFused(P, dev, self.mlp_up, self.mlp_down)
+
+    def segments(self, P):
+        """(name, launches per step, fn(i)) of every segment of one step, in timing order."""
+        seg = [("attn_layer", 2, lambda i: self.attn.layer(P, i)),
+               ("attn_k1", 1, lambda i: self.attn.k1(P, i)),
+               ("attn_k2", 1, lambda i: self.attn.k2(P, i))]
+        seg += [("awq%d" % m, 1, (lambda i, m=m: self.awq.run(P, i, m))) for m in AWQ_MS]
+        seg += [("qkv%d" % m, 2, (lambda i, c=c: c.layer(P, i))) for m, c in self.qkv.items()]
+        seg += [("qkv%d_k1" % m, 1, (lambda i, c=c: c.k1(P, i))) for m, c in self.qkv.items()]
+        seg += [("qkv%d_k2" % m, 1, (lambda i, c=c: c.k2(P, i))) for m, c in self.qkv.items()]
+        for m in QKV_FUSED_MS:
+            if m in self.qkv:
+                c = self.qkv[m]
+                seg += [("qkv%d_fused" % m, 2, (lambda i, c=c: c.qkv_fused(P, i))),
+                        ("qkv%d_torch_norm_rope" % m, 0, (lambda i, c=c: c.qkv_torch_norm_rope(P, i)))]
+        if self.mlp_up is not None:
+            seg += [("mlp_up", 2, lambda i: self.mlp_up.layer(P, i)),
+                    ("mlp_down", 2, lambda i: self.mlp_down.layer(P, i)),
+                    ("mlp_up_fused", 3, lambda i: self.mlp_fused.up_fused(P, i)),
+                    ("mlp_down_gemm", 1, lambda i: self.mlp_fused.down_gemm(P, i))]
+        return seg
 
 
-def svdq_flops():
-    M, K, N = SVDQ_SHAPE
-    return 2.0 * M * N * K
+# ---------------------------------------------------------------- timing
+
+def capture(fn, steps, stream, use_graph):
+    """A callable that runs fn(0..steps-1) on `stream`: one CUDA graph holding all of them, or
+    eager launches."""
+    import torch
+    if not use_graph:
+        def run():
+            with torch.cuda.stream(stream):
+                for i in range(steps):
+                    fn(i)
+        return run
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            fn(i)
+    return g.replay
 
 
-def k1_bytes():
-    M, K, N = SVDQ_SHAPE
-    return 2 * M * K + 2 * K + 4 * K * RANK + M * K / 2 + M * K / 16 + 4 * M * RANK
+def time_segments(runs, stream):
+    """Replays every segment once on `stream` with CUDA events around each; returns the
+    milliseconds of each segment and of the whole region."""
+    import torch
+    ev = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for name, run in runs:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            run()
+        e1.record(stream)
+        ev.append((name, e0, e1))
+    end.record(stream)
+    torch.cuda.synchronize()
+    return {n: e0.elapsed_time(e1) for n, e0, e1 in ev}, start.elapsed_time(end)
 
 
-def k2_bytes():
-    M, K, N = SVDQ_SHAPE
-    return (N + M) * K * (0.5 + 1 / 16) + 2 * RANK * N + 2 * N + 4 * M * RANK + 2 * M * N
-
-
-def awq_bytes(m):
-    return AWQ_N * AWQ_K / 2 + 4 * AWQ_N * AWQ_K / 64 + 2 * m * AWQ_K + 2 * m * AWQ_N
+def time_dynamic_variant(P, wl, stream, steps, use_graph, reps=3):
+    """The dynamic-activation-scale layer (a variant, timed after the main region): kernel 5
+    alone and the whole layer (kernels 5, 1, 2), each a graph of `steps` launches or layers."""
+    import torch
+    out = {}
+    for name, fn in (("amax", wl.attn.amax), ("layer", wl.attn.dyn_layer)):
+        with torch.cuda.stream(stream):
+            for i in range(wl.attn.nsets):
+                fn(P, i)                              # warm-up (eager)
+        torch.cuda.synchronize()
+        run = capture(lambda i, fn=fn: fn(P, i), steps, stream, use_graph)
+        run()
+        best = None
+        for _ in range(reps):
+            ms, _ = time_segments([(name, run)], stream)
+            best = ms[name] if best is None else min(best, ms[name])
+        out[name + "_us"] = best * 1e3 / steps
+    M, K, N = ATTN
+    out["amax_gbs"] = 2.0 * M * K / (out["amax_us"] * 1e-6) / 1e9
+    out["layer_tflops"] = svdq_flops(M, K, N) / (out["layer_us"] * 1e-6) / 1e12
+    out["note"] = "g_a from the batch's amax (kernel 5) instead of calibration; best of %d graphs of %d" % (reps, steps)
+    return out
 
 
 def run_ours(args, world, rank, local):
     import torch
     import bit_diffusion_transformer_act_b200 as P
     dev = torch.device("cuda", torch.cuda.current_device())
+    props = torch.cuda.get_device_properties(dev)
+    l2_bytes = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+    sms = props.multi_processor_count
     peaks = load_peaks()
-    wl = Workload(P, dev)
+    wl = Workloads(P, dev, l2_bytes)
     stream = torch.cuda.Stream()
-    names = ["k1", "k2"] + ["awq%d" % m for m in AWQ_MS]
-
-    def launch(name, i):
-        if name == "k1":
-            wl.k1(P, i)
-        elif name == "k2":
-            wl.k2(P, i)
-        else:
-            wl.awq(P, i, int(name[3:]))
-
-    # one graph per kernel kind: NREP passes over the NSETS rotating copies (a batch of 24 launches),
-    # plus single-set graphs for remainders
-    with torch.cuda.stream(stream):
-        for i in range(NSETS):                       # eager warm-up (sets attributes, loads modules)
-            for n in names:
-                launch(n, i)
-    torch.cuda.synchronize()
-    graphs, singles = {}, {}
+    segs = wl.segments(P)
     use_graph = not args.no_graph
-    if use_graph:
-        for n in names:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(NREP):
-                    for i in range(NSETS):
-                        launch(n, i)
-            graphs[n] = g
-            singles[n] = []
-            for i in range(NSETS):
-                g1 = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g1, stream=stream):
-                    launch(n, i)
-                singles[n].append(g1)
-    torch.cuda.synchronize()
+    K = args.steps
 
-    def run_steps(nsteps, events):
-        """Runs nsteps steps on `stream`; appends (name, start, end, launches) event records."""
-        done = 0
-        while done < nsteps:
-            chunk = min(NSETS * NREP, nsteps - done)
-            for n in names:
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                if use_graph and chunk == NSETS * NREP:
-                    graphs[n].replay()
-                elif use_graph:
-                    for i in range(chunk):
-                        singles[n][i % NSETS].replay()
-                else:
-                    with torch.cuda.stream(stream):
-                        for i in range(chunk):
-                            launch(n, i % NSETS)
-                e1.record(stream)
-                if events is not None:
-                    events.append((n, e0, e1, chunk))
-            done += chunk
-
+    # warm-up: W steps of every segment, eager (sets kernel attributes, loads modules)
     with torch.cuda.stream(stream):
-        run_steps(max(args.warmup, 3), None)
+        for i in range(max(args.warmup, 3)):
+            for _, _, fn in segs:
+                fn(i)
+    torch.cuda.synchronize()
+    runs = [(name, capture(fn, K, stream, use_graph)) for name, _, fn in segs]
+    for _, run in runs:                              # one untimed replay (graph upload)
+        with torch.cuda.stream(stream):
+            run()
     torch.cuda.synchronize()
 
-    events = []
     barrier(world)
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clocks:
-        start.record(stream)
-        with torch.cuda.stream(stream):
-            run_steps(args.steps, events)
-        end.record(stream)
-        torch.cuda.synchronize()
+        seg_ms, total_ms = time_segments(runs, stream)
     barrier(world)
-    total_ms = start.elapsed_time(end)
-    per = {n: [0.0, 0] for n in names}
-    for n, e0, e1, c in events:
-        per[n][0] += e0.elapsed_time(e1)
-        per[n][1] += c
-    avg_ms = {n: per[n][0] / max(per[n][1], 1) for n in names}
-    svdq_ms = per["k1"][0] + per["k2"][0]
-    svdq_ms_max = allreduce_max(svdq_ms, world)
-    total_ms_max = allreduce_max(total_ms, world)
-    awq_ms = {m: per["awq%d" % m][0] for m in AWQ_MS}
-    awq_ms_max = {m: allreduce_max(awq_ms[m], world) for m in AWQ_MS}
     status = P.svdq_device_status()
     if status:
         raise RuntimeError("device status %d after the timed region" % status)
-    variants = {"svdq_dynamic_act_scale": time_dynamic_variant(P, wl, stream, use_graph)}
+    seg_ms_max = {n: allreduce_max(v, world) for n, v in seg_ms.items()}
+    total_ms_max = allreduce_max(total_ms, world)
+    launches = K * sum(c for _, c, _ in segs)
+    clk = clocks.summary()
 
-    value = job_rate(world, args.steps, svdq_flops(), svdq_ms_max) / 1e12
     fp4_peak = FP4_OVER_BF16 * peaks["bf16_tflops"]
-    k2_tflops = svdq_flops() / (avg_ms["k2"] * 1e-3) / 1e12
-    k1_gbs = k1_bytes() / (avg_ms["k1"] * 1e-3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    mhz = clk["sm_mhz"] or 1965.0
+    fp4_clock_peak = FP4_FLOP_PER_SM_CLK * sms * mhz * 1e6 / 1e12
+
+    def us(name):
+        return seg_ms[name] * 1e3 / K
+
+    M, Kd, N = ATTN
+    fl = svdq_flops(M, Kd, N)
+    value = job_rate(world, K, fl, seg_ms_max["attn_layer"]) / 1e12
+    k2_tflops = fl / (us("attn_k2") * 1e-6) / 1e12
+    k1_gbs = k1_bytes(M, Kd) / (us("attn_k1") * 1e-6) / 1e9
+    traffic, traffic_note = captured_traffic()
+
+    def layer_row(name, M_, K_, N_):
+        t = us(name)
+        fl_ = svdq_flops(M_, K_, N_)
+        by = k1_bytes(M_, K_) + k2_bytes(M_, K_, N_)
+        t_math = fl_ / (fp4_peak * 1e12) * 1e6
+        t_mem = by / (hbm * 1e9) * 1e6
+        return {"M": M_, "K": K_, "N": N_, "us": t, "tflops": fl_ / (t * 1e-6) / 1e12,
+                "frac_fp4": fl_ / (t * 1e-6) / 1e12 / fp4_peak, "gbs": by / (t * 1e-6) / 1e9,
+                "frac_hbm": by / (t * 1e-6) / 1e9 / hbm, "bound": "tensor" if t_math >= t_mem else "hbm",
+                "roofline_frac": max(t_math, t_mem) / t, "algorithmic_bytes": by, "flops": fl_}
+
     awq_per_m = {}
     for m in AWQ_MS:
-        gbs = awq_bytes(m) / (avg_ms["awq%d" % m] * 1e-3) / 1e9
-        agg = job_rate(world, args.steps, awq_bytes(m), awq_ms_max[m]) / 1e9
-        awq_per_m[str(m)] = {"us": avg_ms["awq%d" % m] * 1e3, "gbs": gbs, "gbs_all_ranks": agg,
-                             "frac_hbm": gbs / peaks["hbm_gbs"]}
-    awq_all = job_rate(world, args.steps, sum(awq_bytes(m) for m in AWQ_MS), sum(awq_ms_max.values())) / 1e9
+        t = us("awq%d" % m)
+        gbs = awq_bytes(m) / (t * 1e-6) / 1e9
+        awq_per_m[str(m)] = {"us": t, "gbs": gbs, "frac_hbm": gbs / hbm,
+                             "gbs_all_ranks": job_rate(world, K, awq_bytes(m), seg_ms_max["awq%d" % m]) / 1e9}
+    awq_all = job_rate(world, K, sum(awq_bytes(m) for m in AWQ_MS),
+                       sum(seg_ms_max["awq%d" % m] for m in AWQ_MS)) / 1e9
+
+    def qkv_row(m):
+        row = layer_row("qkv%d" % m, m, QKV_K, QKV_N)
+        t1, t2 = us("qkv%d_k1" % m), us("qkv%d_k2" % m)
+        g_bytes = k2_bytes(m, QKV_K, QKV_N)
+        row["kernels"] = {"quant_act_lowrank_kernel": {"us": t1, "frac_hbm": k1_bytes(m, QKV_K) / (t1 * 1e-6) / 1e9 / hbm},
+                          "nvfp4_gemm_kernel": {"us": t2, "tflops": svdq_flops(m, QKV_K, QKV_N) / (t2 * 1e-6) / 1e12,
+                                                "frac_hbm": g_bytes / (t2 * 1e-6) / 1e9 / hbm,
+                                                "roofline_frac": max(svdq_flops(m, QKV_K, QKV_N) / (fp4_peak * 1e12),
+                                                                     g_bytes / (hbm * 1e9)) / (t2 * 1e-6)}}
+        return row
+
+    configs = {"qkv_sweep": [qkv_row(m) for m in wl.qkv]}
+    fused = {}
+    for m in QKV_FUSED_MS:
+        if "qkv%d_fused" % m not in seg_ms:
+            continue
+        row = layer_row("qkv%d_fused" % m, m, QKV_K, QKV_N)
+        t_plain, t_torch = us("qkv%d" % m), us("qkv%d_torch_norm_rope" % m)
+        row.update({"plain_layer_us": t_plain, "unfused_us": t_plain + t_torch, "torch_norm_rope_us": t_torch,
+                    "speedup_vs_unfused": (t_plain + t_torch) / row["us"],
+                    "epilogue_cost_vs_plain": row["us"] / t_plain})
+        fused[str(m)] = row
+    configs["qkv_fused_rmsnorm_rope"] = {
+        "heads": QKV_HEADS, "head_dim": 128, "per_m": fused,
+        "note": "kernel 1 + the GEMM with the RMSNorm + RoPE epilogue, against the plain layer and the plain "
+                "layer followed by RMSNorm + RoPE as separate PyTorch operations (the unfused pipeline)"}
+    if wl.mlp_up is not None:
+        configs["mlp_pair"] = {"up": layer_row("mlp_up", *MLP_UP), "down_gelu_input": layer_row("mlp_down", *MLP_DOWN)}
+        t_pair = us("mlp_up") + us("mlp_down")
+        configs["mlp_pair"]["pair"] = {"us": t_pair, "tflops": (svdq_flops(*MLP_UP) + svdq_flops(*MLP_DOWN))
+                                       / (t_pair * 1e-6) / 1e12}
+        t_fused = us("mlp_up_fused") + us("mlp_down_gemm")
+        configs["mlp_pair"]["fused_gelu_requant"] = {
+            "up_fused_us": us("mlp_up_fused"), "down_gemm_us": us("mlp_down_gemm"), "pair_us": t_fused,
+            "tflops": (svdq_flops(*MLP_UP) + svdq_flops(*MLP_DOWN)) / (t_fused * 1e-6) / 1e12,
+            "speedup_vs_unfused_pair": t_pair / t_fused,
+            "note": "kernel 1 on X, the up GEMM with GELU and the down projection's activation pass in its "
+                    "epilogue (kernels 6, 7), then the down GEMM: the 4608 x 12288 hidden state is never stored"}
 
     result = {
         "metric": METRIC,
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
-        "steps": args.steps,
+        "steps": K,
         "warmup": args.warmup,
-        "ms_per_step": total_ms_max / args.steps,
+        "ms_per_step": total_ms_max / K,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -430,84 +615,126 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": "SVDQ W4A4 NVFP4 DiT attention projection M=4096 K=3072 N=3072 rank 32 group 16 "
-                        "+ AWQ W4A16 adaLN K=3072 N=18432 group 64 at M=1,2,4,8,16,32,64",
-            "svdq": {"M": SVDQ_SHAPE[0], "K": SVDQ_SHAPE[1], "N": SVDQ_SHAPE[2], "rank": RANK, "group": 16},
-            "awq": {"M": list(AWQ_MS), "K": AWQ_K, "N": AWQ_N, "group": 64},
-            "l2": "inputs, weights and outputs rotate over 8 resident copies (> 2x L2 per cycle); no flush",
-            "launch": "CUDA graphs of 24 launches per kernel (3 passes over the 8 copies)" if use_graph else "eager",
+                        "(kernel 1 chained into kernel 2)",
+            "also_per_step": "each kernel of that layer alone; AWQ W4A16 adaLN K=3072 N=18432 group 64 at "
+                             "M=1,2,4,8,16,32,64; SVDQ QKV K=3072 N=9216 at M=64,256,1024,4608,18432; "
+                             "SVDQ MLP up 4608x3072->12288 and down 4608x12288->3072 (GELU inputs)",
+            "l2": "every segment rotates over resident copies of inputs, weights and outputs touching "
+                  "more than 2x L2 per cycle; no flush",
+            "launch": ("one CUDA graph per segment holding exactly `steps` launches (or layers)" if use_graph
+                       else "eager"),
             "parallelism": "replicas x%d" % world,
             "seed": 0,
         },
-        "svdq_ms_per_step": svdq_ms_max / args.steps,
         "roofline": {
             "bound": "tensor", "achieved": k2_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-            "frac": k2_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
-            "traffic_unit": "bytes per launch (dram read + write, ncu, cold caches)",
-            "traffic_source": "profiles/nvfp4_gemm_attention_4096x3072x3072.md",
-            "kernel": "nvfp4_gemm_kernel<256>",
-            "peak_note": "dense FP4 = 4 x measured bf16 burst (%s), nominal 9/2.25 ratio" % peaks["source"],
+            "frac": k2_tflops / fp4_peak, "traffic": traffic,
+            "traffic_unit": "bytes per launch (dram read + write)", "traffic_note": traffic_note,
+            "kernel": "nvfp4_gemm_kernel<256> (attention M=4096 K=N=3072)",
+            "peak_note": "dense FP4 = 4 x measured bf16 burst (%s), the nominal 9/2.25 ratio" % peaks["source"],
+            "frac_clock_matched": k2_tflops / fp4_clock_peak,
+            "clock_matched_peak": fp4_clock_peak,
+            "clock_matched_note": "nominal dense FP4 issue rate (32768 FLOP per SM per clock) x %d SMs at the "
+                                  "median sampled SM clock" % sms,
+            "frac_of_9pf_datasheet": k2_tflops / 9000.0,
         },
         "kernels": {
-            "quant_act_lowrank_kernel": {"us": avg_ms["k1"] * 1e3, "bound": "hbm", "gbs": k1_gbs,
-                                         "frac": k1_gbs / peaks["hbm_gbs"], "bytes": k1_bytes()},
-            "nvfp4_gemm_kernel": {"us": avg_ms["k2"] * 1e3, "bound": "tensor", "tflops": k2_tflops,
-                                  "frac": k2_tflops / fp4_peak, "flops": svdq_flops(),
-                                  "frac_of_9pf_datasheet": k2_tflops / 9000.0},
-            "layer": {"us": (avg_ms["k1"] + avg_ms["k2"]) * 1e3,
-                      "tflops": svdq_flops() / ((avg_ms["k1"] + avg_ms["k2"]) * 1e-3) / 1e12},
+            "quant_act_lowrank_kernel": {"us": us("attn_k1"), "bound": "hbm", "gbs": k1_gbs, "frac": k1_gbs / hbm,
+                                         "bytes": k1_bytes(M, Kd)},
+            "nvfp4_gemm_kernel": {"us": us("attn_k2"), "bound": "tensor", "tflops": k2_tflops,
+                                  "frac": k2_tflops / fp4_peak, "flops": fl},
+            "layer_chained": {"us": us("attn_layer"), "tflops": fl / (us("attn_layer") * 1e-6) / 1e12,
+                              "frac_fp4": fl / (us("attn_layer") * 1e-6) / 1e12 / fp4_peak},
         },
-        "variants": variants,
-        "awq": {"value": awq_all, "unit": "GB/s", "frac_hbm": awq_all / peaks["hbm_gbs"], "per_m": awq_per_m,
-                "hbm_peak_gbs": peaks["hbm_gbs"]},
-        "gpu_launches": (2 + len(AWQ_MS)) * args.steps,
-        "clocks": clocks.summary(),
+        "configs": configs,
+        "awq": {"value": awq_all, "unit": "GB/s", "frac_hbm": awq_all / hbm, "per_m": awq_per_m,
+                "hbm_peak_gbs": hbm},
+        "variants": {"svdq_dynamic_act_scale": time_dynamic_variant(P, wl, stream, K, use_graph)},
+        "gpu_launches": launches,
+        "clocks": clk,
     }
-    result["e2e"] = e2e_ours(args, P, wl, dev, world)
+    del runs
+    result["e2e"] = e2e_ours(args, P, wl.attn, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline()
     return result
 
 
-def e2e_ours(args, P, wl, dev, world):
-    """The same layer through the public API with the input in pinned host memory and the
-    output read back to pinned host memory, every step inside the timed region."""
+def e2e_ours(args, P, case, dev, world, chunks=8):
+    """The attention layer through the public API with the input in pinned host memory and
+    the output read back to pinned host memory, every step inside the timed region.  The rows
+    go in `chunks` pieces through three streams -- host-to-device copies, the two kernels,
+    device-to-host copies -- so that both copy directions and the kernels overlap."""
     import torch
-    M, K, N = SVDQ_SHAPE
-    hX = torch.from_numpy(wl.host_X).to(torch.bfloat16).pin_memory()
+    M, K, N = case.M, case.K, case.N
+    s0 = case.sets[0]
+    hX = s0["X"].cpu().pin_memory()
     hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    s0 = wl.sets[0]
-    dX = torch.empty_like(s0["X"])
+    dX, codes, scales, U, Y = s0["X"], s0["codes"], s0["scales"], s0["U"], s0["Y"]
+    rows = M // chunks
+    assert rows % 128 == 0 and rows * chunks == M
+    sc_per_row_block = (K // 64) * 512
+    s_in, s_k, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(chunks)]
+    ev_k1 = [torch.cuda.Event() for _ in range(chunks)]
+    ev_k2 = [torch.cuda.Event() for _ in range(chunks)]
+    ev_out = [torch.cuda.Event() for _ in range(chunks)]
+    first = [True]
 
     def step():
-        dX.copy_(hX, non_blocking=True)
-        codes, scales, U = P.svdq_quantize_act_lowrank_down(dX, wl.smooth, s0["W"], wl.g_a, RANK,
-                                                            s0["codes"], s0["scales"], s0["U"])
-        P.svdq_w4a4_nvfp4_linear(codes, scales, U, wl.g_a, s0["W"], wl.g_w, M, N, K, RANK, s0["Y"])
-        hY.copy_(s0["Y"], non_blocking=True)
+        for c in range(chunks):
+            r0, r1 = c * rows, (c + 1) * rows
+            b0, b1 = (r0 // 128) * sc_per_row_block, (r1 // 128) * sc_per_row_block
+            with torch.cuda.stream(s_in):
+                if not first[0]:
+                    s_in.wait_event(ev_k1[c])         # the previous step's kernel 1 has read this chunk
+                dX[r0:r1].copy_(hX[r0:r1], non_blocking=True)
+                ev_in[c].record(s_in)
+            with torch.cuda.stream(s_k):
+                s_k.wait_event(ev_in[c])
+                P.svdq_quantize_act_lowrank_down(dX[r0:r1], case.smooth, s0["W"], case.g_a, RANK,
+                                                 codes[r0:r1], scales[b0:b1], U[r0:r1])
+                ev_k1[c].record(s_k)
+                if not first[0]:
+                    s_k.wait_event(ev_out[c])         # the previous step's output has left this chunk
+                P.svdq_w4a4_nvfp4_linear(codes[r0:r1], scales[b0:b1], U[r0:r1], case.g_a, s0["W"], case.g_w,
+                                         rows, N, K, RANK, Y[r0:r1])
+                ev_k2[c].record(s_k)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_k2[c])
+                hY[r0:r1].copy_(Y[r0:r1], non_blocking=True)
+                ev_out[c].record(s_out)
+        first[0] = False
 
     for _ in range(3):
         step()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s_in)
+    s_k.wait_event(e0)                               # every stream starts after e0
+    s_out.wait_event(e0)
     for _ in range(args.e2e_steps):
         step()
-    e1.record()
+    s_out.wait_event(ev_k2[-1])
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = allreduce_max(e0.elapsed_time(e1), world)
-    val = world * args.e2e_steps * svdq_flops() / (ms * 1e-3) / 1e12
+    val = world * args.e2e_steps * svdq_flops(M, K, N) / (ms * 1e-3) / 1e12
+    ok = bool(torch.equal(hY.to(dev), Y))
     return {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": hX.numel() * 2,
-            "d2h_bytes_per_step": hY.numel() * 2, "steps": args.e2e_steps,
-            "note": "SVDQ layer via the C ABI; pinned host X in, pinned host Y out, per step"}
+            "d2h_bytes_per_step": hY.numel() * 2, "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps,
+            "note": "attention layer via the public API; pinned host X in, pinned host Y out, every step, "
+                    "in %d row chunks over copy-in, kernel and copy-out streams" % chunks,
+            "host_output_matches_device": ok}
 
 
 # ---------------------------------------------------------------- CPU oracle legs
 
 def _oracle_layer_prepared():
     import synth
-    from oracle import awq, nvfp4, svdq
-    M, K, N = SVDQ_SHAPE
+    from oracle import nvfp4, svdq
+    M, K, N = ATTN
     w = synth.svdq_workload(M, K, N)
     cw, sw, gw = svdq.quantize_weights(w.R)                 # offline, like packing (untimed)
     wq = nvfp4.dequantize(cw, sw, gw)
@@ -516,7 +743,6 @@ def _oracle_layer_prepared():
 
 
 def _oracle_svdq_rows(w, wq, rows):
-    import numpy as np
     from oracle import nvfp4, svdq
     X = w.X[:rows]
     cx, sx = svdq.quantize_activations(X, w.smooth_inv, w.g_a)
@@ -541,14 +767,14 @@ def cpu_baseline():
     """The oracle as it stands on this host's cores: the full attention layer and the full
     AWQ weight at M=64 (weights quantized once beforehand, as the packer does offline)."""
     w, wq, a = _oracle_layer_prepared()
-    M, K, N = SVDQ_SHAPE
+    M, K, N = ATTN
     t = time.perf_counter()
     _oracle_svdq_rows(w, wq, M)
     dt = time.perf_counter() - t
     t = time.perf_counter()
     _oracle_awq_rows(a, 64, AWQ_N)
     da = time.perf_counter() - t
-    return {"value": svdq_flops() / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+    return {"value": svdq_flops(M, K, N) / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": "whole attention layer M=4096 K=N=3072 in float64 NumPy (activation quantization, "
                       "dequantize, matmul, low-rank, bias), %.2f s; weights quantized beforehand" % dt,
             "awq": {"value": awq_bytes(64) / da / 1e9, "unit": "GB/s", "sample": "M=64, whole N=18432 (%.2f s)" % da}}
@@ -563,14 +789,14 @@ def run_reference(args, world, rank):
     _oracle_svdq_rows(w, wq, 64)
     per_row = (time.perf_counter() - t) / 64
     budget = 120.0 / max(args.steps + args.warmup, 1)       # whole run within a few minutes
-    rows = int(max(1, min(SVDQ_SHAPE[0], budget / per_row)))
+    rows = int(max(1, min(ATTN[0], budget / per_row)))
     for _ in range(args.warmup):
         _oracle_svdq_rows(w, wq, rows)
     t = time.perf_counter()
     for _ in range(args.steps):
         _oracle_svdq_rows(w, wq, rows)
     dt = time.perf_counter() - t
-    M, K, N = SVDQ_SHAPE
+    M, K, N = ATTN
     val = args.steps * 2.0 * rows * N * K / dt / 1e12
     return {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -583,16 +809,27 @@ def run_reference(args, world, rank):
 
 
 def run_profile_case(args):
-    """Each kernel launched eagerly `steps` times on one resident copy of the workload."""
+    """Each kernel launched eagerly `steps` times on one resident copy of a workload (small
+    enough for ncu captures): the attention layer and the AWQ layer, the QKV layer at M = 64,
+    or the fused QKV layer at M = 4608."""
     import torch
     import bit_diffusion_transformer_act_b200 as P
-    global NSETS
-    NSETS = 1
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = Workload(P, dev)
+    l2 = 126 * 2 ** 20
+    import synth
+    if args.case == "attention":
+        attn = SvdqCase(P, dev, synth.svdq_workload(*ATTN), ATTN[0], l2, nsets=1)
+        awq = AwqCase(P, dev, l2, nsets=1)
+        jobs = [("k1", lambda: attn.k1(P, 0)), ("k2", lambda: attn.k2(P, 0))] + \
+               [("awq%d" % m, (lambda m=m: awq.run(P, 0, m))) for m in AWQ_MS]
+    elif args.case == "qkv64":
+        c = SvdqCase(P, dev, synth.svdq_workload(64, QKV_K, QKV_N), 64, l2, nsets=1)
+        jobs = [("k1", lambda: c.k1(P, 0)), ("k2", lambda: c.k2(P, 0))]
+    else:
+        c = SvdqCase(P, dev, synth.svdq_workload(4608, QKV_K, QKV_N), 4608, l2, nsets=1)
+        c.set_qkv(dev, QKV_HEADS, QKV_EPS)
+        jobs = [("k2", lambda: c.k2(P, 0)), ("qkv_fused", lambda: c.qkv_fused(P, 0))]
     out = {}
-    jobs = [("k1", lambda: wl.k1(P, 0)), ("k2", lambda: wl.k2(P, 0))] + \
-           [("awq%d" % m, (lambda m=m: wl.awq(P, 0, m))) for m in AWQ_MS]
     for name, fn in jobs:
         fn()
         torch.cuda.synchronize()
