@@ -68,7 +68,7 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="one resident copy, eager launches of every kernel (for ncu captures); prints timings")
-    ap.add_argument("--case", default="attention", choices=["attention", "qkv64", "qkv4608_fused"],
+    ap.add_argument("--case", default="attention", choices=["attention", "qkv64", "qkv4608_fused", "mlp_fused"],
                     help="workload of --profile-case")
     return ap.parse_args(argv)
 
@@ -825,10 +825,15 @@ def run_profile_case(args):
     elif args.case == "qkv64":
         c = SvdqCase(P, dev, synth.svdq_workload(64, QKV_K, QKV_N), 64, l2, nsets=1)
         jobs = [("k1", lambda: c.k1(P, 0)), ("k2", lambda: c.k2(P, 0))]
-    else:
+    elif args.case == "qkv4608_fused":
         c = SvdqCase(P, dev, synth.svdq_workload(4608, QKV_K, QKV_N), 4608, l2, nsets=1)
         c.set_qkv(dev, QKV_HEADS, QKV_EPS)
         jobs = [("k2", lambda: c.k2(P, 0)), ("qkv_fused", lambda: c.qkv_fused(P, 0))]
+    else:
+        up = SvdqCase(P, dev, synth.svdq_workload(*MLP_UP), MLP_UP[0], l2, nsets=1)
+        down = SvdqCase(P, dev, synth.svdq_workload(*MLP_DOWN, gelu_input=True), MLP_DOWN[0], l2, nsets=1)
+        f = MlpFused(P, dev, up, down)
+        jobs = [("up_k2", lambda: up.k2(P, 0)), ("up_fused", lambda: f.up_fused(P, 0))]
     out = {}
     for name, fn in jobs:
         fn()

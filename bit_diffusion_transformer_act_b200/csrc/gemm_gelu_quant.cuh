@@ -19,7 +19,8 @@
 //   warp 1     tensor memory, block-scaled and low-rank MMAs of the up projection (leader).
 //   warps 2-9  epilogue: a warp owns 32 rows (its tensor-memory lane quarter) and two of the
 //              tile's four 32-column chunks.  Per element y = alpha acc + b, rounded to bf16;
-//              h = bf16(GELU(y)) with erff in fp32; h is written into a 128 x 64 shared-memory
+//              h = bf16(GELU(y)) in fp32 pairs (erfc by a published Chebyshev fit, below); h is
+//              written into a 128 x 64 shared-memory
 //              slab (the A operand of the low-rank MMA, 128-byte swizzle) and quantized in
 //              registers with the down projection's smoothing and scale (the quantizer of
 //              kernel 1: codes and scale bytes stored straight to global memory).
@@ -70,8 +71,10 @@ constexpr int OFF_SLAB = STAGES * STAGE_BYTES;
 constexpr int OFF_L1 = OFF_SLAB + 2 * SLAB_BYTES;
 constexpr int OFF_BAR = OFF_L1 + 2 * L1BUF_BYTES;
 constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
-constexpr int OFF_VEC = (OFF_MISC + 64 + 127) / 128 * 128;   // per epilogue warp: bias, then smooth_inv (BN bf16 each)
-constexpr int SMEM_BYTES = OFF_VEC + kEpiWarps * 512 + 1024;
+// per epilogue warp: the tile's bias (BN bf16), then its -smooth_inv (BN fp32)
+constexpr int VEC_BYTES = BN * 2 + BN * 4;
+constexpr int OFF_VEC = (OFF_MISC + 64 + 127) / 128 * 128;
+constexpr int SMEM_BYTES = OFF_VEC + kEpiWarps * VEC_BYTES + 1024;
 // tensor memory: accumulators [0, 128) and [128, 256), scale regions [256, 320), U [320, 352)
 constexpr int SF_COLS = 4 * (BK / 64) + 4 * (BK / 64);
 constexpr uint32_t TM_SF = 2 * BN;
@@ -113,8 +116,49 @@ __device__ __forceinline__ uint32_t idesc_u() {
          (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-__device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f));
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU(x) = x Phi(x) = x erfc(-x / sqrt 2) / 2 for two values at once.  erfc is the Chebyshev
+// fit of Numerical Recipes (Press, Teukolsky, Vetterling, Flannery, 2nd ed., section 6.2,
+// "erfcc"): for z >= 0, erfc(z) = t exp(-z^2 + P(t)) with t = 1 / (1 + z/2) and a degree-9
+// polynomial P, fractional error below 1.2e-7 everywhere; erfc(-z) = 2 - erfc(z).  Branch-free,
+// Horner's rule on packed fp32 pairs, the reciprocal and the exponential on the SFU (a few ulp).
+// Relative error against x Phi(x) (float32 evaluation of this sequence): below 2.2e-6 for
+// |x| <= 4 and 2.1e-5 anywhere (the fp32 rounding of the exponent -z^2 + P grows with z^2) --
+// far below half a bf16 ulp (2^-9), so the bf16 rounding that follows differs from that of the
+// exact value only next to a midpoint, by one ulp.
+// Large negative x give -0 (as x Phi(x) rounds), large positive x give x.
+__device__ __forceinline__ uint64_t gelu2(uint64_t x2) {
+  const uint64_t nz = f32x2_mul(x2, f32x2_pack(0.70710678118654752f, 0.70710678118654752f));   // -z
+  float z0, z1;
+  f32x2_unpack(nz, z0, z1);
+  z0 = -z0;
+  z1 = -z1;
+  const float a0 = fabsf(z0), a1 = fabsf(z1);
+  const uint64_t t = f32x2_pack(rcp_approx(fmaf(0.5f, a0, 1.0f)), rcp_approx(fmaf(0.5f, a1, 1.0f)));
+  auto c2 = [](float c) { return f32x2_pack(c, c); };
+  uint64_t q = c2(0.17087277f);
+  q = f32x2_fma(q, t, c2(-0.82215223f));
+  q = f32x2_fma(q, t, c2(1.48851587f));
+  q = f32x2_fma(q, t, c2(-1.13520398f));
+  q = f32x2_fma(q, t, c2(0.27886807f));
+  q = f32x2_fma(q, t, c2(-0.18628806f));
+  q = f32x2_fma(q, t, c2(0.09678418f));
+  q = f32x2_fma(q, t, c2(0.37409196f));
+  q = f32x2_fma(q, t, c2(1.00002368f));
+  q = f32x2_fma(q, t, c2(-1.26551223f));
+  // exponent -z^2 + P(t), in base 2
+  const uint64_t e = f32x2_mul(f32x2_fma(nz, f32x2_pack(z0, z1), q), c2(1.44269504088896341f));
+  float e0, e1, t0, t1;
+  f32x2_unpack(e, e0, e1);
+  f32x2_unpack(t, t0, t1);
+  const float r0 = t0 * ex2_approx(e0), r1 = t1 * ex2_approx(e1);
+  const float c0 = z0 < 0.f ? 2.0f - r0 : r0, c1 = z1 < 0.f ? 2.0f - r1 : r1;   // erfc(z)
+  return f32x2_mul(f32x2_mul(x2, c2(0.5f)), f32x2_pack(c0, c1));
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -376,7 +420,7 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     const int ew = warp - 2;
     const int eh = ew >> 2;                        // chunks eh and eh + 2 of each tile
     const float alpha = p.alpha;
-    uint8_t* svec = gbase + OFF_VEC + ew * 512;    // [0, 256): bias; [256, 512): smooth_inv (negated in use)
+    uint8_t* svec = gbase + OFF_VEC + ew * VEC_BYTES;   // [0, 256): bias (bf16); [256, 768): -smooth_inv (fp32)
     const int r = quarter * 32 + lane;             // this thread's row within the CTA's 128
     int i = 0, parts = 0;
     for (int t = t_begin; t < t_end; ++t, ++i) {
@@ -385,11 +429,12 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const int m = mblk + r;
       const int n0 = nt * BN;
       const int b = i & 1;
-      if (lane < 16) {
+      if (lane < 16)
         *reinterpret_cast<uint4*>(svec + lane * 16) = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
-      } else {
-        *reinterpret_cast<uint4*>(svec + lane * 16) =
-            __ldg(reinterpret_cast<const uint4*>(p.smooth + n0) + (lane - 16));
+      {
+        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(p.smooth + n0) + lane);   // 4 factors per lane
+        *reinterpret_cast<float4*>(svec + 256 + lane * 16) =
+            make_float4(-bf16lo_to_f32(sv.x), -bf16hi_to_f32(sv.x), -bf16lo_to_f32(sv.y), -bf16hi_to_f32(sv.y));
       }
       __syncwarp();
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full(b), (i >> 1) & 1, abort_flag, 38))) break;
@@ -420,10 +465,14 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int k = q * 8 + w * 2;
-            const float y0 = fmaf(alpha, __uint_as_float(R[jj][k]), bf16lo_to_f32(bw[w]));
-            const float y1 = fmaf(alpha, __uint_as_float(R[jj][k + 1]), bf16hi_to_f32(bw[w]));
+            const uint64_t y = f32x2_fma(f32x2_pack(alpha, alpha), f32x2_pack(__uint_as_float(R[jj][k]),
+                                                                               __uint_as_float(R[jj][k + 1])),
+                                         f32x2_pack(bf16lo_to_f32(bw[w]), bf16hi_to_f32(bw[w])));
+            float y0, y1, h0, h1;
+            f32x2_unpack(y, y0, y1);
             const uint32_t yb = pack_bf16x2(y0, y1);
-            hw[q * 4 + w] = pack_bf16x2(gelu_erf(bf16lo_to_f32(yb)), gelu_erf(bf16hi_to_f32(yb)));
+            f32x2_unpack(gelu2(f32x2_pack(bf16lo_to_f32(yb), bf16hi_to_f32(yb))), h0, h1);
+            hw[q * 4 + w] = pack_bf16x2(h0, h1);
           }
         }
         // the slab must have been consumed by the low-rank MMAs two slabs back
@@ -447,7 +496,7 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         __syncwarp();
         if (lane == 0) mbar_arrive_remote_cluster(map_to_cta(slab_ready(buf), 0));
         // the down projection's activation pass on h: -h smooth_inv in pairs, two 16-groups
-        const uint32_t* sm2 = reinterpret_cast<const uint32_t*>(svec + 256 + c * 64);
+        const uint64_t* sm2 = reinterpret_cast<const uint64_t*>(svec + 256 + c * 128);   // -smooth_inv pairs
         uint32_t sc2 = 0;
         uint2 cb[2];
 #pragma unroll
@@ -455,9 +504,8 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           uint64_t nx[8];
 #pragma unroll
           for (int w = 0; w < 8; ++w) {
-            const uint32_t hv = hw[gq * 8 + w], sv = sm2[gq * 8 + w];
-            nx[w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(hv), bf16hi_to_f32(hv)),
-                              f32x2_pack(-bf16lo_to_f32(sv), -bf16hi_to_f32(sv)));
+            const uint32_t hv = hw[gq * 8 + w];
+            nx[w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(hv), bf16hi_to_f32(hv)), sm2[gq * 8 + w]);
           }
           sc2 |= quantize_group(nx, p.g, p.inv_g, cb[gq]) << (8 * gq);
         }

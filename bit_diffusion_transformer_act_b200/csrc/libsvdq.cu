@@ -138,6 +138,23 @@ int launch_status() {
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
+// The failure path of every kernel's bounded waits, on its own: one warp waits (through the
+// same mbar_wait_bounded) for a phase of a shared-memory mbarrier at which nothing ever
+// arrives, so the wait runs out after its limit, records SVDQ_ERR_TIMEOUT (site 99) in the
+// device status word and the kernel returns.  No copy or tensor-core operation is in flight.
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = svdq::smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    svdq::mbar_init(b, 1);
+    abort_flag = 0;
+    svdq::fence_mbar_init();
+  }
+  __syncwarp();
+  (void)__all_sync(0xFFFFFFFFu, svdq::mbar_wait_bounded(b, 0, &abort_flag, 99));
+}
+
 }  // namespace
 
 extern "C" {
@@ -661,6 +678,13 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     else SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<64>, k4::Cfg<64>::SMEM, k4::kThreads, q);
   }
 #undef SVDQ_AWQ_LAUNCH
+  return launch_status();
+}
+
+int svdq_selftest_wait_timeout(void* stream) {
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
   return launch_status();
 }
 

@@ -51,6 +51,7 @@ def _load():
         "svdq_unswizzle_scales": ([vp, i, i, vp], i),
         "svdq_swizzle_scales": ([vp, i, i, vp], i),
         "svdq_device_status": ([i], i),
+        "svdq_selftest_wait_timeout": ([vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -65,7 +66,7 @@ EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes"
             "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status",
             "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn",
             "svdq_act_amax_noalloc", "svdq_w4a4_nvfp4_linear_qkv", "svdq_gelu_quant_workspace_bytes",
-            "svdq_w4a4_nvfp4_linear_gelu_quant")
+            "svdq_w4a4_nvfp4_linear_gelu_quant", "svdq_selftest_wait_timeout")
 
 
 def _check(fn, st):

@@ -290,6 +290,14 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales,
 int svdq_unswizzle_scales(const void* swizzled, int rows, int K, uint8_t* out);
 int svdq_swizzle_scales(const uint8_t* plain, int rows, int K, void* swizzled);
 
+/* Diagnostic of the failure path (the pages have no counterpart): launches one warp that waits,
+ * through the same bounded wait as every kernel, for an mbarrier phase at which nothing
+ * arrives.  The wait gives up after its limit (about one second), records SVDQ_ERR_TIMEOUT in
+ * the device status word and the kernel returns; no copy or tensor-core operation is in
+ * flight, so the context stays usable.  Returns the launch status; read the outcome with
+ * svdq_device_status.  Asynchronous on `stream`. */
+int svdq_selftest_wait_timeout(void* stream);
+
 /* Reads (and with clear != 0, resets) the device-side status word of the
  * current device that kernels set when a bounded wait runs out or a dynamic
  * scale product is out of range.  Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (which

@@ -305,7 +305,9 @@ def _run_awq(P, a, bias=None):
 
 
 # M <= 8: the mma.sync kernel; 9 <= M <= 64: the tcgen05 kernel with 16, 32 or 64 token columns
-@pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (9, 256, 64), (12, 512, 192),
+# (K >= 1024 with an even stage count splits the K chain of kernel 3 between two CTAs)
+@pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (2, 1024, 320), (7, 1536, 192),
+                                   (9, 256, 64), (12, 512, 192),
                                    (16, 1024, 256), (24, 1024, 384), (33, 512, 320), (48, 768, 448),
                                    (64, 256, 128), (64, 1536, 512)])
 def test_awq_shapes(P, M, K, N):
@@ -315,11 +317,11 @@ def test_awq_shapes(P, M, K, N):
     check_output(Y, oawq.forward(a.X, a.q, a.scales, a.zeros, b))
 
 
-@pytest.mark.parametrize("M", [5, 40])
-def test_awq_integer_case_is_exact(P, M):
+@pytest.mark.parametrize("M,K", [(5, 512), (40, 512), (6, 2048)])
+def test_awq_integer_case_is_exact(P, M, K):
     # s = 1, z = 8, small integer activations: every partial sum is an exact integer in fp32
     rng = np.random.default_rng(3)
-    K, N = 512, 128
+    N = 128
     a = synth.awq_workload(M, K, N)
     a.X[:] = rng.integers(-4, 5, size=(M, K))
     a.scales[:] = 1.0
