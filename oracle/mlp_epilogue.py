@@ -24,10 +24,13 @@ from .formats import bf16_round
 
 
 def gelu(x):
-    """x * Phi(x) with the standard normal distribution function Phi (the erf form)."""
+    """x * Phi(x) with the standard normal distribution function Phi (the erf form of GELU),
+    evaluated as Phi(x) = erfc(-x / sqrt 2) / 2: the same function as (1 + erf(x / sqrt 2)) / 2,
+    but float64 keeps its relative accuracy where Phi is tiny (1 + erf cancels for x below about
+    -7, and is exactly 0 from about -8.3 on although x Phi(x) is still a normal bf16 value)."""
     x = np.asarray(x, dtype=np.float64)
-    erf = np.vectorize(math.erf, otypes=[np.float64])
-    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+    erfc = np.vectorize(math.erfc, otypes=[np.float64])
+    return 0.5 * x * erfc(-x / math.sqrt(2.0))
 
 
 def hidden_state(y_up):

@@ -44,7 +44,8 @@ def test_requantize_applies_the_down_projection_smoothing_and_scale():
 
 def _gelu_decimal(x, digits=60):
     """x Phi(x) from the Maclaurin series of erf in `digits`-digit decimal arithmetic (an
-    evaluation independent of math.erf, accurate far beyond float64 for |x| <= 8)."""
+    evaluation independent of math.erf / math.erfc; with enough digits it stays accurate in the
+    tails, where the series' terms grow to about e^(x^2 / 2) before they cancel)."""
     from decimal import Decimal, getcontext
     getcontext().prec = digits
     X = Decimal(x)
@@ -84,3 +85,16 @@ def test_hidden_state_rounds_the_exact_gelu_at_its_nearest_bf16_midpoint():
     assert E.hidden_state(np.array([ys[i]]))[0] == expect
     # and float64 agrees with the 60-digit evaluation to well below the distance
     assert abs(Decimal(float(g[i])) - exact) < Decimal(float(dist[i] * abs(g[i]))) / 1000
+
+
+def test_gelu_keeps_relative_accuracy_in_the_negative_tail():
+    # at x = -10, Phi(x) = 7.6e-24: 1 + erf(x / sqrt 2) rounds to 0 in float64, the erfc form
+    # keeps full relative accuracy.  The reference is the decimal series at 150 digits.
+    from decimal import Decimal
+    for x in (-6.0, -8.0, -10.0, -12.5):
+        exact = _gelu_decimal(x, digits=150)
+        got = E.gelu(np.array([x]))[0]
+        assert got != 0.0
+        assert abs(Decimal(got) - exact) <= abs(exact) * Decimal("1e-13"), (x, got, exact)
+    # and its bf16 rounding is a normal, non-zero value there
+    assert E.hidden_state(np.array([-10.0]))[0] < 0.0
