@@ -106,15 +106,17 @@ def quantize_e2m1(v):
 
 
 def bf16_round(x):
-    """Round float64/float32 values to the nearest bfloat16 (ties to even), as float64.
+    """Round float64 values to the nearest bfloat16 (ties to even), once, as float64.
 
-    bfloat16 keeps the top 16 bits of the IEEE float32 pattern; the value is
-    first rounded to float32 (exact for every input used here, which already
-    fit in float32), then the low 16 bits are rounded away with ties to even.
+    bfloat16 has 8 significant bits and the exponent range of float32 (normal down to 2^-126,
+    subnormal steps of 2^-133).  The rounding is done straight from the float64 value: going
+    through float32 first would round twice, and a value just beside a bf16 midpoint that
+    float32 rounds onto the midpoint would then tip by ties-to-even.  Values beyond the largest
+    bf16 round to 2^128 (infinity when stored); zeros keep their sign; NaN stays NaN.
     """
-    f = np.asarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    u = (u + 0x7FFF + lsb) >> 16
-    out = (u << 16).astype(np.uint32).view(np.float32)
-    return out.astype(np.float64)
+    v = np.asarray(x, dtype=np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        _, e = np.frexp(v)                              # |v| in [2^(e-1), 2^e)
+        shift = np.maximum(e - 8, -133)                 # weight of the last kept bit
+        out = np.ldexp(np.rint(np.ldexp(v, -shift)), shift)   # rint: to nearest, ties to even
+    return np.where((v == 0.0) | ~np.isfinite(v), v, out)

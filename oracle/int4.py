@@ -32,18 +32,16 @@ it by far more than float64's rounding error.
 
 import numpy as np
 
+from .formats import bf16_round
+
 GROUP = 64
 CODE_MIN, CODE_MAX = -8, 7
 
 
 def bf16_rne(v):
-    """float64 values rounded to the nearest bfloat16 (ties to even), directly from float64
-    (no intermediate float32 rounding).  Normal range only (|v| >= 2^-126) or zero."""
-    v = np.asarray(v, dtype=np.float64)
-    m, e = np.frexp(v)                               # v = m 2^e, |m| in [0.5, 1)
-    q = np.rint(m * 256.0)                           # 8 significant bits, ties to even
-    out = np.ldexp(q, e - 8)
-    return np.where(v == 0.0, 0.0, out)
+    """float64 values rounded to the nearest bfloat16 (ties to even), once, straight from
+    float64 (formats.bf16_round)."""
+    return bf16_round(v)
 
 
 def quantize(x):

@@ -35,14 +35,16 @@ def gelu(x):
 
 def hidden_state(y_up):
     """h = bf16(GELU(bf16(y))): the hidden state as the unfused pipeline stores it -- the up
-    projection's output rounded to bf16, its GELU evaluated here in float64 (essentially exact)
-    and rounded once to bf16.
+    projection's output rounded to bf16, its GELU evaluated here in float64 (the erfc form:
+    essentially exact, relative error about 1e-16 everywhere) and rounded once to bf16.
 
-    A kernel that evaluates GELU in fp32 (a few ulp of error) rounds to the same bf16 value
-    except where the exact GELU lies within that error of a bf16 rounding midpoint, and there it
-    may land one bf16 ulp away.  The contract a fused kernel is held to is therefore stated on
-    its own intermediate values: its h is within one bf16 ulp of hidden_state(its own bf16 y),
-    and its codes and scales equal quantize_activations of its own h bit for bit."""
+    Since bf16(y) takes 65536 values, h is a function of 16 bits; a kernel may take it from a
+    table of this function (computed in double precision and rounded once, it equals this one
+    for every input).  A kernel that evaluates GELU in fp32 instead rounds the same way except
+    where the exact value lies within that evaluation's error of a bf16 midpoint.  The contract
+    a fused kernel is held to is stated on its own intermediate values: its h equals (or, with
+    an fp32 GELU, lies within one bf16 ulp of) hidden_state of its own bf16 y, and its codes and
+    scales equal quantize_activations of its own h bit for bit."""
     return bf16_round(gelu(bf16_round(np.asarray(y_up, dtype=np.float64))))
 
 

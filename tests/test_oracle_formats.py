@@ -111,3 +111,25 @@ def test_bf16_round_vs_torch():
     x = np.concatenate([rng.standard_normal(100000) * 10, rng.uniform(-1, 1, 1000) * 1e-30]).astype(np.float32)
     ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
     assert np.array_equal(F.bf16_round(x), ref)
+
+
+def test_bf16_round_is_a_single_rounding_from_float64_including_subnormals():
+    # float32 values (normal and subnormal): the same as torch's float32 -> bfloat16 cast
+    rng = np.random.default_rng(9)
+    v = (rng.standard_normal(50000) * np.exp2(rng.integers(-149, 127, 50000))).astype(np.float32)
+    v = v[np.isfinite(v)]
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(F.bf16_round(v.astype(np.float64)), ref)
+    # a float64 just above the midpoint 1 + 2^-8 rounds up, although float32 would first land on
+    # the midpoint and then tie to even (down)
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert F.bf16_round(np.array([x]))[0] == 1.0 + 2.0 ** -7
+    # bf16 subnormals: steps of 2^-133; a quarter step rounds down, three quarters up, a half to even
+    s = 2.0 ** -133
+    assert F.bf16_round(np.array([8 * s + s / 4, 8 * s + 3 * s / 4, 9 * s + s / 2, 10 * s + s / 2])).tolist() == \
+        [8 * s, 9 * s, 10 * s, 10 * s]
+    assert F.bf16_round(np.array([s / 2, s / 2 + 2.0 ** -160])).tolist() == [0.0, s]
+    # signs, zeros, infinities, NaN, overflow
+    out = F.bf16_round(np.array([-0.0, np.inf, -np.inf, np.nan, 2.0 ** 128 * 0.9999]))
+    assert np.signbit(out[0]) and out[0] == 0.0 and out[1] == np.inf and out[2] == -np.inf and np.isnan(out[3])
+    assert out[4] == 2.0 ** 128
