@@ -334,6 +334,39 @@ class SvdqCase:
                                      self.M, self.N, self.K, RANK, s["Y"])
 
 
+class Int4Case:
+    """The attention layer in the int4 / group-64 row (the same seeded workload), rotating sets."""
+
+    def __init__(self, P, dev, w, M, l2_bytes):
+        import torch
+        import synth
+        K, N = w.K, w.N
+        blob = P.svdq_int4_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2), synth.bf16_bits(w.bias),
+                                        synth.bf16_bits(w.smooth_inv))
+        self.M, self.K, self.N = M, K, N
+        self.smooth = bf16_dev(w.smooth_inv, dev)
+        X = bf16_dev(w.X[:M], dev)
+        blob_d = torch.from_numpy(blob).to(dev)
+        self.nsets = n_sets(blob.nbytes + 2 * M * K + M * K + 2 * M * N, l2_bytes)
+        self.sets = [{"X": X.clone(), "W": blob_d.clone(),
+                      "codes": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                      "scales": torch.empty((K // 64, M), dtype=torch.bfloat16, device=dev),
+                      "U": torch.empty((M, 2 * RANK), dtype=torch.bfloat16, device=dev),
+                      "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev)} for _ in range(self.nsets)]
+
+    def k1(self, P, i):
+        s = self.sets[i % self.nsets]
+        P.svdq_int4_quantize_act_lowrank_down(s["X"], self.smooth, s["W"], RANK, s["codes"], s["scales"], s["U"])
+
+    def k2(self, P, i):
+        s = self.sets[i % self.nsets]
+        P.svdq_w4a4_int4_linear(s["codes"], s["scales"], s["U"], s["W"], self.M, self.N, self.K, RANK, s["Y"])
+
+    def layer(self, P, i):
+        self.k1(P, i)
+        self.k2(P, i)
+
+
 class MlpFused:
     """The MLP pair with the up projection's fused epilogue (GELU + the down projection's
     activation pass): kernel 1 on X, kernels 6 and 7, then the down projection's GEMM on their
@@ -344,6 +377,7 @@ class MlpFused:
         self.up, self.down = up, down
         M, F = up.M, up.N
         self.ws_bytes = P.svdq_gelu_quant_workspace_bytes(M, F)
+        self.gelu = P.svdq_gelu_table_fill(device=dev)
         self.nsets = min(up.nsets, down.nsets)
         self.sets = [{"codes": torch.empty((M, F // 2), dtype=torch.uint8, device=dev),
                       "scales": torch.empty((P.svdq_act_scale_bytes(M, F),), dtype=torch.uint8, device=dev),
@@ -355,7 +389,7 @@ class MlpFused:
         self.up.k1(P, i % self.nsets)
         P.svdq_w4a4_nvfp4_linear_gelu_quant(u["codes"], u["scales"], u["U"], self.up.g_a, u["W"], self.up.g_w,
                                             self.up.M, self.up.N, self.up.K, self.down.smooth, d["W"], self.down.g_a,
-                                            RANK, s["codes"], s["scales"], s["U"], s["ws"])
+                                            RANK, s["codes"], s["scales"], s["U"], s["ws"], gelu_table=self.gelu)
 
     def down_gemm(self, P, i):
         d, s = self.down.sets[i % self.nsets], self.sets[i % self.nsets]
@@ -390,7 +424,9 @@ class AwqCase:
 class Workloads:
     def __init__(self, P, dev, l2_bytes, extra=True):
         import synth
-        self.attn = SvdqCase(P, dev, synth.svdq_workload(*ATTN), ATTN[0], l2_bytes)
+        wa = synth.svdq_workload(*ATTN)
+        self.attn = SvdqCase(P, dev, wa, ATTN[0], l2_bytes)
+        self.int4 = Int4Case(P, dev, wa, ATTN[0], l2_bytes) if extra else None
         self.awq = AwqCase(P, dev, l2_bytes)
         self.qkv, self.mlp_up, self.mlp_down = {}, None, None
         if extra:
@@ -409,6 +445,10 @@ class Workloads:
                ("attn_k1", 1, lambda i: self.attn.k1(P, i)),
                ("attn_k2", 1, lambda i: self.attn.k2(P, i))]
         seg += [("awq%d" % m, 1, (lambda i, m=m: self.awq.run(P, i, m))) for m in AWQ_MS]
+        if self.int4 is not None:
+            seg += [("int4_layer", 2, lambda i: self.int4.layer(P, i)),
+                    ("int4_k1", 1, lambda i: self.int4.k1(P, i)),
+                    ("int4_k2", 1, lambda i: self.int4.k2(P, i))]
         seg += [("qkv%d" % m, 2, (lambda i, c=c: c.layer(P, i))) for m, c in self.qkv.items()]
         seg += [("qkv%d_k1" % m, 1, (lambda i, c=c: c.k1(P, i))) for m, c in self.qkv.items()]
         seg += [("qkv%d_k2" % m, 1, (lambda i, c=c: c.k2(P, i))) for m, c in self.qkv.items()]
@@ -573,6 +613,16 @@ def run_ours(args, world, rank, local):
         return row
 
     configs = {"qkv_sweep": [qkv_row(m) for m in wl.qkv]}
+    if "int4_layer" in seg_ms:
+        configs["int4_attention"] = {
+            "M": M, "K": Kd, "N": N, "layer_us": us("int4_layer"),
+            "layer_tflops": fl / (us("int4_layer") * 1e-6) / 1e12,
+            "quant_act_us": us("int4_k1"), "gemm_us": us("int4_k2"),
+            "gemm_tops": fl / (us("int4_k2") * 1e-6) / 1e12,
+            "gemm_frac_fp8_peak": fl / (us("int4_k2") * 1e-6) / 1e12 / (2.0 * peaks["bf16_tflops"]),
+            "vs_nvfp4_layer": us("attn_layer") / us("int4_layer"),
+            "note": "the int4 / group-64 row: codes carried as E4M3 bytes through the fp8 MMA, per-group scales "
+                    "in the epilogue; frac against the measured-derived dense fp8 peak (2 x bf16)"}
     fused = {}
     for m in QKV_FUSED_MS:
         if "qkv%d_fused" % m not in seg_ms:

@@ -23,6 +23,10 @@ from .ops import (  # noqa: F401
     svdq_w4a4_nvfp4_linear_qkv,
     svdq_w4a4_nvfp4_linear_gelu_quant,
     svdq_gelu_quant_workspace_bytes,
+    svdq_gelu_table_fill,
+    svdq_int4_pack_weights,
+    svdq_int4_quantize_act_lowrank_down,
+    svdq_w4a4_int4_linear,
     awq_w4a16_linear,
     svdq_act_amax,
     svdq_act_amax_noalloc,

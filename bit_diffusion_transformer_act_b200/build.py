@@ -13,7 +13,7 @@ LIB_DIR = os.path.join(HERE, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libsvdq.so")
 SOURCES = ["libsvdq.cu", "host_pack.cpp"]
 DEPS = SOURCES + ["ptx.cuh", "quant_act.cuh", "gemm_nvfp4.cuh", "awq_w4a16.cuh", "awq_umma.cuh", "act_amax.cuh", "layout.h",
-                  "nvfp4_quant.cuh", "gemm_gelu_quant.cuh",
+                  "nvfp4_quant.cuh", "gemm_gelu_quant.cuh", "gemm_int4.cuh",
                   os.path.join("..", "..", "include", "svdq.h")]
 
 NVCC_FLAGS = [

@@ -19,8 +19,8 @@
 //   warp 1     tensor memory, block-scaled and low-rank MMAs of the up projection (leader).
 //   warps 2-9  epilogue: a warp owns 32 rows (its tensor-memory lane quarter) and two of the
 //              tile's four 32-column chunks.  Per element y = alpha acc + b, rounded to bf16;
-//              h = bf16(GELU(y)) in fp32 pairs (erfc by a published Chebyshev fit, below); h is
-//              written into a 128 x 64 shared-memory
+//              h = bf16(GELU(y)) is one gather from a 64K-entry table of bf16(GELU(x)) for
+//              every bf16 x (filled in double precision); h is written into a 128 x 64 shared-memory
 //              slab (the A operand of the low-rank MMA, 128-byte swizzle) and quantized in
 //              registers with the down projection's smoothing and scale (the quantizer of
 //              kernel 1: codes and scale bytes stored straight to global memory).
@@ -98,6 +98,7 @@ struct Params {
   uint8_t* scales;                 // swizzled [ceil(M/128) * 128, N/16] out
   float* ws;                       // partial U: [npairs][slots][256][32]
   __nv_bfloat16* h_out;            // [M, N] or null: the hidden state, for inspection
+  const uint16_t* gelu;            // [65536]: bf16(GELU(x)) for every bf16 pattern x
   int M, N, K;
   int tiles_n, tiles;
   int slots;
@@ -116,49 +117,29 @@ __device__ __forceinline__ uint32_t idesc_u() {
          (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
+// bf16 nearest (ties to even) to a double, rounded once: 8 significant bits, the exponent range
+// of fp32 (subnormal steps of 2^-133); overflow gives infinity.
+__device__ __forceinline__ uint16_t bf16_rne_from_double(double v) {
+  if (isnan(v)) return 0x7FC0;
+  const uint16_t sign = signbit(v) ? 0x8000 : 0;
+  const double a = fabs(v);
+  if (a == 0.0) return sign;
+  if (isinf(a)) return sign | 0x7F80;
+  int e;
+  (void)frexp(a, &e);                              // a in [2^(e-1), 2^e)
+  const int step = max(e - 8, -133);               // weight of the last kept bit
+  const double r = ldexp(rint(ldexp(a, -step)), step);   // rint: to nearest, ties to even
+  return sign | static_cast<uint16_t>(__float_as_uint(static_cast<float>(r)) >> 16);   // exact (or inf)
 }
 
-// GELU(x) = x Phi(x) = x erfc(-x / sqrt 2) / 2 for two values at once.  erfc is the Chebyshev
-// fit of Numerical Recipes (Press, Teukolsky, Vetterling, Flannery, 2nd ed., section 6.2,
-// "erfcc"): for z >= 0, erfc(z) = t exp(-z^2 + P(t)) with t = 1 / (1 + z/2) and a degree-9
-// polynomial P, fractional error below 1.2e-7 everywhere; erfc(-z) = 2 - erfc(z).  Branch-free,
-// Horner's rule on packed fp32 pairs, the reciprocal and the exponential on the SFU (a few ulp).
-// Relative error against x Phi(x) (float32 evaluation of this sequence): below 2.2e-6 for
-// |x| <= 4 and 2.1e-5 anywhere (the fp32 rounding of the exponent -z^2 + P grows with z^2) --
-// far below half a bf16 ulp (2^-9), so the bf16 rounding that follows differs from that of the
-// exact value only next to a midpoint, by one ulp.
-// Large negative x give -0 (as x Phi(x) rounds), large positive x give x.
-__device__ __forceinline__ uint64_t gelu2(uint64_t x2) {
-  const uint64_t nz = f32x2_mul(x2, f32x2_pack(0.70710678118654752f, 0.70710678118654752f));   // -z
-  float z0, z1;
-  f32x2_unpack(nz, z0, z1);
-  z0 = -z0;
-  z1 = -z1;
-  const float a0 = fabsf(z0), a1 = fabsf(z1);
-  const uint64_t t = f32x2_pack(rcp_approx(fmaf(0.5f, a0, 1.0f)), rcp_approx(fmaf(0.5f, a1, 1.0f)));
-  auto c2 = [](float c) { return f32x2_pack(c, c); };
-  uint64_t q = c2(0.17087277f);
-  q = f32x2_fma(q, t, c2(-0.82215223f));
-  q = f32x2_fma(q, t, c2(1.48851587f));
-  q = f32x2_fma(q, t, c2(-1.13520398f));
-  q = f32x2_fma(q, t, c2(0.27886807f));
-  q = f32x2_fma(q, t, c2(-0.18628806f));
-  q = f32x2_fma(q, t, c2(0.09678418f));
-  q = f32x2_fma(q, t, c2(0.37409196f));
-  q = f32x2_fma(q, t, c2(1.00002368f));
-  q = f32x2_fma(q, t, c2(-1.26551223f));
-  // exponent -z^2 + P(t), in base 2
-  const uint64_t e = f32x2_mul(f32x2_fma(nz, f32x2_pack(z0, z1), q), c2(1.44269504088896341f));
-  float e0, e1, t0, t1;
-  f32x2_unpack(e, e0, e1);
-  f32x2_unpack(t, t0, t1);
-  const float r0 = t0 * ex2_approx(e0), r1 = t1 * ex2_approx(e1);
-  const float c0 = z0 < 0.f ? 2.0f - r0 : r0, c1 = z1 < 0.f ? 2.0f - r1 : r1;   // erfc(z)
-  return f32x2_mul(f32x2_mul(x2, c2(0.5f)), f32x2_pack(c0, c1));
+// The GELU table: entry i (a bf16 bit pattern x) holds bf16(x Phi(x)), Phi(x) = erfc(-x / sqrt 2) / 2
+// evaluated in double precision and rounded once.  h = bf16(GELU(y)) with y already rounded to
+// bf16 is then one gather.
+__global__ void __launch_bounds__(256) gelu_table_kernel(uint16_t* __restrict__ table) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 65536) return;
+  const double x = static_cast<double>(__uint_as_float(static_cast<uint32_t>(i) << 16));
+  table[i] = bf16_rne_from_double(0.5 * x * erfc(-x / sqrt(2.0)));
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -450,14 +431,15 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       if (lane == 0) mbar_arrive_remote(map_to_cta(acc_empty(b), 0));
       const bool block_live = mblk < p.M;          // the scale buffer holds this 128-row block
       bool ok = true;
+      // First both chunks' h (table gathers) and their hand-over to the low-rank MMA, then the
+      // quantization and the global stores: the slab's cluster-scope release arrival orders
+      // every earlier write of the thread, and global stores still in flight would hold it up.
+      uint32_t hw[2][16];
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         const int c = eh + 2 * jj;                 // chunk of the tile, in slab jj
-        const int sn = 2 * i + jj;
-        const int buf = sn & 1;
-        // y, then h = bf16(GELU(bf16(y))), as bf16 pairs
-        uint32_t hw[16];
         const uint4* bias4 = reinterpret_cast<const uint4*>(svec + c * 64);
+        uint32_t yb[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint4 bv = bias4[q];
@@ -468,33 +450,49 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const uint64_t y = f32x2_fma(f32x2_pack(alpha, alpha), f32x2_pack(__uint_as_float(R[jj][k]),
                                                                                __uint_as_float(R[jj][k + 1])),
                                          f32x2_pack(bf16lo_to_f32(bw[w]), bf16hi_to_f32(bw[w])));
-            float y0, y1, h0, h1;
+            float y0, y1;
             f32x2_unpack(y, y0, y1);
-            const uint32_t yb = pack_bf16x2(y0, y1);
-            f32x2_unpack(gelu2(f32x2_pack(bf16lo_to_f32(yb), bf16hi_to_f32(yb))), h0, h1);
-            hw[q * 4 + w] = pack_bf16x2(h0, h1);
+            yb[q * 4 + w] = pack_bf16x2(y0, y1);
           }
         }
+        // h = bf16(GELU(y)) for the 32 values: all gathers in flight together
+        uint32_t hl[16], hh[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          hl[k] = __ldg(p.gelu + (yb[k] & 0xFFFFu));
+          hh[k] = __ldg(p.gelu + (yb[k] >> 16));
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) hw[jj][k] = hl[k] | (hh[k] << 16);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int c = eh + 2 * jj;
+        const int sn = 2 * i + jj;
+        const int buf = sn & 1;
         // the slab must have been consumed by the low-rank MMAs two slabs back
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(slab_free(buf), ((sn >> 1) & 1) ^ 1, abort_flag, 39))) {
           ok = false;
           break;
         }
-        {
-          const uint32_t row = base + OFF_SLAB + buf * SLAB_BYTES + static_cast<uint32_t>(r) * 128;
-          const uint32_t sw = static_cast<uint32_t>(r & 7);
+        const uint32_t row = base + OFF_SLAB + buf * SLAB_BYTES + static_cast<uint32_t>(r) * 128;
+        const uint32_t sw = static_cast<uint32_t>(r & 7);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t u = static_cast<uint32_t>((c & 1) * 4 + q);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         ::"r"(row + ((u ^ sw) << 4)), "r"(hw[4 * q]), "r"(hw[4 * q + 1]), "r"(hw[4 * q + 2]),
-                           "r"(hw[4 * q + 3])
-                         : "memory");
-          }
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t u = static_cast<uint32_t>((c & 1) * 4 + q);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(row + ((u ^ sw) << 4)), "r"(hw[jj][4 * q]), "r"(hw[jj][4 * q + 1]), "r"(hw[jj][4 * q + 2]),
+                         "r"(hw[jj][4 * q + 3])
+                       : "memory");
         }
         fence_proxy_async_smem();                  // the tensor core reads the slab through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive_remote_cluster(map_to_cta(slab_ready(buf), 0));
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int c = eh + 2 * jj;
         // the down projection's activation pass on h: -h smooth_inv in pairs, two 16-groups
         const uint64_t* sm2 = reinterpret_cast<const uint64_t*>(svec + 256 + c * 128);   // -smooth_inv pairs
         uint32_t sc2 = 0;
@@ -504,7 +502,7 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           uint64_t nx[8];
 #pragma unroll
           for (int w = 0; w < 8; ++w) {
-            const uint32_t hv = hw[gq * 8 + w];
+            const uint32_t hv = hw[jj][gq * 8 + w];
             nx[w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(hv), bf16hi_to_f32(hv)), sm2[gq * 8 + w]);
           }
           sc2 |= quantize_group(nx, p.g, p.inv_g, cb[gq]) << (8 * gq);
@@ -516,7 +514,8 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           if (p.h_out) {
             uint4* hd = reinterpret_cast<uint4*>(p.h_out + static_cast<size_t>(m) * p.N + col);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) hd[q] = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+              hd[q] = make_uint4(hw[jj][4 * q], hw[jj][4 * q + 1], hw[jj][4 * q + 2], hw[jj][4 * q + 3]);
           }
         }
         if (block_live) {                          // rows past M in the last block get zero scales
@@ -525,7 +524,6 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           *reinterpret_cast<uint16_t*>(sdst) = m < p.M ? static_cast<uint16_t>(sc2) : uint16_t(0);
         }
       }
-      if (!ok) break;
       if (ends_part(t)) {
         // the pair's low-rank partial of this row block: one warp per lane quarter reads it out
         if (eh == 0) {

@@ -11,6 +11,7 @@
 // rounding midpoint is at least 2^-24 (relative) away from it, while double
 // rounding errs by 2^-53: the decisions equal those of exact arithmetic.
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <vector>
@@ -70,6 +71,22 @@ double pow2_global_scale(double amax) {
   while (g * limit < amax) g *= 2.0;
   while ((g * 0.5) * limit >= amax) g *= 0.5;
   return g;
+}
+
+// bf16 nearest (ties to even) to a double, rounded once (8 significant bits, bf16 subnormal
+// steps of 2^-133); finite inputs.
+uint16_t double_to_bf16_rne(double v) {
+  const uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+  const double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  (void)std::frexp(a, &e);
+  const int step = std::max(e - 8, -133);
+  const double r = std::ldexp(std::nearbyint(std::ldexp(a, -step)), step);
+  const float f = static_cast<float>(r);            // exact (or infinity)
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return static_cast<uint16_t>(sign | (u >> 16));
 }
 
 float bf16_to_float(uint16_t b) {
@@ -184,6 +201,67 @@ int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
   h.w_global_scale = static_cast<float>(g);
   std::memcpy(blob, &h, sizeof(h));
   *w_global_scale = static_cast<float>(g);
+  return SVDQ_OK;
+}
+
+size_t svdq_int4_packed_weight_bytes(int N, int K, int rank) {
+  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || rank != svdq::kRank) return 0;
+  return svdq::blob_layout_int4(N, K, rank).total;
+}
+
+int svdq_int4_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2, const uint16_t* bias,
+                           const uint16_t* smooth_inv, int N, int K, int rank, void* out, size_t out_bytes) {
+  if (!R || !L1 || !L2 || !smooth_inv || !out) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || rank != svdq::kRank) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  const svdq::BlobLayout L = svdq::blob_layout_int4(N, K, rank);
+  if (out_bytes < L.total) return SVDQ_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(N), k = static_cast<size_t>(K);
+  for (size_t i = 0; i < n * k; ++i)
+    if (!std::isfinite(R[i])) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  uint8_t* blob = static_cast<uint8_t*>(out);
+  std::memset(blob, 0, L.total);
+  uint8_t* codes = blob + L.codes;
+  float* scales = reinterpret_cast<float*>(blob + L.scales);       // [K/64][N]
+  // per (row, 64-group): s = RNE_bf16(amax / 7) rounded once from the double quotient (amax has
+  // at most 24 significant bits, 7 three: a quotient on a bf16 midpoint is exact in double, one
+  // off it is far more than double's error away); c = clamp(RNE(x / s), -8, 7), by the same
+  // argument decided exactly; c stored as its E4M3 byte
+  for (size_t row = 0; row < n; ++row) {
+    const float* x = R + row * k;
+    for (size_t gi = 0; gi < k / 64; ++gi) {
+      double amax = 0.0;
+      for (int t = 0; t < 64; ++t) amax = std::fmax(amax, std::fabs(static_cast<double>(x[gi * 64 + t])));
+      const uint16_t sb = double_to_bf16_rne(amax / 7.0);
+      scales[gi * n + row] = bf16_to_float(sb);
+      const double s = bf16_to_float(sb);
+      for (int t = 0; t < 64; ++t) {
+        double c = 0.0;
+        if (s != 0.0) c = std::fmin(7.0, std::fmax(-8.0, std::nearbyint(static_cast<double>(x[gi * 64 + t]) / s)));
+        const uint8_t mag = e4m3_code_rne(std::fabs(c));      // integers up to 8 are exact in E4M3
+        codes[row * k + gi * 64 + t] = static_cast<uint8_t>(mag | (c < 0.0 ? 0x80 : 0));
+      }
+    }
+  }
+  uint16_t* l1s_hi = reinterpret_cast<uint16_t*>(blob + L.l1s);
+  uint16_t* l1s_lo = l1s_hi + static_cast<size_t>(rank) * k;
+  for (size_t j = 0; j < static_cast<size_t>(rank); ++j)
+    for (size_t kk = 0; kk < k; ++kk) {
+      const float prod = bf16_to_float(smooth_inv[kk]) * bf16_to_float(L1[kk * rank + j]);
+      const uint16_t hi = float_to_bf16_rne(prod);
+      l1s_hi[j * k + kk] = hi;
+      l1s_lo[j * k + kk] = float_to_bf16_rne(prod - bf16_to_float(hi));
+    }
+  uint16_t* l2t = reinterpret_cast<uint16_t*>(blob + L.l2t);
+  for (size_t row = 0; row < n; ++row)
+    for (size_t j = 0; j < static_cast<size_t>(rank); ++j) l2t[row * rank + j] = L2[j * n + row];
+  if (bias) std::memcpy(blob + L.bias, bias, n * 2);
+  svdq::BlobHeader h;
+  std::memset(&h, 0, sizeof(h));
+  std::memcpy(h.magic, "SVDQINT4", 8);
+  h.abi_version = svdq::kAbiVersion;
+  h.N = N; h.K = K; h.rank = rank;
+  h.w_global_scale = 1.0f;
+  std::memcpy(blob, &h, sizeof(h));
   return SVDQ_OK;
 }
 

@@ -52,6 +52,26 @@ inline BlobLayout blob_layout(size_t N, size_t K, size_t rank) {
   return L;
 }
 
+// Packed weight blob of the int4 / group-64 row (svdq_int4_pack_weights): the same 1 KB header
+// ("SVDQINT4") and l1s section, then
+//   codes        u8   [N][K]      each int4 code -7..7 as its E4M3 byte (exact: the fp8 MMA
+//                                 multiplies the integers exactly)
+//   scales       f32  [K/64][N]   the per-64 bf16 scales widened to fp32 (exact), group-major:
+//                                 a tile's columns of one group are contiguous
+//   l2t          bf16 [N][rank]   L2 transposed (no per-tensor scale in this format)
+//   bias         bf16 [N]
+inline BlobLayout blob_layout_int4(size_t N, size_t K, size_t rank) {
+  BlobLayout L;
+  size_t off = kBlobAlign;
+  L.l1s = off;    off = align_up(off + 2 * rank * K * 2, kBlobAlign);
+  L.codes = off;  off = align_up(off + N * K, kBlobAlign);
+  L.scales = off; off = align_up(off + N * (K / 64) * 4, kBlobAlign);
+  L.l2t = off;    off = align_up(off + N * rank * 2, kBlobAlign);
+  L.bias = off;   off = align_up(off + N * 2, kBlobAlign);
+  L.total = off;
+  return L;
+}
+
 struct BlobHeader {
   char magic[8];        // "SVDQNVF4"
   int32_t abi_version;

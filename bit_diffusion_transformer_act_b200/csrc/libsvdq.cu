@@ -20,6 +20,7 @@
 #include "awq_w4a16.cuh"
 #include "awq_umma.cuh"
 #include "gemm_gelu_quant.cuh"
+#include "gemm_int4.cuh"
 
 // Scratch of svdq_act_amax_noalloc: kernel 5's result word, partial maximum and block
 // counter, for callers that cannot allocate device memory.  Every GPU that loads this
@@ -163,7 +164,7 @@ extern "C" {
 // amax word of kernel 5.
 static int quantize_impl(const void* X, const void* smooth_inv, const void* packed_w, int M, int K, int rank,
                          float act_global_scale, const void* act_amax, void* act_codes, void* act_scales,
-                         void* lowrank_act, void* stream) {
+                         void* lowrank_act, void* stream, bool int4 = false) {
   if (M < 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
   if (!act_amax && !is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
   if (act_amax && (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
@@ -209,7 +210,9 @@ static int quantize_impl(const void* X, const void* smooth_inv, const void* pack
                  2 * k1::kRank, K, k1::kChunk, 2 * k1::kRank, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
   const int smem = k1::kSmemBytes;
-  if (!set_smem_once<k1::quant_act_lowrank_kernel>(smem, dev)) return SVDQ_ERR_CUDA;
+  if (!set_smem_once<k1::quant_act_lowrank_kernel<false>>(smem, dev) ||
+      !set_smem_once<k1::quant_act_lowrank_kernel<true>>(smem, dev))
+    return SVDQ_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rowblocks, ks, 1);
@@ -225,7 +228,8 @@ static int quantize_impl(const void* X, const void* smooth_inv, const void* pack
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel, tX, tL, p) != cudaSuccess) {
+  if ((int4 ? cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel<true>, tX, tL, p)
+            : cudaLaunchKernelEx(&cfg, k1::quant_act_lowrank_kernel<false>, tX, tL, p)) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }
@@ -421,6 +425,16 @@ static void gelu_quant_partition(int M, int N, int dev, int* npairs, int* slots)
   *slots = sl;
 }
 
+size_t svdq_gelu_table_bytes(void) { return 65536 * sizeof(uint16_t); }
+
+int svdq_gelu_table_fill(void* table, void* stream) {
+  if (!table || !aligned16(table)) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  svdq::k6::gelu_table_kernel<<<256, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint16_t*>(table));
+  return launch_status();
+}
+
 size_t svdq_gelu_quant_workspace_bytes(int M, int N) {
   if (M <= 0 || N <= 0 || N % 128 != 0) return 0;
   int dev = 0;
@@ -437,8 +451,8 @@ int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_sca
                                       float act_global_scale, const void* packed_w, float w_global_scale, int M,
                                       int N, int K, int rank, const void* down_smooth_inv, const void* down_packed_w,
                                       float down_act_global_scale, void* out_codes, void* out_scales,
-                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes, void* h_out,
-                                      void* stream) {
+                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes,
+                                      const void* gelu_table, void* h_out, void* stream) {
   if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_scale(act_global_scale) || !is_pow2_scale(w_global_scale) || !is_pow2_scale(down_act_global_scale))
     return SVDQ_ERR_INVALID_ARG;
@@ -447,11 +461,11 @@ int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_sca
   if (!(alpha >= 0x1p-126 && alpha <= 0x1p126)) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!act_codes || !act_scales || !lowrank_act || !packed_w || !down_smooth_inv || !down_packed_w || !out_codes ||
-      !out_scales || !out_lowrank_act || !workspace)
+      !out_scales || !out_lowrank_act || !workspace || !gelu_table)
     return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
       !aligned16(down_smooth_inv) || !aligned16(down_packed_w) || !aligned16(out_codes) || !aligned16(out_scales) ||
-      !aligned16(out_lowrank_act) || !aligned16(workspace) || (h_out && !aligned16(h_out)))
+      !aligned16(out_lowrank_act) || !aligned16(workspace) || !aligned16(gelu_table) || (h_out && !aligned16(h_out)))
     return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
@@ -470,6 +484,7 @@ int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_sca
   p.scales = static_cast<uint8_t*>(out_scales);
   p.ws = static_cast<float*>(workspace);
   p.h_out = static_cast<__nv_bfloat16*>(h_out);
+  p.gelu = static_cast<const uint16_t*>(gelu_table);
   p.M = M;
   p.N = N;
   p.K = K;
@@ -523,6 +538,63 @@ int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_sca
   cfg2.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg2, k6::u_reduce_kernel, static_cast<const float*>(workspace), M, p.tiles_n, p.tiles, P,
                          slots, p.inv_g, static_cast<__nv_bfloat16*>(out_lowrank_act)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+int svdq_int4_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                        int rank, void* act_codes, void* act_scales, void* lowrank_act, void* stream) {
+  return quantize_impl(X, smooth_inv, packed_w, M, K, rank, 1.0f, nullptr, act_codes, act_scales, lowrank_act, stream,
+                       true);
+}
+
+int svdq_w4a4_int4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act, const void* packed_w,
+                          int M, int N, int K, int rank, void* Y, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || rank <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
+      !aligned16(Y))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if (int st = current_device_ok(&dev)) return st;
+  namespace k8 = svdq::k8;
+  const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
+  const svdq::BlobLayout L = svdq::blob_layout_int4(N, K, rank);
+  k8::Params p;
+  p.a_scales = static_cast<const uint16_t*>(act_scales);
+  p.w_scales = reinterpret_cast<const float*>(blob + L.scales);
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_n = N / k8::BN;
+  p.tiles = ((M + k8::BM - 1) / k8::BM) * p.tiles_n;
+  CUtensorMap tA, tB, tU, tL2, tY;
+  if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, k8::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, 128, k8::BN,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tU, lowrank_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, 2 * rank, 2 * rank, k8::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, k8::BN,
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_tmap(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ERR_CUDA;
+  if (!set_smem_once<k8::int4_gemm_kernel>(k8::SMEM_BYTES, dev)) return SVDQ_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(p.tiles, sm_count(dev)), 1, 1);
+  cfg.blockDim = dim3(k8::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = k8::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k8::int4_gemm_kernel, tA, tB, tU, tL2, tY, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }

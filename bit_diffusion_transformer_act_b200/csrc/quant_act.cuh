@@ -100,6 +100,60 @@ __device__ __forceinline__ uint32_t idesc_lowrank() {
          (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
+// The int4 / group-64 row's quantizer of one 64-column group held by two neighbouring lanes (32
+// columns each, as 16 pairs of -x_hat): both lanes form the group's amax (one exchange), the
+// bf16 scale s = RNE_bf16(amax / 7) rounded once from the exact quotient, and this lane's 32
+// codes RNE(x_hat / s) as E4M3 bytes (the integers -7..7 are exact in E4M3; with s rounded to
+// nearest, |x_hat / s| <= 7 (1 + 2^-8) < 7.5, so no code needs clamping).  Returns s's bits.
+// amax / 7 is the correctly rounded fp32 quotient; when that lands exactly on a bf16 midpoint
+// the exact quotient decides the side (7 times the midpoint, 12 significant bits, is exact).
+// x_hat / s: the corrected quotient as in the nvfp4 quantizer (x_hat has at most 16 significant
+// bits and s 8, so an exact half-integer quotient is computed exactly and any other is at least
+// 2^-16 away from one).  Scales below 2^-126 (amax < 7 * 2^-126) are not supported.
+__device__ __forceinline__ uint16_t quantize_int4_group(const uint64_t (&nx)[16], uint4 (&out)[2]) {
+  float a[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f32x2_unpack(nx[i], a[2 * i], a[2 * i + 1]);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) amax = fmax3(amax, fabsf(a[i]), fabsf(a[i + 1]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  const float q = __fdiv_rn(amax, 7.0f);
+  const uint32_t qb = __float_as_uint(q);
+  uint32_t sb;
+  if ((qb & 0xFFFFu) == 0x8000u) {
+    const float t = 7.0f * q;                      // exact
+    sb = amax > t ? (qb >> 16) + 1u : (amax < t ? (qb >> 16) : (pack_bf16x2(q, 0.f) & 0xFFFFu));
+  } else {
+    sb = pack_bf16x2(q, 0.f) & 0xFFFFu;            // round to nearest even
+  }
+  const float s = __uint_as_float(sb << 16);
+  if (s == 0.f) {
+    out[0] = out[1] = make_uint4(0u, 0u, 0u, 0u);
+    return 0;
+  }
+  const float rn = -rcp_approx(s);                 // -1/s: the pairs hold -x_hat
+  const uint64_t rn2 = f32x2_pack(rn, rn), s2 = f32x2_pack(s, s);
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint64_t q0 = f32x2_mul(nx[i + j], rn2);          // x_hat / s, first guess
+      const uint64_t e = f32x2_fma(q0, s2, nx[i + j]);        // q0 s - x_hat, exact
+      f32x2_unpack(f32x2_fma(e, rn2, q0), v[2 * j], v[2 * j + 1]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = rintf(v[j]);          // to nearest integer, ties to even
+    w[i / 2] = cvt_e4m3x2(v[0], v[1]) | (cvt_e4m3x2(v[2], v[3]) << 16);
+  }
+  out[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  out[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  return static_cast<uint16_t>(sb);
+}
+
+template <bool kInt4 = false>
 __global__ void __launch_bounds__(kThreads, 2)
 quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL,
                          const Params p) {
@@ -199,7 +253,40 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
     // scale bytes 2h, 2h + 1 of this row's word in the chunk's 512-byte atom
     uint8_t* scale_base = p.scales + static_cast<size_t>(m0 / 128) * (p.K / 64) * 512 + (r % 32) * 16 +
                           (r / 32) * 4 + 2 * h;
-    for (int c = 0; c < nck; ++c) {
+    for (int c = 0; kInt4 && c < nck; ++c) {
+      // int4 / group 64: the chunk is one group, shared by this lane and its neighbour
+      const int s = c % kStages;
+      const uint32_t ph = (c / kStages) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 13))) break;
+      const uint32_t row = base + s * kStageBytes + r * 128;
+      const float* sm = smooth + c * kChunk + h * 32;
+      uint64_t nx[16];
+#pragma unroll
+      for (int uu = 0; uu < 4; ++uu) {
+        const uint32_t u = static_cast<uint32_t>(h * 4 + uu);
+        uint32_t xw[4];
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(xw[0]), "=r"(xw[1]), "=r"(xw[2]), "=r"(xw[3]) : "r"(row + ((u ^ sw) << 4)));
+        const ulonglong2 s01 = *reinterpret_cast<const ulonglong2*>(sm + uu * 8);
+        const ulonglong2 s23 = *reinterpret_cast<const ulonglong2*>(sm + uu * 8 + 4);
+        const uint64_t sp[4] = {s01.x, s01.y, s23.x, s23.y};
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          nx[uu * 4 + w] = f32x2_mul(f32x2_pack(bf16lo_to_f32(xw[w]), bf16hi_to_f32(xw[w])), sp[w]);
+      }
+      uint4 cw[2];
+      const uint16_t sb = quantize_int4_group(nx, cw);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed(empty(s));
+      if (m < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kbeg + c * kChunk + h * 32);
+        dst[0] = cw[0];
+        dst[1] = cw[1];
+        if (h == 0)                                // group-major [K/64][M]
+          reinterpret_cast<uint16_t*>(p.scales)[static_cast<size_t>((kbeg / 64) + c) * p.M + m] = sb;
+      }
+    }
+    for (int c = 0; !kInt4 && c < nck; ++c) {
       const int s = c % kStages;
       const uint32_t ph = (c / kStages) & 1u;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), ph, abort_flag, 13))) break;

@@ -41,8 +41,14 @@ def _load():
         "svdq_w4a4_nvfp4_linear": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp], i),
         "svdq_w4a4_nvfp4_linear_qkv": ([vp, vp, vp, f, vp, f, i, i, i, i, i, i, vp, vp, f, vp, vp, vp, vp], i),
         "svdq_gelu_quant_workspace_bytes": ([i, i], sz),
-        "svdq_w4a4_nvfp4_linear_gelu_quant": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp, f, vp, vp, vp, vp, sz, vp, vp],
-                                              i),
+        "svdq_gelu_table_bytes": ([], sz),
+        "svdq_int4_packed_weight_bytes": ([i, i, i], sz),
+        "svdq_int4_pack_weights": ([vp, vp, vp, vp, vp, i, i, i, vp, sz], i),
+        "svdq_int4_quantize_act_lowrank_down": ([vp, vp, vp, i, i, i, vp, vp, vp, vp], i),
+        "svdq_w4a4_int4_linear": ([vp, vp, vp, vp, i, i, i, i, vp, vp], i),
+        "svdq_gelu_table_fill": ([vp, vp], i),
+        "svdq_w4a4_nvfp4_linear_gelu_quant": ([vp, vp, vp, f, vp, f, i, i, i, i, vp, vp, f, vp, vp, vp, vp, sz, vp, vp,
+                                               vp], i),
         "awq_w4a16_linear": ([vp, vp, vp, vp, vp, i, i, i, vp, vp], i),
         "svdq_act_amax": ([vp, vp, i, i, vp, vp], i),
         "svdq_act_amax_noalloc": ([vp, vp, i, i, vp, vp], i),
@@ -66,7 +72,9 @@ EXPORTED = ("svdq_status_string", "svdq_abi_version", "svdq_packed_weight_bytes"
             "awq_w4a16_linear", "svdq_unswizzle_scales", "svdq_swizzle_scales", "svdq_device_status",
             "svdq_act_amax", "svdq_quantize_act_lowrank_down_dyn", "svdq_w4a4_nvfp4_linear_dyn",
             "svdq_act_amax_noalloc", "svdq_w4a4_nvfp4_linear_qkv", "svdq_gelu_quant_workspace_bytes",
-            "svdq_w4a4_nvfp4_linear_gelu_quant", "svdq_selftest_wait_timeout")
+            "svdq_w4a4_nvfp4_linear_gelu_quant", "svdq_selftest_wait_timeout", "svdq_gelu_table_bytes",
+            "svdq_gelu_table_fill", "svdq_int4_packed_weight_bytes", "svdq_int4_pack_weights",
+            "svdq_int4_quantize_act_lowrank_down", "svdq_w4a4_int4_linear")
 
 
 def _check(fn, st):
@@ -156,6 +164,33 @@ def svdq_pack_weights(R, L1_bits, L2_bits, bias_bits, smooth_bits):
                                _np_ptr(smooth_bits), N, K, rank, _np_ptr(out), nbytes, ctypes.byref(g))
     _check("svdq_pack_weights", st)
     return out, float(g.value)
+
+
+def svdq_int4_pack_weights(R, L1_bits, L2_bits, bias_bits, smooth_bits):
+    """The int4 / group-64 row's packed weights (numpy uint8 blob) of R float32 [N, K], L1 bits
+    [K, r], L2 bits [r, N], bias bits [N] or None, smooth_inv bits [K]."""
+    R = np.ascontiguousarray(R, dtype=np.float32)
+    N, K = R.shape
+    L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    rank = L1_bits.shape[1]
+    if L1_bits.shape != (K, rank) or L2_bits.shape != (rank, N):
+        raise ValueError("L1 must be [K, r] and L2 [r, N]")
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        if bias_bits.shape != (N,):
+            raise ValueError("bias must be [N]")
+    smooth_bits = np.ascontiguousarray(smooth_bits, dtype=np.uint16)
+    if smooth_bits.shape != (K,):
+        raise ValueError("smooth_inv must be [K]")
+    nbytes = int(LIB.svdq_int4_packed_weight_bytes(N, K, rank))
+    if nbytes == 0:
+        _check("svdq_int4_pack_weights", 2)
+    out = np.empty(nbytes, dtype=np.uint8)
+    _check("svdq_int4_pack_weights", LIB.svdq_int4_pack_weights(_np_ptr(R), _np_ptr(L1_bits), _np_ptr(L2_bits),
+                                                                 _np_ptr(bias_bits), _np_ptr(smooth_bits), N, K,
+                                                                 rank, _np_ptr(out), nbytes))
+    return out
 
 
 def svdq_unswizzle_scales(swizzled, rows, K):
@@ -255,10 +290,31 @@ def svdq_gelu_quant_workspace_bytes(M, N):
     return int(LIB.svdq_gelu_quant_workspace_bytes(M, N))
 
 
+def svdq_gelu_table_fill(table=None, device=None):
+    """The GELU table (uint8 [svdq_gelu_table_bytes()] CUDA tensor) filled by the library."""
+    if table is None:
+        table = torch.empty((int(LIB.svdq_gelu_table_bytes()),), dtype=torch.uint8,
+                            device=device if device is not None else torch.device("cuda", torch.cuda.current_device()))
+    _require_blob(table, "gelu_table", int(LIB.svdq_gelu_table_bytes()))
+    _check("svdq_gelu_table_fill", LIB.svdq_gelu_table_fill(_ptr(table), _stream()))
+    return table
+
+
+_GELU_TABLES = {}
+
+
+def _gelu_table(device):
+    """A filled GELU table per device, made on first use (on the current stream)."""
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _GELU_TABLES:
+        _GELU_TABLES[key] = svdq_gelu_table_fill(device=torch.device("cuda", key))
+    return _GELU_TABLES[key]
+
+
 def svdq_w4a4_nvfp4_linear_gelu_quant(act_codes, act_scales, lowrank_act, act_global_scale, packed_w, w_global_scale,
                                       M, N, K, down_smooth_inv, down_packed_w, down_act_global_scale, rank=RANK,
                                       out_codes=None, out_scales=None, out_lowrank_act=None, workspace=None,
-                                      h_out=None):
+                                      h_out=None, gelu_table=None):
     """The MLP up projection with GELU and the down projection's activation pass fused: returns the
     down projection's (act_codes uint8 [M, N/2], act_scales, lowrank_act bf16 [M, 2r]) for its
     smooth_inv (bf16 [N]), packed weights (its low-rank section is used) and g_a.  h_out (bf16
@@ -283,6 +339,9 @@ def svdq_w4a4_nvfp4_linear_gelu_quant(act_codes, act_scales, lowrank_act, act_gl
     _require(out_scales, torch.uint8, (svdq_act_scale_bytes(M, N),), "out_scales")
     _require(out_lowrank_act, torch.bfloat16, (M, 2 * rank), "out_lowrank_act")
     _require_blob(workspace, "workspace", ws_bytes)
+    if gelu_table is None:
+        gelu_table = _gelu_table(dev)
+    _require_blob(gelu_table, "gelu_table", int(LIB.svdq_gelu_table_bytes()))
     if h_out is not None:
         _require(h_out, torch.bfloat16, (M, N), "h_out")
     st = LIB.svdq_w4a4_nvfp4_linear_gelu_quant(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act),
@@ -290,9 +349,48 @@ def svdq_w4a4_nvfp4_linear_gelu_quant(act_codes, act_scales, lowrank_act, act_gl
                                                M, N, K, rank, _ptr(down_smooth_inv), _ptr(down_packed_w),
                                                float(down_act_global_scale), _ptr(out_codes), _ptr(out_scales),
                                                _ptr(out_lowrank_act), _ptr(workspace), workspace.numel(),
-                                               _ptr(h_out), _stream())
+                                               _ptr(gelu_table), _ptr(h_out), _stream())
     _check("svdq_w4a4_nvfp4_linear_gelu_quant", st)
     return out_codes, out_scales, out_lowrank_act
+
+
+def svdq_int4_quantize_act_lowrank_down(X, smooth_inv, packed_w, rank=RANK, act_codes=None, act_scales=None,
+                                        lowrank_act=None):
+    """The int4 row's activation pass: (act_codes uint8 [M, K] (E4M3 bytes of the int4 codes),
+    act_scales bf16 [K/64, M] (group-major), lowrank_act bf16 [M, 2r] (U as hi then lo))."""
+    M, K = X.shape
+    dev = X.device
+    _require_blob(packed_w, "packed_w", _l1_section_end(K, rank))
+    _require(X, torch.bfloat16, (M, K), "X")
+    _require(smooth_inv, torch.bfloat16, (K,), "smooth_inv")
+    if act_codes is None:
+        act_codes = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    if act_scales is None:
+        act_scales = torch.empty((K // 64, M), dtype=torch.bfloat16, device=dev)
+    if lowrank_act is None:
+        lowrank_act = torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev)
+    _require(act_codes, torch.uint8, (M, K), "act_codes")
+    _require(act_scales, torch.bfloat16, (K // 64, M), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    st = LIB.svdq_int4_quantize_act_lowrank_down(_ptr(X), _ptr(smooth_inv), _ptr(packed_w), M, K, rank,
+                                                 _ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act), _stream())
+    _check("svdq_int4_quantize_act_lowrank_down", st)
+    return act_codes, act_scales, lowrank_act
+
+
+def svdq_w4a4_int4_linear(act_codes, act_scales, lowrank_act, packed_w, M, N, K, rank=RANK, Y=None):
+    """Y bf16 [M, N] of the int4 / group-64 row."""
+    _require(act_codes, torch.uint8, (M, K), "act_codes")
+    _require(act_scales, torch.bfloat16, (K // 64, M), "act_scales")
+    _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
+    _require_blob(packed_w, "packed_w", int(LIB.svdq_int4_packed_weight_bytes(N, K, rank)))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    st = LIB.svdq_w4a4_int4_linear(_ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act), _ptr(packed_w), M, N, K,
+                                   rank, _ptr(Y), _stream())
+    _check("svdq_w4a4_int4_linear", st)
+    return Y
 
 
 def svdq_act_amax(X, smooth_inv, act_amax=None):

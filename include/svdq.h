@@ -182,15 +182,15 @@ int svdq_w4a4_nvfp4_linear_qkv(const void* act_codes, const void* act_scales, co
  * pages name the fusion only; the reading used is that it computes what the unfused pipeline
  * computes, without the hidden state ever reaching memory:
  *   y = bf16(g_a g_w (Q(X_hat) Q(R)^T) + lowrank_act L2 + b)        (svdq_w4a4_nvfp4_linear)
- *   h = bf16(GELU(y)),  GELU(x) = x Phi(x) (erf form, evaluated in fp32)
+ *   h = bf16(GELU(y)),  GELU(x) = x Phi(x) (erf form)
  *   out_codes, out_scales, out_lowrank_act = svdq_quantize_act_lowrank_down(h, down_smooth_inv,
  *       down_packed_w, down_act_global_scale)   (the down projection's activation pass on h)
  * The low-rank product U = h_hat L1 of the down projection needs every column of a row; the GEMM
  * keeps it in tensor memory over each CTA pair's consecutive output tiles of a row block and
  * writes one fp32 partial per (pair, row block) to `workspace`; kernel 7 sums them in a fixed
  * order (repeat calls are bit-identical).  Against the unfused pipeline the result can differ
- * only where fp32 GELU lands on the other side of a bf16 rounding midpoint than the exact value
- * (h one bf16 ulp apart); codes and scales are exact for the h this call forms.
+ * only through the fp32 rounding of y before GELU (and of an fp32 GELU, if the unfused pipeline
+ * used one); codes and scales are exact for the h this call forms.
  *   act_codes, act_scales, lowrank_act, packed_w, g's: as svdq_w4a4_nvfp4_linear (N = the MLP
  *     width, the down projection's K)
  *   down_smooth_inv   device bf16 [N]; down_packed_w the down projection's packed blob (only its
@@ -199,15 +199,55 @@ int svdq_w4a4_nvfp4_linear_qkv(const void* act_codes, const void* act_scales, co
  *   out_codes   u8 [M, N/2]; out_scales u8 [svdq_act_scale_bytes(M, N)]; out_lowrank_act bf16 [M, 2 rank]
  *   workspace   device scratch of at least svdq_gelu_quant_workspace_bytes(M, N) bytes
  *     (the caller allocates it; contents need no initialisation and are overwritten)
+ *   gelu_table  device buffer of svdq_gelu_table_bytes() bytes filled by svdq_gelu_table_fill
+ *     (once; read only here): GELU of a bf16 y rounded to bf16 is one lookup, and h is then the
+ *     double-precision GELU rounded once -- the unfused pipeline's value except where its fp32
+ *     GELU would round the other way at a bf16 midpoint
  *   h_out       device bf16 [M, N] or NULL: if given, also receives h (for inspection)
  * N % 128 == 0, K % 64 == 0, rank == 32; 16-byte aligned pointers.  Asynchronous on `stream`. */
 size_t svdq_gelu_quant_workspace_bytes(int M, int N);   /* for the current device; 0 if invalid */
+size_t svdq_gelu_table_bytes(void);                      /* 131072: 65536 bf16 entries */
+/* Fills `table` (device, 16-byte aligned, svdq_gelu_table_bytes()) with bf16(x Phi(x)) for every
+ * bf16 bit pattern x, Phi(x) = erfc(-x / sqrt 2) / 2 in double precision, rounded once to
+ * nearest even.  Asynchronous on `stream`. */
+int svdq_gelu_table_fill(void* table, void* stream);
 int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_scales, const void* lowrank_act,
                                       float act_global_scale, const void* packed_w, float w_global_scale, int M,
                                       int N, int K, int rank, const void* down_smooth_inv, const void* down_packed_w,
                                       float down_act_global_scale, void* out_codes, void* out_scales,
-                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes, void* h_out,
-                                      void* stream);
+                                      void* out_lowrank_act, void* workspace, size_t workspace_bytes,
+                                      const void* gelu_table, void* h_out, void* stream);
+
+/* ------------------------------------------------- SVDQ W4A4, int4 / group 64 */
+
+/* The svdq_w4a4 row with int4 precision and group size 64 ("Nunchaku Lite" docs, "Supported
+ * quantization types"; the docs add that nvfp4 is the faster of the two on Blackwell).  The
+ * pages give no formula; the reading: symmetric signed 4-bit codes, one bf16 scale per 64 K
+ * elements of every row of both operands, s = RNE_bf16(amax / 7) rounded once from the exact
+ * quotient, codes RNE(x / s) (within -7..7, the 8-bit scale rounding to nearest), the same
+ * smoothing and rank-32 low-rank branch as the nvfp4 row, no per-tensor scale:
+ *     y = sum_g s_a[m, g] s_w[n, g] sum_{k in g} c_a[m, k] c_w[n, k] + (X_hat L1) L2 + b.
+ * The tensor cores have no 4-bit integer MMA: a code travels as its E4M3 byte (every integer
+ * -8..8 is exact in E4M3) and the fp8 MMA (fp32 accumulation) multiplies the integers
+ * exactly; each group's sum gets its own accumulator and the epilogue applies s_a s_w.
+ *
+ * svdq_int4_pack_weights: R, L1, L2, bias, smooth_inv as svdq_pack_weights (N % 128 == 0,
+ *   K % 64 == 0, rank 32); blob of svdq_int4_packed_weight_bytes: 1 KB header ("SVDQINT4"),
+ *   the low-rank factor section as svdq_pack_weights, codes u8 [N, K] (E4M3 bytes), the scales
+ *   widened to fp32 and group-major [K/64, N], L2^T bf16 [N, rank], bias bf16 [N].
+ * svdq_int4_quantize_act_lowrank_down: kernel 1's pass with this quantizer -- act_codes u8
+ *   [M, K] (E4M3 bytes), act_scales bf16 [K/64, M] (group-major), lowrank_act bf16 [M, 2 rank]
+ *   (U as hi then lo).  X, smooth_inv, packed_w (its low-rank section) as the nvfp4 call.
+ *   Activation scales below 2^-126 (a group amax below 7 * 2^-126) are not supported.
+ * svdq_w4a4_int4_linear: Y bf16 [M, N] from those and the packed weights.
+ * Errors and asynchrony as the nvfp4 calls. */
+size_t svdq_int4_packed_weight_bytes(int N, int K, int rank);
+int svdq_int4_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2, const uint16_t* bias,
+                           const uint16_t* smooth_inv, int N, int K, int rank, void* out, size_t out_bytes);
+int svdq_int4_quantize_act_lowrank_down(const void* X, const void* smooth_inv, const void* packed_w, int M, int K,
+                                        int rank, void* act_codes, void* act_scales, void* lowrank_act, void* stream);
+int svdq_w4a4_int4_linear(const void* act_codes, const void* act_scales, const void* lowrank_act, const void* packed_w,
+                          int M, int N, int K, int rank, void* Y, void* stream);
 
 /* -------------------------------------------- dynamic per-tensor activation scale */
 

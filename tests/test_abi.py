@@ -108,17 +108,35 @@ def test_qkv_entry_point_rejects_bad_arguments_before_any_device_work():
 def test_gelu_quant_entry_point_rejects_bad_arguments_before_any_device_work():
     L = P.LIB
 
-    def call(M=4, N=256, K=64, g=1.0, gd=1.0, ws=FAKE, wsb=1 << 30, h=None, codes=FAKE):
+    def call(M=4, N=256, K=64, g=1.0, gd=1.0, ws=FAKE, wsb=1 << 30, h=None, codes=FAKE, table=FAKE):
         return L.svdq_w4a4_nvfp4_linear_gelu_quant(FAKE, FAKE, FAKE, g, FAKE, 1.0, M, N, K, 32, FAKE, FAKE, gd,
-                                                   codes, FAKE, FAKE, ws, wsb, h, None)
+                                                   codes, FAKE, FAKE, ws, wsb, table, h, None)
     assert call(N=192) == 2                             # N % 128
     assert call(K=96) == 2
     assert call(g=0.3) == 1 and call(gd=3.0) == 1       # scales must be powers of two
-    assert call(ws=None) == 1 and call(codes=None) == 1
+    assert call(ws=None) == 1 and call(codes=None) == 1 and call(table=None) == 1
+    assert call(table=ctypes.c_void_p((1 << 20) + 2)) == 1
     assert call(h=ctypes.c_void_p((1 << 20) + 8)) == 1  # misaligned optional output
     assert call(M=-1) == 1
     assert call(M=0, ws=None, codes=None) == 0          # empty batch: nothing needed
     assert P.svdq_gelu_quant_workspace_bytes(4, 200) == 0
+    assert P.LIB.svdq_gelu_table_bytes() == 131072
+    assert L.svdq_gelu_table_fill(None, None) == 1
+
+
+def test_int4_entry_points_reject_bad_arguments_before_any_device_work():
+    L = P.LIB
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.svdq_int4_packed_weight_bytes(128, 64, 32) > 0
+    assert L.svdq_int4_packed_weight_bytes(100, 64, 32) == 0 and L.svdq_int4_packed_weight_bytes(128, 96, 32) == 0
+    assert L.svdq_int4_quantize_act_lowrank_down(None, FAKE, FAKE, 4, 64, 32, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_int4_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 96, 32, FAKE, FAKE, FAKE, None) == 2
+    assert L.svdq_int4_quantize_act_lowrank_down(odd, FAKE, FAKE, 4, 64, 32, FAKE, FAKE, FAKE, None) == 1
+    assert L.svdq_w4a4_int4_linear(FAKE, FAKE, FAKE, FAKE, 4, 192, 64, 32, FAKE, None) == 2
+    assert L.svdq_w4a4_int4_linear(FAKE, FAKE, FAKE, FAKE, 4, 128, 64, 16, FAKE, None) == 2
+    assert L.svdq_w4a4_int4_linear(FAKE, None, FAKE, FAKE, 4, 128, 64, 32, FAKE, None) == 1
+    assert L.svdq_w4a4_int4_linear(FAKE, FAKE, FAKE, FAKE, 4, 128, 64, 32, odd, None) == 1
+    assert L.svdq_w4a4_int4_linear(None, None, None, None, 0, 128, 64, 32, None, None) == 0
 
 
 def test_dynamic_scale_entry_points_reject_bad_arguments_before_any_device_work():

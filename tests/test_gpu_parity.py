@@ -238,6 +238,20 @@ def test_qkv_rmsnorm_rope_epilogue(P, name, M, K, heads):
 
 # ---------------------------------------------------------------- fused MLP up projection (GELU + re-quantization)
 
+def test_gelu_table_is_the_oracle_hidden_state_of_every_bf16_value(P):
+    from oracle import mlp_epilogue as E
+    table = P.svdq_gelu_table_fill()
+    torch.cuda.synchronize()
+    got = table.cpu().numpy().view(np.uint16)
+    x = synth.bf16_from_bits(np.arange(65536, dtype=np.uint32).astype(np.uint16)).astype(np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        ref = E.hidden_state(x)
+    ref_bits = (ref.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(synth.bf16_from_bits(got)), nan)
+    assert np.array_equal(got[~nan], ref_bits[~nan]), np.argwhere(got[~nan] != ref_bits[~nan])[:5]
+
+
 MLP = [
     ("tiny 300x256->512, down ->256", 300, 256, 512, 256),
     ("M tail and row blocks over pairs 1000x512->1536, down ->384", 1000, 512, 1536, 384),
@@ -288,6 +302,43 @@ def test_mlp_up_gelu_requantize_epilogue(P, name, M, K, F, Nd):
                                   M, Nd, F)
     torch.cuda.synchronize()
     check_output(Yd.float().cpu().numpy()[rows], svdq.forward(hg[rows], dn.smooth_inv, dn.R, dn.L1, dn.L2, dn.bias, g_dn))
+    assert P.svdq_device_status() == 0
+
+
+# ---------------------------------------------------------------- SVDQ W4A4, int4 / group 64
+
+INT4 = [
+    ("tiny 256x512->512", 256, 512, 512),
+    ("M tail and an odd group count 300x320->384", 300, 320, 384),
+    ("attention 4096x3072->3072", 4096, 3072, 3072),
+]
+
+
+@pytest.mark.parametrize("name,M,K,N", INT4, ids=[c[0] for c in INT4])
+def test_int4_layer(P, name, M, K, N):
+    from oracle import int4 as Q
+    w = synth.svdq_workload(M, K, N)
+    blob = P.svdq_int4_pack_weights(w.R, synth.bf16_bits(w.L1), synth.bf16_bits(w.L2), synth.bf16_bits(w.bias),
+                                    synth.bf16_bits(w.smooth_inv))
+    packed = torch.from_numpy(blob).cuda()
+    codes, scales, U = P.svdq_int4_quantize_act_lowrank_down(_bf16_dev(w.X), _bf16_dev(w.smooth_inv), packed)
+    Y = P.svdq_w4a4_int4_linear(codes, scales, U, packed, M, N, K)
+    torch.cuda.synchronize()
+    # activation codes (E4M3 bytes of the integers) and bf16 scales: bit-exact, every row
+    cx, sx = Q.quantize_activations(w.X, w.smooth_inv)
+    vals = codes.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(vals, cx.astype(np.float64)), np.argwhere(vals != cx)[:5]
+    assert np.array_equal(scales.float().cpu().numpy().T.astype(np.float64), sx)
+    # the low-rank activations (U = hi + lo, no per-tensor scale in this format)
+    Uc = U.float().cpu().numpy().astype(np.float64)
+    Ug = Uc[:, :32] + Uc[:, 32:]
+    rows = sample_rows(M, 41)
+    Xh = Q.smooth(w.X[rows], w.smooth_inv)
+    U_ref = Xh @ w.L1.astype(np.float64)
+    assert np.all(np.abs(Ug[rows] - U_ref) <= 1e-5 * (np.abs(Xh) @ np.abs(w.L1.astype(np.float64)))
+                  + 2.0 ** -15 * np.abs(U_ref) + 1e-30)
+    # the layer
+    check_output(Y.float().cpu().numpy()[rows], Q.forward(w.X[rows], w.smooth_inv, w.R, w.L1, w.L2, w.bias))
     assert P.svdq_device_status() == 0
 
 

@@ -93,3 +93,36 @@ def test_pack_rejects_bad_shapes_and_values():
     R[3, 5] = np.nan
     with pytest.raises(P.SvdqError):
         P.svdq_pack_weights(R, L1, L2, None, sm)
+
+
+def test_int4_packer_matches_the_oracle_bit_for_bit():
+    # codes (as E4M3 bytes of the integers), the bf16 scales (widened, group-major), L2^T and bias
+    import torch
+    from oracle import int4 as Q
+    rng = np.random.default_rng(17)
+    N, K = 256, 320
+    R = (rng.standard_normal((N, K)) * np.exp2(rng.integers(-6, 2, (N, 1)))).astype(np.float32)
+    R[3] = 0.0                                                      # a zero row: scales 0, codes 0
+    R[5, 64:128] = 7.0 * 0.5                                        # a group of exact code 7 at s = 0.5
+    L1 = synth.to_bf16(rng.standard_normal((K, 32)) * 0.1)
+    L2 = synth.to_bf16(rng.standard_normal((32, N)) * 0.1)
+    b = synth.to_bf16(rng.standard_normal(N) * 0.01)
+    sm = synth.to_bf16(np.exp(rng.uniform(-1, 1, K)))
+    blob = P.svdq_int4_pack_weights(R, synth.bf16_bits(L1), synth.bf16_bits(L2), synth.bf16_bits(b),
+                                    synth.bf16_bits(sm))
+    off_l1s = 1024
+    off_codes = off_l1s + ((2 * 32 * K * 2 + 1023) // 1024) * 1024
+    codes = blob[off_codes:off_codes + N * K].reshape(N, K)
+    off_sc = off_codes + ((N * K + 1023) // 1024) * 1024
+    scales = blob[off_sc:off_sc + N * (K // 64) * 4].view(np.float32).reshape(K // 64, N)
+    c_ref, s_ref = Q.quantize(R)
+    vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(vals, c_ref.astype(np.float64))
+    assert np.array_equal(scales.T.astype(np.float64), s_ref)
+    assert bytes(blob[:8]) == b"SVDQINT4"
+    off_l2t = off_sc + ((N * (K // 64) * 4 + 1023) // 1024) * 1024
+    l2t = blob[off_l2t:off_l2t + N * 32 * 2].view(np.uint16).reshape(N, 32)
+    assert np.array_equal(l2t, synth.bf16_bits(L2).T)
+    off_b = off_l2t + ((N * 32 * 2 + 1023) // 1024) * 1024
+    assert np.array_equal(blob[off_b:off_b + 2 * N].view(np.uint16), synth.bf16_bits(b))
+    assert P.LIB.svdq_int4_packed_weight_bytes(N, K, 32) == blob.size
