@@ -98,3 +98,38 @@ def test_gelu_keeps_relative_accuracy_in_the_negative_tail():
         assert abs(Decimal(got) - exact) <= abs(exact) * Decimal("1e-13"), (x, got, exact)
     # and its bf16 rounding is a normal, non-zero value there
     assert E.hidden_state(np.array([-10.0]))[0] < 0.0
+
+
+def _hidden_bits(patterns):
+    """bf16 bit patterns of hidden_state over bf16 inputs given as bit patterns."""
+    u = np.asarray(patterns, dtype=np.uint32)
+    with np.errstate(all="ignore"):
+        x = (u << 16).view(np.float32).astype(np.float64)
+        h = E.hidden_state(x)
+    return (np.asarray(h, dtype=np.float32).view(np.uint32) >> 16).astype(np.int64)
+
+
+def test_hidden_state_closed_forms_over_every_bf16_pattern():
+    """Outside a window of magnitudes the table of bf16(x Phi(x)) over bf16 x has closed forms:
+    x for x >= 4 (1 - Phi(x) < 2^-14 is below half an ulp), -0 for x <= -16 (x Phi(x) underflows
+    below half the smallest bf16 subnormal), x / 2 exactly for 2^-125 <= |x| < 2^-31 (the x^2 /
+    sqrt(2 pi) term is below half an ulp of x / 2), and on the subnormal grid x / 2 rounded to
+    nearest even.  The fused MLP epilogue reads a window [2^-31, 256) of the table and applies
+    these forms elsewhere; this pins them on the oracle over all 65536 patterns."""
+    u = np.arange(65536, dtype=np.int64)
+    h = _hidden_bits(u)
+    w, s = u & 0x7FFF, u >> 15
+    finite = w < 0x7F80
+    big = finite & (w >= 0x4380)                       # |x| >= 256
+    assert np.array_equal(h[big & (s == 0)], u[big & (s == 0)])
+    assert np.all(h[big & (s == 1)] == 0x8000)
+    assert np.all(h[(w >= 0x4080) & finite & (s == 0)] == u[(w >= 0x4080) & finite & (s == 0)])   # x >= 4
+    assert np.all(h[(w >= 0x4180) & finite & (s == 1)] == 0x8000)                                # x <= -16
+    mid = (w >= 0x100) & (w < 0x3000)                  # 2^-125 <= |x| < 2^-31
+    assert np.array_equal(h[mid], u[mid] - 0x80)
+    sub = w < 0x100
+    half_even = (w >> 1) + (w & (w >> 1) & 1)
+    assert np.array_equal(h[sub], (u[sub] & 0x8000) | half_even[sub])
+    assert h[0x7F80] == 0x7F80 and h[0xFF80] == 0xFFC0
+    nan = (w > 0x7F80)
+    assert np.array_equal(h[nan], u[nan] | 0x40)
