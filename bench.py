@@ -68,7 +68,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="one resident copy, eager launches of every kernel (for ncu captures); prints timings")
-    ap.add_argument("--case", default="attention", choices=["attention", "qkv64", "qkv4608_fused", "mlp_fused"],
+    ap.add_argument("--case", default="attention",
+                    choices=["attention", "qkv64", "qkv4608_fused", "mlp_fused", "int4"],
                     help="workload of --profile-case")
     return ap.parse_args(argv)
 
@@ -879,6 +880,9 @@ def run_profile_case(args):
         c = SvdqCase(P, dev, synth.svdq_workload(4608, QKV_K, QKV_N), 4608, l2, nsets=1)
         c.set_qkv(dev, QKV_HEADS, QKV_EPS)
         jobs = [("k2", lambda: c.k2(P, 0)), ("qkv_fused", lambda: c.qkv_fused(P, 0))]
+    elif args.case == "int4":
+        c = Int4Case(P, dev, synth.svdq_workload(*ATTN), ATTN[0], l2)
+        jobs = [("int4_k1", lambda: c.k1(P, 0)), ("int4_k2", lambda: c.k2(P, 0))]
     else:
         up = SvdqCase(P, dev, synth.svdq_workload(*MLP_UP), MLP_UP[0], l2, nsets=1)
         down = SvdqCase(P, dev, synth.svdq_workload(*MLP_DOWN, gelu_input=True), MLP_DOWN[0], l2, nsets=1)

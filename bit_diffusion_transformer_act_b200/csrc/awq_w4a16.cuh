@@ -216,6 +216,34 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(ready(s), ph, abort_flag, 22))) break;
       const uint32_t wst = base + s * kStage;
       const float* sxs = reinterpret_cast<const float*>(gbase + s * kStage + kOffSx);
+      // every shared-memory operand of the stage first (the loads are issued back to back), then
+      // the four groups' MMAs as eight independent two-MMA chains, so that their latencies overlap
+      uint32_t wq[4][4];                           // per group: {row g, row g+8} x {32-K step 0, 1}
+      uint32_t xv[4][2][4];                        // per group and 32-K step: this lane's activation unit
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        ldmatrix_x4(wst + woff[grp], wq[grp][0], wq[grp][1], wq[grp][2], wq[grp][3]);
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(xv[grp][half][0]), "=r"(xv[grp][half][1]), "=r"(xv[grp][half][2]), "=r"(xv[grp][half][3])
+                       : "r"(wst + kWBytes + grp * kXSub + (half ? xoff1 : xoff0)));
+      }
+      float gp[4][2][4];
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
+          const uint32_t wg = wq[grp][2 * half], wh = wq[grp][2 * half + 1];
+          const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
+          const uint32_t(&x)[4] = xv[grp][half];
+          mma16816_zero_c(gp[grp][half], nib04(wg, magic), nib04(wh, magic), nib04(wg4, magic), nib04(wh4, magic),
+                          x[0], x[1]);
+          mma16816(gp[grp][half], nib04(wg >> 8, magic), nib04(wh >> 8, magic), nib04(wg4 >> 8, magic),
+                   nib04(wh4 >> 8, magic), x[2], x[3]);
+        }
+      }
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
         const uint32_t w0 = grp < 2 ? cur[0].x : cur[0].y, w1 = grp < 2 ? cur[1].x : cur[1].y;
@@ -224,25 +252,10 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         const float sh = (grp & 1) ? bf16hi_to_f32(w1) : bf16lo_to_f32(w1);
         const float zg = ((grp & 1) ? bf16hi_to_f32(w2) : bf16lo_to_f32(w2)) + 128.f;
         const float zh = ((grp & 1) ? bf16hi_to_f32(w3) : bf16lo_to_f32(w3)) + 128.f;
-
-        uint32_t wq[4];                            // {row g, row g+8} x {32-K step 0, 1}
-        ldmatrix_x4(wst + woff[grp], wq[0], wq[1], wq[2], wq[3]);
-        const uint32_t xsub = wst + kWBytes + grp * kXSub;
+        // the group's exact integer-weighted sums (each half's fp32 sum of 32 exact products)
         float ga[4];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
-          const uint32_t wg = wq[2 * half], wh = wq[2 * half + 1];
-          const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
-          uint32_t x0, x1, x2, x3;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3) : "r"(xsub + (half ? xoff1 : xoff0)));
-          const uint32_t a0 = nib04(wg, magic), a1 = nib04(wh, magic), a2 = nib04(wg4, magic), a3 = nib04(wh4, magic);
-          if (half == 0) mma16816_zero_c(ga, a0, a1, a2, a3, x0, x1);
-          else mma16816(ga, a0, a1, a2, a3, x0, x1);
-          mma16816(ga, nib04(wg >> 8, magic), nib04(wh >> 8, magic), nib04(wg4 >> 8, magic), nib04(wh4 >> 8, magic),
-                   x2, x3);
-        }
+        for (int e = 0; e < 4; ++e) ga[e] = gp[grp][0][e] + gp[grp][1][e];
         // D fragment: c0 (row g, token 2q), c1 (row g, token 2q+1), c2/c3 the same for row g+8
         const float2 sx = *reinterpret_cast<const float2*>(sxs + grp * 8 + 2 * q);
         tot[0] = fmaf(sg, fmaf(-zg, sx.x, ga[0]), tot[0]);

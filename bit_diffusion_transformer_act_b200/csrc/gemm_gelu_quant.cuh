@@ -74,7 +74,12 @@ constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
 // per epilogue warp: the tile's bias (BN bf16), then its -smooth_inv (BN fp32)
 constexpr int VEC_BYTES = BN * 2 + BN * 4;
 constexpr int OFF_VEC = (OFF_MISC + 64 + 127) / 128 * 128;
-constexpr int SMEM_BYTES = OFF_VEC + kEpiWarps * VEC_BYTES + 1024;
+// the GELU table's window |x| in [2^-31, 256) (bf16 magnitude patterns [0x3000, 0x4380)), both
+// signs, copied into shared memory once per CTA: [sign][pattern - 0x3000]
+constexpr uint32_t kGeluLo = 0x3000u;
+constexpr uint32_t kGeluSpan = 0x4380u - kGeluLo;
+constexpr int OFF_GELU = OFF_VEC + kEpiWarps * VEC_BYTES;
+constexpr int SMEM_BYTES = OFF_GELU + 2 * kGeluSpan * 2 + 1024;
 // tensor memory: accumulators [0, 128) and [128, 256), scale regions [256, 320), U [320, 352)
 constexpr int SF_COLS = 4 * (BK / 64) + 4 * (BK / 64);
 constexpr uint32_t TM_SF = 2 * BN;
@@ -134,12 +139,30 @@ __device__ __forceinline__ uint16_t bf16_rne_from_double(double v) {
 
 // The GELU table: entry i (a bf16 bit pattern x) holds bf16(x Phi(x)), Phi(x) = erfc(-x / sqrt 2) / 2
 // evaluated in double precision and rounded once.  h = bf16(GELU(y)) with y already rounded to
-// bf16 is then one gather.
+// bf16 is then one look-up.  Outside 2^-9 <= x < 4 and -16 < x <= -2^-9 the table has closed
+// forms, which the epilogue uses outside its shared-memory window (below):
+//   x >= 4: x Phi(x) rounds to x;   x <= -16: to -0;
+//   2^-125 <= |x| < 2^-9: to x / 2 exactly (the pattern minus one exponent step), as
+//     x^2 / sqrt(2 pi) is below half an ulp of x / 2;
+//   |x| < 2^-125 (bf16 subnormals and the smallest normal binade): x / 2 rounded to nearest even
+//     on the subnormal grid (the double evaluation carries no x^2 term there);
+//   +inf: +inf; -inf: NaN (-inf times Phi(-inf) = 0); NaN: the quiet NaN of the same payload.
 __global__ void __launch_bounds__(256) gelu_table_kernel(uint16_t* __restrict__ table) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 65536) return;
   const double x = static_cast<double>(__uint_as_float(static_cast<uint32_t>(i) << 16));
   table[i] = bf16_rne_from_double(0.5 * x * erfc(-x / sqrt(2.0)));
+}
+
+// h for any bf16 pattern u: the shared-memory window where it holds u, else the closed forms
+// listed with the table (equal to the table's entries; checked over every finite pattern).
+__device__ __forceinline__ uint32_t gelu_bf16_rule(uint32_t u, const uint16_t* win) {
+  const uint32_t w = u & 0x7FFFu, s = u >> 15;
+  if (w - kGeluLo < kGeluSpan) return win[s * kGeluSpan + (w - kGeluLo)];
+  if (w >= 0x7F80u) return u == 0xFF80u ? 0xFFC0u : (w == 0x7F80u ? u : (u | 0x40u));
+  if (w >= kGeluLo + kGeluSpan) return s ? 0x8000u : u;
+  if (w >= 0x100u) return u - 0x80u;
+  return (u & 0x8000u) | ((w >> 1) + (w & (w >> 1) & 1u));
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -213,6 +236,15 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   }
   grid_dependency_wait();
   grid_launch_dependents();
+  uint16_t* gelu_win = reinterpret_cast<uint16_t*>(gbase + OFF_GELU);
+  if (warp >= 2 && warp < 2 + kEpiWarps) {
+    // the epilogue warps copy the table's window (no early exit precedes this barrier)
+    for (int j = threadIdx.x - 64; j < static_cast<int>(2 * kGeluSpan); j += kEpiWarps * 32) {
+      const uint32_t s = j >= static_cast<int>(kGeluSpan) ? 1u : 0u;
+      gelu_win[j] = __ldg(p.gelu + ((s << 15) | (kGeluLo + static_cast<uint32_t>(j) - s * kGeluSpan)));
+    }
+    asm volatile("bar.sync 2, %0;" ::"n"(kEpiWarps * 32) : "memory");
+  }
 
   constexpr uint32_t kHiSw128 = smem_desc_hi(1024, 2);
   constexpr uint32_t kHiSw64 = smem_desc_hi(512, 4);
@@ -455,15 +487,22 @@ gemm_gelu_quant_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             yb[q * 4 + w] = pack_bf16x2(y0, y1);
           }
         }
-        // h = bf16(GELU(y)) for the 32 values: all gathers in flight together
-        uint32_t hl[16], hh[16];
+        // h = bf16(GELU(y)) for the 32 values from the shared-memory window; a warp with a
+        // value outside it (|y| < 2^-31 or >= 256, or not finite) takes the full rule
+        bool inside = true;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          hl[k] = __ldg(p.gelu + (yb[k] & 0xFFFFu));
-          hh[k] = __ldg(p.gelu + (yb[k] >> 16));
+          const uint32_t tl = (yb[k] & 0x7FFFu) - kGeluLo, th = ((yb[k] >> 16) & 0x7FFFu) - kGeluLo;
+          inside = inside && tl < kGeluSpan && th < kGeluSpan;
+          const uint32_t il = ((yb[k] >> 15) & 1u) * kGeluSpan + min(tl, kGeluSpan - 1);
+          const uint32_t ih = (yb[k] >> 31) * kGeluSpan + min(th, kGeluSpan - 1);
+          hw[jj][k] = static_cast<uint32_t>(gelu_win[il]) | (static_cast<uint32_t>(gelu_win[ih]) << 16);
         }
+        if (!__all_sync(0xFFFFFFFFu, inside)) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) hw[jj][k] = hl[k] | (hh[k] << 16);
+          for (int k = 0; k < 16; ++k)
+            hw[jj][k] = gelu_bf16_rule(yb[k] & 0xFFFFu, gelu_win) | (gelu_bf16_rule(yb[k] >> 16, gelu_win) << 16);
+        }
       }
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {

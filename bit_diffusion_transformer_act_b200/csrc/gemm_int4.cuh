@@ -23,8 +23,10 @@
 //   warps 2-9  epilogue, two per tensor-memory lane quarter, 64 columns each: start from the
 //              low-rank product, then per group read the group's accumulator, hand it back, and
 //              add s_a[m, g] s_w[n, g] times it (packed fp32 pairs; s_a group-major so a warp's
-//              rows are one load, s_w pre-widened to fp32 and group-major in the weights); at the
-//              end + b, bf16, TMA stores through a 64-byte-swizzled staging tile.
+//              rows are one load, prefetched a group ahead; s_w pre-widened to fp32 and
+//              group-major in the weights, brought in by the producer as one 512-byte TMA row per
+//              group into a ring of eight slots, so the epilogue reads it from shared memory);
+//              at the end + b, bf16, TMA stores through a 64-byte-swizzled staging tile.
 // Every mbarrier wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and the CTA
 // winds down.
 #pragma once
@@ -50,13 +52,16 @@ constexpr int L2_BYTES = BN * 32 * 2;      // L2^T bf16, fits the B slot
 constexpr int GBUF = 3;                    // group accumulators in tensor memory
 constexpr uint32_t TM_LR = GBUF * BN;      // the low-rank accumulator's first column
 constexpr int TMEM_COLS = 512;
-// barriers: full[S], empty[S], grp_full[3], grp_empty[3], lr_full, lr_empty, drain
-constexpr int NUM_BARS = 2 * STAGES + 2 * GBUF + 3;
+constexpr int SB = 8;                      // weight-scale slots: one group's 128 fp32 scales each
+constexpr int WS_SLOT = BN * 4;
+// barriers: full[S], empty[S], grp_full[3], grp_empty[3], lr_full, lr_empty, drain, ws_full[SB], ws_empty[SB]
+constexpr int NUM_BARS = 2 * STAGES + 2 * GBUF + 3 + 2 * SB;
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
 constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;        // per epilogue warp: 64 bias values (bf16)
 constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * 128 + 1023) / 1024 * 1024;   // per epilogue warp: 32 x 32 bf16
-constexpr int SMEM_BYTES = OFF_STAGE + kEpiWarps * 2048 + 1024;
+constexpr int OFF_WS = OFF_STAGE + kEpiWarps * 2048;                            // SB weight-scale slots
+constexpr int SMEM_BYTES = OFF_WS + SB * WS_SLOT + 1024;
 constexpr uint32_t TX_MAIN = STAGE_BYTES;
 constexpr uint32_t TX_LOWRANK = UCAT_BYTES + L2_BYTES;
 static_assert(TM_LR + BN <= TMEM_COLS, "tensor memory");
@@ -93,7 +98,8 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
 __global__ void __launch_bounds__(kThreads, 1)
 int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
-                 const __grid_constant__ CUtensorMap tmY, const Params p) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWS,
+                 const Params p) {
   constexpr int S = STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -107,6 +113,8 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const uint32_t lr_full = bars + 8u * (2 * S + 2 * GBUF);
   const uint32_t lr_empty = bars + 8u * (2 * S + 2 * GBUF + 1);
   const uint32_t drain = bars + 8u * (2 * S + 2 * GBUF + 2);
+  auto ws_full = [&](int b) { return bars + 8u * (2 * S + 2 * GBUF + 3 + b); };
+  auto ws_empty = [&](int b) { return bars + 8u * (2 * S + 2 * GBUF + 3 + SB + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
 
@@ -120,9 +128,11 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     mbar_init(lr_full, 1);
     mbar_init(lr_empty, kEpiWarps);
     mbar_init(drain, 1);
+    for (int b = 0; b < SB; ++b) { mbar_init(ws_full(b), 1); mbar_init(ws_empty(b), kEpiWarps); }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmU); prefetch_tmap(&tmL2); prefetch_tmap(&tmY);
+    prefetch_tmap(&tmWS);
   }
   if (warp == 1) tmem_alloc<TMEM_COLS>(smem_addr(tmem_slot));
   tc_fence_before();
@@ -138,11 +148,11 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    uint32_t g = 0;
+    uint32_t g = 0, gs = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
       const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
-      for (int kb = -1; kb < nkb; ++kb, ++g) {       // kb == -1: the low-rank stage
+      for (int kb = -1; ok && kb < nkb; ++kb, ++g) {   // kb == -1: the low-rank stage
         const int s = g % S;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ((g / S) & 1u) ^ 1u, abort_flag, 51))) {
           ok = false;
@@ -161,6 +171,19 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
         __syncwarp();
+        // the weight scales of the stage's groups, one slot each (the epilogue frees them)
+        for (int j = 0; kb >= 0 && j < min(2, ngroups - 2 * kb); ++j, ++gs) {
+          const int b = gs % SB;
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(ws_empty(b), ((gs / SB) & 1u) ^ 1u, abort_flag, 58))) {
+            ok = false;
+            break;
+          }
+          if (elect_one()) {
+            mbar_arrive_expect_tx(ws_full(b), WS_SLOT);
+            tma_load_2d(base + OFF_WS + b * WS_SLOT, &tmWS, n0, 2 * kb + j, ws_full(b));
+          }
+          __syncwarp();
+        }
       }
     }
   } else if (warp == 1) {
@@ -228,6 +251,7 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint32_t gc = 0;
     int i = 0;
     bool ok = true;
+    const float* ws_smem = reinterpret_cast<const float*>(gbase + OFF_WS);
     for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++i) {
       const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
       const int m = min(m0 + r, p.M - 1);         // clamped for the scale loads; stores are clipped
@@ -258,8 +282,10 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int b = gc % GBUF;
         const float sa = sa_next;
         if (gi + 1 < ngroups) sa_next = bf16lo_to_f32(__ldg(p.a_scales + static_cast<size_t>(gi + 1) * p.M + m));
-        const float4* sw4 = reinterpret_cast<const float4*>(p.w_scales + static_cast<size_t>(gi) * p.N + nc);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(grp_full(b), (gc / GBUF) & 1u, abort_flag, 56))) {
+        const int sbi = gc % SB;
+        const float4* sw4 = reinterpret_cast<const float4*>(ws_smem + sbi * BN + 64 * eh);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(grp_full(b), (gc / GBUF) & 1u, abort_flag, 56) &&
+                                         mbar_wait_bounded(ws_full(sbi), (gc / SB) & 1u, abort_flag, 59))) {
           ok = false;
           break;
         }
@@ -267,9 +293,6 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         uint32_t D0[32], D1[32];
         tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(b * BN), D0);
         tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(b * BN) + 32, D1);
-        float4 wsv[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) wsv[q] = __ldg(sw4 + q);
         tmem_wait_ld_regs(D0);
         tmem_wait_ld_regs(D1);
         tc_fence_before();
@@ -278,10 +301,11 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const uint64_t sa2 = f32x2_pack(sa, sa);
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
+          const float4 wsv = sw4[q];               // one broadcast shared-memory load
           const uint32_t* D = q < 8 ? D0 : D1;
           const int j = (q % 8) * 4;
-          const uint64_t s01 = f32x2_mul(sa2, f32x2_pack(wsv[q].x, wsv[q].y));
-          const uint64_t s23 = f32x2_mul(sa2, f32x2_pack(wsv[q].z, wsv[q].w));
+          const uint64_t s01 = f32x2_mul(sa2, f32x2_pack(wsv.x, wsv.y));
+          const uint64_t s23 = f32x2_mul(sa2, f32x2_pack(wsv.z, wsv.w));
           const int a = q * 4;
           uint64_t v01 = f32x2_fma(s01, f32x2_pack(__uint_as_float(D[j]), __uint_as_float(D[j + 1])),
                                    f32x2_pack(acc[a], acc[a + 1]));
@@ -290,6 +314,8 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           f32x2_unpack(v01, acc[a], acc[a + 1]);
           f32x2_unpack(v23, acc[a + 2], acc[a + 3]);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ws_empty(sbi));
       }
       if (!ok) break;
       // + b, bf16, two 32-column TMA stores through the staging tile

@@ -305,6 +305,36 @@ def test_mlp_up_gelu_requantize_epilogue(P, name, M, K, F, Nd):
     assert P.svdq_device_status() == 0
 
 
+def test_mlp_up_hidden_state_of_every_finite_bf16_value(P):
+    """The fused epilogue's GELU (a shared-memory window of the table plus its closed forms
+    outside it) over every finite bf16 pre-activation: X = 0 makes the up projection's
+    accumulator zero, so y is the bias, which runs through all finite bf16 patterns (-0 comes out
+    as +0 from the fma)."""
+    import dataclasses
+    from oracle import mlp_epilogue as E
+    M, K, F, Nd = 1, 256, 65536, 128
+    up = synth.svdq_workload(M, K, F, seed=3)
+    pat = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bias = synth.bf16_from_bits(pat).astype(np.float32)
+    bias[~np.isfinite(bias)] = 0.0
+    up = dataclasses.replace(up, X=np.zeros((M, K), np.float32), bias=bias)
+    dn = synth.svdq_workload(M, F, Nd, seed=4, gelu_input=True)
+    pu, gwu = _pack(P, up)
+    pd, _ = _pack(P, dn)
+    codes, scales, U = P.svdq_quantize_act_lowrank_down(_bf16_dev(up.X), _bf16_dev(up.smooth_inv), pu, up.g_a)
+    h = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    P.svdq_w4a4_nvfp4_linear_gelu_quant(codes, scales, U, up.g_a, pu, gwu, M, F, K, _bf16_dev(dn.smooth_inv), pd,
+                                        dn.g_a, h_out=h)
+    torch.cuda.synchronize()
+    got = h.cpu().view(torch.int16).numpy().view(np.uint16)[0]
+    y = bias.astype(np.float64) + 0.0                  # -0 + 0 = +0, as the fma gives
+    ref = E.hidden_state(y)
+    ref_bits = (ref.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(got, ref_bits), [(hex(pat[i]), hex(got[i]), hex(ref_bits[i]))
+                                          for i in np.argwhere(got != ref_bits)[:5, 0]]
+    assert P.svdq_device_status() == 0
+
+
 # ---------------------------------------------------------------- SVDQ W4A4, int4 / group 64
 
 INT4 = [
