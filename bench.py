@@ -351,7 +351,7 @@ class Int4Case:
         self.nsets = n_sets(blob.nbytes + 2 * M * K + M * K + 2 * M * N, l2_bytes)
         self.sets = [{"X": X.clone(), "W": blob_d.clone(),
                       "codes": torch.empty((M, K), dtype=torch.uint8, device=dev),
-                      "scales": torch.empty((K // 64, M), dtype=torch.bfloat16, device=dev),
+                      "scales": torch.empty((K // 64, P.int4_padded_rows(M)), dtype=torch.bfloat16, device=dev),
                       "U": torch.empty((M, 2 * RANK), dtype=torch.bfloat16, device=dev),
                       "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev)} for _ in range(self.nsets)]
 

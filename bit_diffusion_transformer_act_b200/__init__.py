@@ -25,6 +25,7 @@ from .ops import (  # noqa: F401
     svdq_gelu_quant_workspace_bytes,
     svdq_gelu_table_fill,
     svdq_int4_pack_weights,
+    int4_padded_rows,
     svdq_int4_quantize_act_lowrank_down,
     svdq_w4a4_int4_linear,
     awq_w4a16_linear,

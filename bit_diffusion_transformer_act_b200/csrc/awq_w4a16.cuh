@@ -42,13 +42,13 @@ constexpr int kWBytes = kRows * 128;       // 16 KB of packed weights per stage
 constexpr int kXSub = 8 * 128;             // one 64-column activation sub-tile (8 tokens)
 constexpr int kOffSx = kWBytes + 4 * kXSub;    // group sums: [4 groups][8 tokens] fp32
 constexpr int kStage = (kOffSx + 4 * 8 * 4 + 1023) / 1024 * 1024;
-constexpr int kStages = 9;
+constexpr int kStages = 5;                 // about 100 KB: two CTAs fit an SM (this launch's and the next's)
 constexpr int kOffBar = kStages * kStage;
 constexpr int kSmem = kOffBar + 8 * 3 * kStages + 16 + 1024;
 constexpr int kProducer = kComputeWarps, kPrepWarp = kComputeWarps + 1;
 constexpr int kThreads = (kComputeWarps + 2) * 32;
 static_assert(kStage % 1024 == 0, "1 KB alignment of swizzled tiles");
-static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
 
 struct Params {
   const __nv_bfloat16* scales;     // [N, K/64]
@@ -84,7 +84,7 @@ __device__ __forceinline__ void mma16816_zero_c(float (&d)[4], uint32_t a0, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
   constexpr int S = kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -114,11 +114,16 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     prefetch_tmap(&tmX);
   }
   __syncthreads();
+  const int npre = min(S, nkb);                    // stages whose weight tiles load before the wait
   if (warp == kProducer && lane == 0) {
-    // The weights, scales and zeros never come from the previous kernel: start the first
-    // stages' tiles and this CTA's scale and zero rows toward L2 while it finishes (hints;
-    // L2 is coherent, so nothing stale can be read).
-    for (int kb = 0; kb < min(S, nkb); ++kb) tma_prefetch_l2_2d(&tmW, kb * (kChunk / 2), n0);
+    // The weights, scales and zeros never come from the previous kernel: the first stages'
+    // weight tiles are loaded while it finishes (with the kernel small enough for two CTAs per
+    // SM, this CTA can be resident next to the previous kernel's), and this CTA's scale and
+    // zero rows are pulled toward L2 (hints; L2 is coherent, so nothing stale can be read).
+    for (int kb = 0; kb < npre; ++kb) {
+      mbar_arrive_expect_tx(full(kb), kWBytes + 4 * kXSub);
+      tma_load_2d(base + kb * kStage, &tmW, kb * (kChunk / 2), n0, full(kb));
+    }
     const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
     const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
     bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
@@ -129,7 +134,15 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
   if (warp == kProducer) {
     // ---------------------------------------------------------------- TMA producer
-    for (int kb = 0; kb < nkb; ++kb) {
+    if (elect_one()) {
+      // the activations of the stages whose weights are already on their way
+      for (int kb = 0; kb < npre; ++kb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d(base + kb * kStage + kWBytes + j * kXSub, &tmX, kb * kChunk + j * 64, 0, full(kb));
+    }
+    __syncwarp();
+    for (int kb = npre; kb < nkb; ++kb) {
       const int s = kb % S;
       const uint32_t ph = (kb / S) & 1u;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 21))) break;

@@ -14,18 +14,18 @@
 // products (at most 3136 in magnitude) is exact in the fp32 accumulator.  Because both
 // operands carry their own scale per group, the scale product s_a s_w differs for every
 // (row, column, group): each group gets its own accumulator, and the epilogue applies the
-// scales.  Persistent CTAs over 128 x 128 output tiles, 384 threads:
+// scales.  Persistent CTAs over 128 x 128 output tiles, 576 threads:
 //   warp 0     TMA producer: per tile the low-rank tiles ([U hi | U lo], L2^T) as one stage, then
 //              per 128-K stage the 128 x 128-byte code tiles of A and B (128-byte swizzle).
 //   warp 1     tensor memory and the MMA issue: the low-rank product (four bf16 MMAs, K = 16)
 //              into its own 128-column accumulator, then per group two fp8 MMAs (K = 32) into
 //              one of three rotating 128-column group accumulators.
-//   warps 2-9  epilogue, two per tensor-memory lane quarter, 64 columns each: start from the
+//   warps 2-17 epilogue, four per tensor-memory lane quarter, 32 columns each: start from the
 //              low-rank product, then per group read the group's accumulator, hand it back, and
-//              add s_a[m, g] s_w[n, g] times it (packed fp32 pairs; s_a group-major so a warp's
-//              rows are one load, prefetched a group ahead; s_w pre-widened to fp32 and
-//              group-major in the weights, brought in by the producer as one 512-byte TMA row per
-//              group into a ring of eight slots, so the epilogue reads it from shared memory);
+//              add s_a[m, g] s_w[n, g] times it (packed fp32 pairs; both scales group-major --
+//              s_w pre-widened to fp32 in the weights, s_a bf16 with rows padded to 128 -- and
+//              brought in by the producer, per group a 512-byte and a 256-byte TMA row, into a
+//              ring of eight slots, so the epilogue's loop reads no global memory);
 //              at the end + b, bf16, TMA stores through a 64-byte-swizzled staging tile.
 // Every mbarrier wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and the CTA
 // winds down.
@@ -42,7 +42,8 @@ constexpr int BN = 128;
 constexpr int BK = 128;                    // K per stage: two groups
 constexpr int kGroup = 64;
 constexpr int STAGES = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;              // four per tensor-memory lane quarter
+constexpr int kCols = BN / (kEpiWarps / 4);  // accumulator columns per epilogue warp (32)
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int A_BYTES = BM * BK;           // E4M3 codes
 constexpr int B_BYTES = BN * BK;
@@ -52,14 +53,14 @@ constexpr int L2_BYTES = BN * 32 * 2;      // L2^T bf16, fits the B slot
 constexpr int GBUF = 3;                    // group accumulators in tensor memory
 constexpr uint32_t TM_LR = GBUF * BN;      // the low-rank accumulator's first column
 constexpr int TMEM_COLS = 512;
-constexpr int SB = 8;                      // weight-scale slots: one group's 128 fp32 scales each
-constexpr int WS_SLOT = BN * 4;
+constexpr int SB = 8;                      // scale slots: one group's 128 fp32 weight scales, then its
+constexpr int WS_SLOT = BN * 4 + BM * 2;   // 128 bf16 activation scales
 // barriers: full[S], empty[S], grp_full[3], grp_empty[3], lr_full, lr_empty, drain, ws_full[SB], ws_empty[SB]
 constexpr int NUM_BARS = 2 * STAGES + 2 * GBUF + 3 + 2 * SB;
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
-constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;        // per epilogue warp: 64 bias values (bf16)
-constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * 128 + 1023) / 1024 * 1024;   // per epilogue warp: 32 x 32 bf16
+constexpr int OFF_BIAS = (OFF_MISC + 64 + 127) / 128 * 128;        // per epilogue warp: kCols bias values (bf16)
+constexpr int OFF_STAGE = (OFF_BIAS + kEpiWarps * kCols * 2 + 1023) / 1024 * 1024;   // per epilogue warp: 32 x 32 bf16
 constexpr int OFF_WS = OFF_STAGE + kEpiWarps * 2048;                            // SB weight-scale slots
 constexpr int SMEM_BYTES = OFF_WS + SB * WS_SLOT + 1024;
 constexpr uint32_t TX_MAIN = STAGE_BYTES;
@@ -70,8 +71,6 @@ static_assert(UCAT_BYTES <= A_BYTES && L2_BYTES <= B_BYTES, "low-rank tiles fit 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 struct Params {
-  const uint16_t* a_scales;        // bf16 [K/64][M] (group-major)
-  const float* w_scales;           // fp32 [K/64][N] (group-major)
   const __nv_bfloat16* bias;       // [N]
   int M, N, K;
   int tiles_n, tiles;
@@ -99,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWS,
-                 const Params p) {
+                 const __grid_constant__ CUtensorMap tmAS, const Params p) {
   constexpr int S = STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -132,7 +131,7 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmU); prefetch_tmap(&tmL2); prefetch_tmap(&tmY);
-    prefetch_tmap(&tmWS);
+    prefetch_tmap(&tmWS); prefetch_tmap(&tmAS);
   }
   if (warp == 1) tmem_alloc<TMEM_COLS>(smem_addr(tmem_slot));
   tc_fence_before();
@@ -171,7 +170,8 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
         __syncwarp();
-        // the weight scales of the stage's groups, one slot each (the epilogue frees them)
+        // the scales of the stage's groups (weights, then activations), one slot each (the
+        // epilogue frees them)
         for (int j = 0; kb >= 0 && j < min(2, ngroups - 2 * kb); ++j, ++gs) {
           const int b = gs % SB;
           if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(ws_empty(b), ((gs / SB) & 1u) ^ 1u, abort_flag, 58))) {
@@ -181,6 +181,7 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (elect_one()) {
             mbar_arrive_expect_tx(ws_full(b), WS_SLOT);
             tma_load_2d(base + OFF_WS + b * WS_SLOT, &tmWS, n0, 2 * kb + j, ws_full(b));
+            tma_load_2d(base + OFF_WS + b * WS_SLOT + BN * 4, &tmAS, m0, 2 * kb + j, ws_full(b));
           }
           __syncwarp();
         }
@@ -242,68 +243,62 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int ew = warp - 2;
-    const int eh = ew >> 2;                        // columns 64 eh .. 64 eh + 63 of the tile
+    const int eh = ew >> 2;                        // columns kCols eh .. kCols (eh + 1) - 1 of the tile
     const int r = quarter * 32 + lane;
-    uint8_t* sbias = gbase + OFF_BIAS + ew * 128;
+    uint8_t* sbias = gbase + OFF_BIAS + ew * (kCols * 2);
     const uint32_t stage_tile = base + OFF_STAGE + ew * 2048;
     const uint32_t stage_row = stage_tile + lane * 64;
     const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
     uint32_t gc = 0;
     int i = 0;
     bool ok = true;
-    const float* ws_smem = reinterpret_cast<const float*>(gbase + OFF_WS);
+    const uint8_t* ws_smem = gbase + OFF_WS;
     for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++i) {
       const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
-      const int m = min(m0 + r, p.M - 1);         // clamped for the scale loads; stores are clipped
-      const int nc = n0 + 64 * eh;                 // this warp's first column
-      if (lane < 8)
+      const int nc = n0 + kCols * eh;              // this warp's first column
+      if (lane < kCols / 8)
         *reinterpret_cast<uint4*>(sbias + lane * 16) = __ldg(reinterpret_cast<const uint4*>(p.bias + nc) + lane);
       __syncwarp();
-      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(64 * eh);
+      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(kCols * eh);
       // start from the low-rank product
-      float acc[64];
+      static_assert(kCols == 32, "one 32-column tensor-memory load per warp and group");
+      float acc[kCols];
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(lr_full, i & 1, abort_flag, 55))) break;
       tc_fence_after();
       {
-        uint32_t R0[32], R1[32];
+        uint32_t R0[32];
         tmem_ld_32x32b_x32(trow + TM_LR, R0);
-        tmem_ld_32x32b_x32(trow + TM_LR + 32, R1);
         tmem_wait_ld_regs(R0);
-        tmem_wait_ld_regs(R1);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) { acc[j] = __uint_as_float(R0[j]); acc[32 + j] = __uint_as_float(R1[j]); }
+        for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(R0[j]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(lr_empty);
       // the groups
-      float sa_next = bf16lo_to_f32(__ldg(p.a_scales + m));
       for (int gi = 0; gi < ngroups; ++gi, ++gc) {
         const int b = gc % GBUF;
-        const float sa = sa_next;
-        if (gi + 1 < ngroups) sa_next = bf16lo_to_f32(__ldg(p.a_scales + static_cast<size_t>(gi + 1) * p.M + m));
         const int sbi = gc % SB;
-        const float4* sw4 = reinterpret_cast<const float4*>(ws_smem + sbi * BN + 64 * eh);
+        const uint8_t* slot = ws_smem + sbi * WS_SLOT;
+        const float4* sw4 = reinterpret_cast<const float4*>(slot) + (kCols / 4) * eh;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(grp_full(b), (gc / GBUF) & 1u, abort_flag, 56) &&
                                          mbar_wait_bounded(ws_full(sbi), (gc / SB) & 1u, abort_flag, 59))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t D0[32], D1[32];
-        tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(b * BN), D0);
-        tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(b * BN) + 32, D1);
-        tmem_wait_ld_regs(D0);
-        tmem_wait_ld_regs(D1);
+        uint32_t D[32];
+        tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(b * BN), D);
+        const float sa = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(slot + BN * 4 + 2 * r));
+        tmem_wait_ld_regs(D);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(grp_empty(b));
         const uint64_t sa2 = f32x2_pack(sa, sa);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < kCols / 4; ++q) {
           const float4 wsv = sw4[q];               // one broadcast shared-memory load
-          const uint32_t* D = q < 8 ? D0 : D1;
-          const int j = (q % 8) * 4;
+          const int j = q * 4;
           const uint64_t s01 = f32x2_mul(sa2, f32x2_pack(wsv.x, wsv.y));
           const uint64_t s23 = f32x2_mul(sa2, f32x2_pack(wsv.z, wsv.w));
           const int a = q * 4;
@@ -318,10 +313,10 @@ int4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (lane == 0) mbar_arrive(ws_empty(sbi));
       }
       if (!ok) break;
-      // + b, bf16, two 32-column TMA stores through the staging tile
+      // + b, bf16, one 32-column TMA store through the staging tile
       if (m0 + quarter * 32 < p.M) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kCols / 32; ++c) {
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
           uint32_t o[16];

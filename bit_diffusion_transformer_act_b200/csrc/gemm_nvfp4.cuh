@@ -209,11 +209,29 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   cluster_sync_all();                              // barriers of both CTAs initialised and visible
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp == 0 && lane == 0 && pair < p.tiles) {
-    // the weights do not depend on the previous kernel: start pulling this CTA's first B
-    // tiles into L2 before waiting for it
-    const int bn_first = (pair % p.tiles_n) * BN + static_cast<int>(cta) * C::BN_HALF;
-    for (int kb = 0; kb < S && kb < nkb; ++kb) tma_prefetch_l2_2d(&tmB, kb * (BK / 2), bn_first);
+  // The weights do not depend on the previous kernel: the first tile's first stages of B and
+  // its scales are loaded before waiting for it (their stages are free at the start; the
+  // full barrier of each stage's issue group gets the whole stage's byte count here, A and
+  // its scales follow after the wait).  A stage's issue group is kb / 2 for the first tile.
+  const int npre = pair < p.tiles ? min(S, nkb) : 0;
+  if (warp == 0) {
+    if (elect_one()) {
+      const int nt0 = pair % p.tiles_n;
+      const int bn0 = nt0 * BN + static_cast<int>(cta) * C::BN_HALF, nb0 = nt0 * BN / 128;
+      for (int kb = 0; kb < npre; ++kb) {
+        const uint32_t sb = base + kb * C::STAGE_BYTES;
+        const uint32_t fbar = full(static_cast<uint32_t>(kb / 2));
+        const uint32_t fb = map_to_cta(fbar, 0);
+        if (leader) mbar_arrive_expect_tx(fbar, C::TX_MAIN);
+        tma_load_2d_pair(sb + C::A_BYTES, &tmB, kb * (BK / 2), bn0, fb);
+#pragma unroll
+        for (int a = 0; a < C::SFB_ATOMS; ++a)
+          tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES + C::SFA_BYTES + a * (BK / 64) * 512, &tmSFB, 0,
+                           (nb0 + a) * natoms + kb * (BK / 64), fb);
+        if (leader && kb + 1 == nkb && (nkb & 1)) mbar_arrive(fbar);   // a one-stage group's second arrival
+      }
+    }
+    __syncwarp();
   }
   // everything above overlaps the previous kernel of the stream; its outputs (this
   // kernel's inputs) and its reads of Y are complete past this point
@@ -241,8 +259,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             const uint32_t ph = (g / S) & 1u;
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 1))) { ok = false; break; }
             const uint32_t sb = base + s * C::STAGE_BYTES;
+            const bool pre = t == pair && kb < npre;  // B, its scales and the byte count went out already
             if (elect_one()) {
-              if (kb < nkb) {
+              if (pre) {
+                tma_load_2d_pair(sb, &tmA, kb * (BK / 2), m0, fb);
+                tma_load_2d_pair(sb + C::A_BYTES + C::B_BYTES, &tmSFA, 0, rb * natoms + kb * (BK / 64), fb);
+              } else if (kb < nkb) {
                 if (leader) mbar_arrive_expect_tx(fbar, C::TX_MAIN);
                 tma_load_2d_pair(sb, &tmA, kb * (BK / 2), m0, fb);
                 tma_load_2d_pair(sb + C::A_BYTES, &tmB, kb * (BK / 2), bn0, fb);
@@ -256,7 +278,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 tma_load_2d_pair(sb, &tmU, 0, m0, fb);
                 tma_load_2d_pair(sb + C::A_BYTES, &tmL2, 0, bn0, fb);
               }
-              if (cnt == 1 && leader) mbar_arrive(fbar);          // a one-stage group's second arrival
+              if (cnt == 1 && leader && !pre) mbar_arrive(fbar);  // a one-stage group's second arrival
             }
             __syncwarp();
             ++g;
@@ -310,6 +332,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 const uint32_t sfa_lo = (sb + C::A_BYTES + C::B_BYTES) >> 4;
                 const uint32_t sfb_lo = sfa_lo + C::SFA_BYTES / 16;
                 const uint32_t tsf = tmem + C::TM_SF + (gg & 1u) * C::SF_COLS;
+                // per 64-K atom its scale copies, then its MMA: a copy waits only for the MMAs
+                // issued before it, so the next atom's copies can run while this atom's MMA does
 #pragma unroll
                 for (int kk = 0; kk < BK / 64; ++kk) {
                   if (kk < na) {
@@ -318,14 +342,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     for (int a = 0; a < C::SFB_ATOMS; ++a)
                       tc_copy_32x128b_x4_pair(tsf + C::SFB_OFF + (kk * C::SFB_ATOMS + a) * 4,
                                               make_desc(sfb_lo + (a * (BK / 64) + kk) * 32, kHiSf));
-                  }
-                }
-#pragma unroll
-                for (int kk = 0; kk < BK / 64; ++kk) {
-                  if (kk < na)
                     umma_nvfp4_pair(dacc, make_desc(a_lo + kk * 2, kHiSw128), make_desc(b_lo + kk * 2, kHiSw128),
                                     id4, tsf + 4 * kk, tsf + C::SFB_OFF + kk * C::SFB_ATOMS * 4 + sfb_shift,
                                     (kbb | kk) != 0 ? 1u : 0u);
+                  }
                 }
               } else {
                 // A: [U hi | U lo] / g_a (128-byte swizzle); B: (L2 / g_w)^T (64-byte swizzle),

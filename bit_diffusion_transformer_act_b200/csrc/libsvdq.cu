@@ -565,15 +565,15 @@ int svdq_w4a4_int4_linear(const void* act_codes, const void* act_scales, const v
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
   const svdq::BlobLayout L = svdq::blob_layout_int4(N, K, rank);
   k8::Params p;
-  p.a_scales = static_cast<const uint16_t*>(act_scales);
-  p.w_scales = reinterpret_cast<const float*>(blob + L.scales);
+  const float* w_scales = reinterpret_cast<const float*>(blob + L.scales);
   p.bias = reinterpret_cast<const __nv_bfloat16*>(blob + L.bias);
   p.M = M;
   p.N = N;
   p.K = K;
   p.tiles_n = N / k8::BN;
   p.tiles = ((M + k8::BM - 1) / k8::BM) * p.tiles_n;
-  CUtensorMap tA, tB, tU, tL2, tY, tWS;
+  CUtensorMap tA, tB, tU, tL2, tY, tWS, tAS;
+  const int mpad = (M + 127) / 128 * 128;
   if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, k8::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tB, blob + L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, 128, k8::BN,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -582,7 +582,9 @@ int svdq_w4a4_int4_linear(const void* act_codes, const void* act_scales, const v
       !make_tmap(&tL2, blob + L.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rank, rank, k8::BN,
                  CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_tmap(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_tmap(&tWS, p.w_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 64, N, k8::BN, 1,
+      !make_tmap(&tWS, w_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 64, N, k8::BN, 1,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap(&tAS, act_scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K / 64, mpad, k8::BM, 1,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ERR_CUDA;
   if (!set_smem_once<k8::int4_gemm_kernel>(k8::SMEM_BYTES, dev)) return SVDQ_ERR_CUDA;
@@ -596,7 +598,7 @@ int svdq_w4a4_int4_linear(const void* act_codes, const void* act_scales, const v
   cfg.stream = static_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k8::int4_gemm_kernel, tA, tB, tU, tL2, tY, tWS, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, k8::int4_gemm_kernel, tA, tB, tU, tL2, tY, tWS, tAS, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }

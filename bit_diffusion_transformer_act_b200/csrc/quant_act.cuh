@@ -253,6 +253,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
     // scale bytes 2h, 2h + 1 of this row's word in the chunk's 512-byte atom
     uint8_t* scale_base = p.scales + static_cast<size_t>(m0 / 128) * (p.K / 64) * 512 + (r % 32) * 16 +
                           (r / 32) * 4 + 2 * h;
+    const int mpad = (p.M + kRows - 1) / kRows * kRows;
     for (int c = 0; kInt4 && c < nck; ++c) {
       // int4 / group 64: the chunk is one group, shared by this lane and its neighbour
       const int s = c % kStages;
@@ -282,9 +283,9 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
         uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kbeg + c * kChunk + h * 32);
         dst[0] = cw[0];
         dst[1] = cw[1];
-        if (h == 0)                                // group-major [K/64][M]
-          reinterpret_cast<uint16_t*>(p.scales)[static_cast<size_t>((kbeg / 64) + c) * p.M + m] = sb;
       }
+      if (h == 0)                                  // group-major [K/64][rows padded to 128]; rows past M
+        reinterpret_cast<uint16_t*>(p.scales)[static_cast<size_t>((kbeg / 64) + c) * mpad + m] = sb;   // read zeros
     }
     for (int c = 0; !kInt4 && c < nck; ++c) {
       const int s = c % kStages;

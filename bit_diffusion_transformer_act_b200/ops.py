@@ -354,11 +354,18 @@ def svdq_w4a4_nvfp4_linear_gelu_quant(act_codes, act_scales, lowrank_act, act_gl
     return out_codes, out_scales, out_lowrank_act
 
 
+def int4_padded_rows(M):
+    """Rows of the int4 row's activation-scale array: M rounded up to a multiple of 128."""
+    return (M + 127) // 128 * 128
+
+
 def svdq_int4_quantize_act_lowrank_down(X, smooth_inv, packed_w, rank=RANK, act_codes=None, act_scales=None,
                                         lowrank_act=None):
     """The int4 row's activation pass: (act_codes uint8 [M, K] (E4M3 bytes of the int4 codes),
-    act_scales bf16 [K/64, M] (group-major), lowrank_act bf16 [M, 2r] (U as hi then lo))."""
+    act_scales bf16 [K/64, Mp] (group-major, rows padded to Mp = a multiple of 128 with zero
+    scales), lowrank_act bf16 [M, 2r] (U as hi then lo))."""
     M, K = X.shape
+    Mp = int4_padded_rows(M)
     dev = X.device
     _require_blob(packed_w, "packed_w", _l1_section_end(K, rank))
     _require(X, torch.bfloat16, (M, K), "X")
@@ -366,11 +373,11 @@ def svdq_int4_quantize_act_lowrank_down(X, smooth_inv, packed_w, rank=RANK, act_
     if act_codes is None:
         act_codes = torch.empty((M, K), dtype=torch.uint8, device=dev)
     if act_scales is None:
-        act_scales = torch.empty((K // 64, M), dtype=torch.bfloat16, device=dev)
+        act_scales = torch.empty((K // 64, Mp), dtype=torch.bfloat16, device=dev)
     if lowrank_act is None:
         lowrank_act = torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev)
     _require(act_codes, torch.uint8, (M, K), "act_codes")
-    _require(act_scales, torch.bfloat16, (K // 64, M), "act_scales")
+    _require(act_scales, torch.bfloat16, (K // 64, Mp), "act_scales")
     _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
     st = LIB.svdq_int4_quantize_act_lowrank_down(_ptr(X), _ptr(smooth_inv), _ptr(packed_w), M, K, rank,
                                                  _ptr(act_codes), _ptr(act_scales), _ptr(lowrank_act), _stream())
@@ -381,7 +388,7 @@ def svdq_int4_quantize_act_lowrank_down(X, smooth_inv, packed_w, rank=RANK, act_
 def svdq_w4a4_int4_linear(act_codes, act_scales, lowrank_act, packed_w, M, N, K, rank=RANK, Y=None):
     """Y bf16 [M, N] of the int4 / group-64 row."""
     _require(act_codes, torch.uint8, (M, K), "act_codes")
-    _require(act_scales, torch.bfloat16, (K // 64, M), "act_scales")
+    _require(act_scales, torch.bfloat16, (K // 64, int4_padded_rows(M)), "act_scales")
     _require(lowrank_act, torch.bfloat16, (M, 2 * rank), "lowrank_act")
     _require_blob(packed_w, "packed_w", int(LIB.svdq_int4_packed_weight_bytes(N, K, rank)))
     if Y is None:

@@ -236,8 +236,9 @@ int svdq_w4a4_nvfp4_linear_gelu_quant(const void* act_codes, const void* act_sca
  *   the low-rank factor section as svdq_pack_weights, codes u8 [N, K] (E4M3 bytes), the scales
  *   widened to fp32 and group-major [K/64, N], L2^T bf16 [N, rank], bias bf16 [N].
  * svdq_int4_quantize_act_lowrank_down: kernel 1's pass with this quantizer -- act_codes u8
- *   [M, K] (E4M3 bytes), act_scales bf16 [K/64, M] (group-major), lowrank_act bf16 [M, 2 rank]
- *   (U as hi then lo).  X, smooth_inv, packed_w (its low-rank section) as the nvfp4 call.
+ *   [M, K] (E4M3 bytes), act_scales bf16 [K/64, Mp] (group-major, Mp = M rounded up to a
+ *   multiple of 128; the rows past M get zero scales), lowrank_act bf16 [M, 2 rank] (U as hi then
+ *   lo).  X, smooth_inv, packed_w (its low-rank section) as the nvfp4 call.
  *   Activation scales below 2^-126 (a group amax below 7 * 2^-126) are not supported.
  * svdq_w4a4_int4_linear: Y bf16 [M, N] from those and the packed weights.
  * Errors and asynchrony as the nvfp4 calls. */

@@ -358,7 +358,10 @@ def test_int4_layer(P, name, M, K, N):
     cx, sx = Q.quantize_activations(w.X, w.smooth_inv)
     vals = codes.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
     assert np.array_equal(vals, cx.astype(np.float64)), np.argwhere(vals != cx)[:5]
-    assert np.array_equal(scales.float().cpu().numpy().T.astype(np.float64), sx)
+    sg = scales.float().cpu().numpy().astype(np.float64)
+    assert sg.shape == (K // 64, (M + 127) // 128 * 128)
+    assert np.array_equal(sg[:, :M].T, sx)
+    assert np.all(sg[:, M:] == 0)
     # the low-rank activations (U = hi + lo, no per-tensor scale in this format)
     Uc = U.float().cpu().numpy().astype(np.float64)
     Ug = Uc[:, :32] + Uc[:, 32:]
