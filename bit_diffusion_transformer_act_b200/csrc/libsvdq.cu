@@ -200,7 +200,7 @@ static int quantize_impl(const void* X, const void* smooth_inv, const void* pack
     if (kgroups % c == 0 && K / c <= k1::kMaxSlice) { ks = c; break; }
   }
   if (ks == 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-  while (ks < 8 && kgroups % (2 * ks) == 0 && rowblocks * ks < 2 * 148) ks *= 2;
+  while (ks < 8 && kgroups % (2 * ks) == 0 && rowblocks * ks < 2 * sm_count(dev)) ks *= 2;
   p.kslices = ks;
 
   CUtensorMap tX, tL;
