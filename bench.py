@@ -440,6 +440,14 @@ class Workloads:
             self.mlp_down = SvdqCase(P, dev, synth.svdq_workload(*MLP_DOWN, gelu_input=True), MLP_DOWN[0], l2_bytes)
             self.mlp_fused = MlpFused(P, dev, self.mlp_up, self.mlp_down)
 
+    def mlp_gelu_torch(self, i):
+        """The unfused pipeline's GELU: the up layer's bf16 output through PyTorch's erf-form
+        GELU into the down layer's input (the rotating sets of the two layers)."""
+        import torch
+        n = min(self.mlp_up.nsets, self.mlp_down.nsets)
+        u, d = self.mlp_up.sets[i % n], self.mlp_down.sets[i % n]
+        torch.ops.aten.gelu.out(u["Y"], approximate="none", out=d["X"])
+
     def segments(self, P):
         """(name, launches per step, fn(i)) of every segment of one step, in timing order."""
         seg = [("attn_layer", 2, lambda i: self.attn.layer(P, i)),
@@ -460,6 +468,7 @@ class Workloads:
                         ("qkv%d_torch_norm_rope" % m, 0, (lambda i, c=c: c.qkv_torch_norm_rope(P, i)))]
         if self.mlp_up is not None:
             seg += [("mlp_up", 2, lambda i: self.mlp_up.layer(P, i)),
+                    ("mlp_gelu_torch", 0, lambda i: self.mlp_gelu_torch(i)),
                     ("mlp_down", 2, lambda i: self.mlp_down.layer(P, i)),
                     ("mlp_up_fused", 3, lambda i: self.mlp_fused.up_fused(P, i)),
                     ("mlp_down_gemm", 1, lambda i: self.mlp_fused.down_gemm(P, i))]
@@ -644,10 +653,16 @@ def run_ours(args, world, rank, local):
         configs["mlp_pair"]["pair"] = {"us": t_pair, "tflops": (svdq_flops(*MLP_UP) + svdq_flops(*MLP_DOWN))
                                        / (t_pair * 1e-6) / 1e12}
         t_fused = us("mlp_up_fused") + us("mlp_down_gemm")
+        t_gelu = us("mlp_gelu_torch")
+        configs["mlp_pair"]["pair_with_gelu"] = {
+            "us": t_pair + t_gelu, "gelu_torch_us": t_gelu,
+            "note": "the unfused pipeline as a model runs it: the up layer, GELU (erf form) of its bf16 output "
+                    "as a PyTorch operation into the down layer's input, the down layer"}
         configs["mlp_pair"]["fused_gelu_requant"] = {
             "up_fused_us": us("mlp_up_fused"), "down_gemm_us": us("mlp_down_gemm"), "pair_us": t_fused,
             "tflops": (svdq_flops(*MLP_UP) + svdq_flops(*MLP_DOWN)) / (t_fused * 1e-6) / 1e12,
             "speedup_vs_unfused_pair": t_pair / t_fused,
+            "speedup_vs_unfused_pair_with_gelu": (t_pair + t_gelu) / t_fused,
             "note": "kernel 1 on X, the up GEMM with GELU and the down projection's activation pass in its "
                     "epilogue (kernels 6, 7), then the down GEMM: the 4608 x 12288 hidden state is never stored"}
 
@@ -715,7 +730,10 @@ def e2e_ours(args, P, case, dev, world, chunks=8):
     """The attention layer through the public API with the input in pinned host memory and
     the output read back to pinned host memory, every step inside the timed region.  The rows
     go in `chunks` pieces through three streams -- host-to-device copies, the two kernels,
-    device-to-host copies -- so that both copy directions and the kernels overlap."""
+    device-to-host copies -- so that both copy directions and the kernels overlap.  The
+    `e2e_steps` steps (copies, calls and their cross-stream order) are captured once into a CUDA
+    graph and replayed: eager, the ≈ 80 host calls per step (each library call encodes its
+    tensor maps) take longer than the step's transfers on the GPU."""
     import torch
     M, K, N = case.M, case.K, case.N
     s0 = case.sets[0]
@@ -760,15 +778,29 @@ def e2e_ours(args, P, case, dev, world, chunks=8):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    first[0] = True                                  # no wait on the eager steps' events in the graph
+    with torch.cuda.graph(graph, stream=cap):
+        fork = torch.cuda.Event()
+        fork.record(cap)
+        for s in (s_in, s_k, s_out):                 # every stream starts after the fork
+            s.wait_event(fork)
+        for _ in range(args.e2e_steps):
+            step()
+        for s in (s_in, s_k, s_out):                 # and the capture stream waits for all three
+            join = torch.cuda.Event()
+            join.record(s)
+            cap.wait_event(join)
+    with torch.cuda.stream(cap):
+        graph.replay()                               # warm-up replay
+    torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    s_k.wait_event(e0)                               # every stream starts after e0
-    s_out.wait_event(e0)
-    for _ in range(args.e2e_steps):
-        step()
-    s_out.wait_event(ev_k2[-1])
-    e1.record(s_out)
+    with torch.cuda.stream(cap):                     # replay() launches on the current stream
+        e0.record(cap)
+        graph.replay()
+        e1.record(cap)
     torch.cuda.synchronize()
     ms = allreduce_max(e0.elapsed_time(e1), world)
     val = world * args.e2e_steps * svdq_flops(M, K, N) / (ms * 1e-3) / 1e12
@@ -776,7 +808,8 @@ def e2e_ours(args, P, case, dev, world, chunks=8):
     return {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": hX.numel() * 2,
             "d2h_bytes_per_step": hY.numel() * 2, "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps,
             "note": "attention layer via the public API; pinned host X in, pinned host Y out, every step, "
-                    "in %d row chunks over copy-in, kernel and copy-out streams" % chunks,
+                    "in %d row chunks over copy-in, kernel and copy-out streams, the %d steps captured in one "
+                    "CUDA graph" % (chunks, args.e2e_steps),
             "host_output_matches_device": ok}
 
 

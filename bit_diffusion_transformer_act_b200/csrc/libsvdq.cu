@@ -10,6 +10,7 @@
 #include <numeric>
 #include <cmath>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/svdq.h"
 #include "layout.h"
@@ -80,17 +81,59 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps by everything that goes into the encoding (a map describes an address
+// range and its layout, not its contents, so a hit is always the map the encoder would give).
+// An eager call of the GEMM needs seven maps; encoding them is most of the call's host cost.
+struct TmapKey {
+  uintptr_t ptr;
+  uint64_t rows, cols;
+  uint32_t box_cols, box_rows;
+  int dt, elem, sw;
+  bool operator==(const TmapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_cols == o.box_cols && box_rows == o.box_rows &&
+           dt == o.dt && elem == o.elem && sw == o.sw;
+  }
+};
+struct TmapKeyHash {
+  size_t operator()(const TmapKey& k) const {
+    uint64_t h = k.ptr * 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {k.rows, k.cols, static_cast<uint64_t>(k.box_cols) << 32 | k.box_rows,
+                       static_cast<uint64_t>(k.dt) << 16 | static_cast<uint64_t>(k.elem) << 8 |
+                           static_cast<uint64_t>(k.sw)})
+      h = (h ^ v) * 0x100000001B3ull;
+    return static_cast<size_t>(h);
+  }
+};
+constexpr size_t kTmapCacheMax = 4096;            // cleared when full
+
 // 2-D row-major tensor [rows, cols] of `elem` bytes per element; box {box_cols, box_rows}.
 bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem, uint64_t rows, uint64_t cols,
                uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  static std::mutex mu;
+  static std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> cache;
+  const TmapKey key{reinterpret_cast<uintptr_t>(ptr), rows, cols, box_cols, box_rows, static_cast<int>(dt), elem,
+                    static_cast<int>(sw)};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *m = it->second;
+      return true;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= kTmapCacheMax) cache.clear();
+  cache.emplace(key, *m);
+  return true;
 }
 
 // Raises the dynamic shared-memory limit of one kernel, once per device.
