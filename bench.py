@@ -726,7 +726,7 @@ def run_ours(args, world, rank, local):
     return result
 
 
-def e2e_ours(args, P, case, dev, world, chunks=8):
+def e2e_ours(args, P, case, dev, world, chunks=4):
     """The attention layer through the public API with the input in pinned host memory and
     the output read back to pinned host memory, every step inside the timed region.  The rows
     go in `chunks` pieces through three streams -- host-to-device copies, the two kernels,
