@@ -123,7 +123,8 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
   }
 }
 
-template <int T>
+// kVec: the scale and zero rows take 8-byte loads of four groups (K % 256 == 0, aligned rows)
+template <int T, bool kVec>
 __global__ void __launch_bounds__(kThreads, 1)
 awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
   using C = Cfg<T>;
@@ -147,7 +148,8 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n0 = blockIdx.x * kRows;
-  const int nkb = p.K / kChunk;
+  const int t0 = blockIdx.y * T;                   // this CTA's first token (M > 64: one CTA row per 64 tokens)
+  const int nkb = (p.K + kChunk - 1) / kChunk;     // the last stage may hold 1-3 groups (K % 64 == 0)
   const int nunits = nkb * 4 / C::UG;                // C::UG groups per unit
   const int gpr = p.K / kGroup;                    // groups per weight row
 
@@ -175,8 +177,8 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     for (int kb = 0; kb < min(S, nkb); ++kb) tma_prefetch_l2_2d(&tmW, kb * (kChunk / 2), n0);
     const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
     const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
-    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
-    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
+    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
+    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
   }
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
@@ -192,7 +194,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         mbar_arrive_expect_tx(full(s), C::STAGE);
         tma_load_2d(sb, &tmW, kb * (kChunk / 2), n0, full(s));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * C::XSUB, &tmX, kb * kChunk + j * 64, 0, full(s));
+        for (int j = 0; j < 4; ++j) tma_load_2d(sb + kWBytes + j * C::XSUB, &tmX, kb * kChunk + j * 64, t0, full(s));
       }
       __syncwarp();
     }
@@ -234,12 +236,15 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(dq * 32) << 16) + static_cast<uint32_t>(C::A_COL0 + h * 16);
     const uint32_t magic = static_cast<uint32_t>(abort_flag[1]);   // 0x43004300, opaque to the compiler
-    const uint2* zrow = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
-    uint2 zn = __ldg(zrow);                        // zeros of the 4 groups of the next stage
+    // groups past K (a partial last stage) read as zero points 0 and their codes as 0 (zero-filled
+    // copies): their A columns are 0
+    const uint16_t* zrow = reinterpret_cast<const uint16_t*>(p.zeros) + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr;
+    constexpr bool vec = kVec;
+    uint2 zn = ld_groups4(zrow, 0, gpr, vec);      // zeros of the 4 groups of the next stage
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % S;
       const uint2 zc = zn;
-      if (kb + 1 < nkb) zn = __ldg(zrow + kb + 1);
+      if (kb + 1 < nkb) zn = ld_groups4(zrow, kb + 1, gpr, vec);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), (kb / S) & 1u, abort_flag, 35))) break;
       const uint8_t* wrow = gbase + s * C::STAGE + r * 128;
       bool ok = true;
@@ -289,16 +294,17 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     const int quarter = warp & 3;                  // tensor-memory lanes 32 quarter .. + 31
     const int r = quarter * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint2* srow = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr);
+    const uint16_t* srow = reinterpret_cast<const uint16_t*>(p.scales) + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr;
+    constexpr bool vec = kVec;
     float tot[T];
 #pragma unroll
     for (int t = 0; t < T; ++t) tot[t] = 0.f;
-    uint2 sn = __ldg(srow), sc = sn;
+    uint2 sn = ld_groups4(srow, 0, gpr, vec), sc = sn;
     for (int u = 0; u < nunits; ++u) {
       const int dp = u % DP;
       if ((u * C::UG) % 4 == 0) {                   // first unit of a stage
         sc = sn;
-        if (u * C::UG / 4 + 1 < nkb) sn = __ldg(srow + u * C::UG / 4 + 1);
+        if (u * C::UG / 4 + 1 < nkb) sn = ld_groups4(srow, u * C::UG / 4 + 1, gpr, vec);
       }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(dfull(dp), (u / DP) & 1u, abort_flag, 37))) break;
       tc_fence_after();
@@ -331,7 +337,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       const float bb = p.bias ? __bfloat162float(p.bias[n0 + r]) : 0.f;
 #pragma unroll
       for (int t = 0; t < T; ++t)
-        if (t < p.M) p.Y[static_cast<size_t>(t) * p.N + n0 + r] = __float2bfloat16_rn(tot[t] + bb);
+        if (t0 + t < p.M) p.Y[static_cast<size_t>(t0 + t) * p.N + n0 + r] = __float2bfloat16_rn(tot[t] + bb);
     }
   }
 

@@ -84,6 +84,8 @@ __device__ __forceinline__ void mma16816_zero_c(float (&d)[4], uint32_t a0, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// kVec: the scale and zero rows take 8-byte loads of four groups (K % 256 == 0, aligned rows)
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 2)
 awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
   constexpr int S = kStages;
@@ -99,7 +101,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n0 = blockIdx.x * kRows;
-  const int nkb = p.K / kChunk;
+  const int nkb = (p.K + kChunk - 1) / kChunk;     // the last stage may hold 1-3 groups (K % 64 == 0)
 
   if (warp == kProducer && lane == 0) {
     for (int s = 0; s < S; ++s) {
@@ -126,8 +128,8 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     }
     const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
     const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
-    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
-    bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
+    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
+    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
   }
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
@@ -194,10 +196,13 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     const int rg = warp * 16 + g;                  // this lane's weight rows: rg and rg + 8
     const int gpr = p.K / kGroup;                  // groups per weight row
     const int na = min(n0 + rg, p.N - 1), nb = min(n0 + rg + 8, p.N - 1);   // clamped for the loads
-    const uint2* sa = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(na) * gpr);
-    const uint2* sb_ = reinterpret_cast<const uint2*>(p.scales + static_cast<size_t>(nb) * gpr);
-    const uint2* za = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(na) * gpr);
-    const uint2* zb = reinterpret_cast<const uint2*>(p.zeros + static_cast<size_t>(nb) * gpr);
+    // rows of scales and zero points; groups past K (a partial last stage) read as 0, and their
+    // codes and activations are zero-filled by the copies, so they add nothing
+    const uint16_t* sa = reinterpret_cast<const uint16_t*>(p.scales) + static_cast<size_t>(na) * gpr;
+    const uint16_t* sb_ = reinterpret_cast<const uint16_t*>(p.scales) + static_cast<size_t>(nb) * gpr;
+    const uint16_t* za = reinterpret_cast<const uint16_t*>(p.zeros) + static_cast<size_t>(na) * gpr;
+    const uint16_t* zb = reinterpret_cast<const uint16_t*>(p.zeros) + static_cast<size_t>(nb) * gpr;
+    constexpr bool vec = kVec;
     // ldmatrix: this lane's row address (matrices: rows 0-7 / 8-15 of the slice, 32-K steps 2 grp / 2 grp + 1)
     const int lrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
     uint32_t woff[4];
@@ -213,8 +218,10 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     uint2 pa[4], pb[4];
     {
       const int k1 = min(1, nkb - 1);
-      pa[0] = __ldg(sa); pa[1] = __ldg(sb_); pa[2] = __ldg(za); pa[3] = __ldg(zb);
-      pb[0] = __ldg(sa + k1); pb[1] = __ldg(sb_ + k1); pb[2] = __ldg(za + k1); pb[3] = __ldg(zb + k1);
+      pa[0] = ld_groups4(sa, 0, gpr, vec); pa[1] = ld_groups4(sb_, 0, gpr, vec);
+      pa[2] = ld_groups4(za, 0, gpr, vec); pa[3] = ld_groups4(zb, 0, gpr, vec);
+      pb[0] = ld_groups4(sa, k1, gpr, vec); pb[1] = ld_groups4(sb_, k1, gpr, vec);
+      pb[2] = ld_groups4(za, k1, gpr, vec); pb[3] = ld_groups4(zb, k1, gpr, vec);
     }
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % S;
@@ -224,7 +231,8 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       for (int t = 0; t < 4; ++t) pa[t] = pb[t];
       {
         const int kk = min(kb + 2, nkb - 1);
-        pb[0] = __ldg(sa + kk); pb[1] = __ldg(sb_ + kk); pb[2] = __ldg(za + kk); pb[3] = __ldg(zb + kk);
+        pb[0] = ld_groups4(sa, kk, gpr, vec); pb[1] = ld_groups4(sb_, kk, gpr, vec);
+        pb[2] = ld_groups4(za, kk, gpr, vec); pb[3] = ld_groups4(zb, kk, gpr, vec);
       }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(ready(s), ph, abort_flag, 22))) break;
       const uint32_t wst = base + s * kStage;

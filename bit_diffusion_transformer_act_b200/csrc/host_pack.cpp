@@ -123,7 +123,7 @@ const char* svdq_status_string(int status) {
 int svdq_abi_version(void) { return svdq::kAbiVersion; }
 
 size_t svdq_packed_weight_bytes(int N, int K, int rank) {
-  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || rank != svdq::kRank) return 0;
+  if (N <= 0 || K <= 0 || N % 64 != 0 || K % 64 != 0 || rank != svdq::kRank) return 0;
   return svdq::blob_layout(N, K, rank).total;
 }
 
@@ -136,7 +136,7 @@ int svdq_pack_weights(const float* R, const uint16_t* L1, const uint16_t* L2,
                       const uint16_t* bias, const uint16_t* smooth_inv, int N, int K, int rank,
                       void* out, size_t out_bytes, float* w_global_scale) {
   if (!R || !L1 || !L2 || !smooth_inv || !out || !w_global_scale) return SVDQ_ERR_INVALID_ARG;
-  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || rank != svdq::kRank)
+  if (N <= 0 || K <= 0 || N % 64 != 0 || K % 64 != 0 || rank != svdq::kRank)
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
   if (out_bytes < L.total) return SVDQ_ERR_INVALID_ARG;

@@ -9,7 +9,9 @@
 //   codes        u8   [N][K/2]    E2M1 codes of R, element 2i in the low nibble
 //   scales       u8   swizzled E4M3 block scales of R (128-row x 64-K atoms)
 //   l2t          bf16 [N][rank]   (L2 / g_w) transposed (rank contiguous)
-//   bias         bf16 [N]         zeros when the layer has no bias
+//   bias         bf16 [N]         zeros when the layer has no bias; zero-padded to a multiple
+//                                 of 256 columns, so an output tile of N's ragged end (N % 64
+//                                 == 0) reads its bias inside the blob
 // Every section starts on a 1024-byte boundary.
 #pragma once
 
@@ -47,7 +49,7 @@ inline BlobLayout blob_layout(size_t N, size_t K, size_t rank) {
   L.codes = off;  off = align_up(off + N * K / 2, kBlobAlign);
   L.scales = off; off = align_up(off + swizzled_scale_bytes(N, K), kBlobAlign);
   L.l2t = off;    off = align_up(off + N * rank * 2, kBlobAlign);
-  L.bias = off;   off = align_up(off + N * 2, kBlobAlign);
+  L.bias = off;   off = align_up(off + align_up(N, 256) * 2, kBlobAlign);
   L.total = off;
   return L;
 }

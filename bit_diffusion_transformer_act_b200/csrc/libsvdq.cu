@@ -315,7 +315,7 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   if (!act_amax && !is_pow2_scale(act_global_scale)) return SVDQ_ERR_INVALID_ARG;
   if (act_amax && (reinterpret_cast<uintptr_t>(act_amax) & 3u)) return SVDQ_ERR_INVALID_ARG;
   if (act_amax) act_global_scale = 1.0f;
-  if (rank != svdq::kRank || K % 64 != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (rank != svdq::kRank || K % 64 != 0 || N % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!act_codes || !act_scales || !lowrank_act || !packed_w || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lowrank_act) || !aligned16(packed_w) ||
@@ -329,9 +329,11 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   namespace k2 = svdq::k2;
   const uint8_t* blob = static_cast<const uint8_t*>(packed_w);
   const svdq::BlobLayout L = svdq::blob_layout(N, K, rank);
-  // Output tile width: the widest that divides N, unless at this M its tiles would leave CTA
-  // pairs idle (few rows: the kernel is bound by streaming the weights, and every pair should
-  // stream its share) -- then the width giving the most tiles up to one per pair.
+  // Output tile width: the widest that divides N (128 with a ragged last tile when N % 128 == 64:
+  // its B rows, scales and L2 rows past N read as zeros, its bias from the blob's zero padding,
+  // and its store is clipped at N), unless at this M its tiles would leave CTA pairs idle (few
+  // rows: the kernel is bound by streaming the weights, and every pair should stream its share)
+  // -- then the width giving the most tiles up to one per pair.
   const int mtiles = (M + 255) / 256;
   const int npairs = sm_count(dev) / 2;
   int BN = (N % 256 == 0) ? 256 : (N % 192 == 0 ? 192 : 128);
@@ -348,7 +350,7 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
   p.M = M;
   p.N = N;
   p.K = K;
-  p.tiles_n = N / BN;
+  p.tiles_n = (N + BN - 1) / BN;
   p.tiles = ((M + 255) / 256) * p.tiles_n;
   p.alpha = static_cast<float>(alpha);
   p.amax = static_cast<const unsigned int*>(act_amax);
@@ -368,7 +370,7 @@ static int linear_impl(const void* act_codes, const void* act_scales, const void
 
   const int natoms = K / 64;
   const uint64_t sfa_rows = static_cast<uint64_t>((M + 127) / 128) * natoms;
-  const uint64_t sfb_rows = static_cast<uint64_t>(N / 128) * natoms;
+  const uint64_t sfb_rows = static_cast<uint64_t>((N + 127) / 128) * natoms;   // scale rows padded to 128
   CUtensorMap tA, tB, tSFA, tSFB, tU, tL2, tY;
   if (!make_tmap(&tA, act_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, 128, k2::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -732,11 +734,11 @@ int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, v
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, const void* zeros, const void* bias,
                      int M, int N, int K, void* Y, void* stream) {
   if (M < 0 || N <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
-  if (M > 64 || N % 64 != 0 || K % 256 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (N % 64 != 0 || K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!X || !qweight || !scales || !zeros || !Y) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(qweight) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(scales) & 7u) ||
-      (reinterpret_cast<uintptr_t>(zeros) & 7u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)))
+  if (!aligned16(X) || !aligned16(qweight) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+      (reinterpret_cast<uintptr_t>(zeros) & 1u) || (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)))
     return SVDQ_ERR_INVALID_ARG;
   int dev;
   if (int st = current_device_ok(&dev)) return st;
@@ -750,14 +752,17 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   p.M = M;
   p.N = N;
   p.K = K;
-  // M <= 8: mma.sync kernel (one 8-token tile); M > 8: tcgen05 kernel with T = 16, 32 or 64 token columns
+  const bool vec = K % 256 == 0 && !(reinterpret_cast<uintptr_t>(scales) & 7u) &&
+                   !(reinterpret_cast<uintptr_t>(zeros) & 7u);   // 8-byte loads of four groups
+  // M <= 8: mma.sync kernel (one 8-token tile); M > 8: tcgen05 kernel with T = 16, 32 or 64 token
+  // columns, M > 64 in 64-token tiles (a grid row per tile; each re-reads the weights, from L2)
   const int tx = M <= 8 ? 8 : (M <= 16 ? 16 : (M <= 32 ? 32 : 64));
   CUtensorMap tW, tX;
   if (!make_tmap(&tW, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, k3::kRows,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, tx, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
-  const dim3 grid((N + k3::kRows - 1) / k3::kRows, 1, 1);
+  const dim3 grid((N + k3::kRows - 1) / k3::kRows, (M + tx - 1) / tx, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
 #define SVDQ_AWQ_LAUNCH(KERNEL, SMEM_, THREADS_, PARAMS_)                                       \
@@ -781,7 +786,8 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   } while (0)
 
   if (tx == 8) {
-    SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel, k3::kSmem, k3::kThreads, p);
+    if (vec) SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<true>, k3::kSmem, k3::kThreads, p);
+    else SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<false>, k3::kSmem, k3::kThreads, p);
   } else {
     namespace k4 = svdq::k4;
     k4::Params q;
@@ -792,9 +798,16 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     q.M = M;
     q.N = N;
     q.K = K;
-    if (tx == 16) SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<16>, k4::Cfg<16>::SMEM, k4::kThreads, q);
-    else if (tx == 32) SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<32>, k4::Cfg<32>::SMEM, k4::kThreads, q);
-    else SVDQ_AWQ_LAUNCH(k4::awq_umma_kernel<64>, k4::Cfg<64>::SMEM, k4::kThreads, q);
+    if (tx == 16) {
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true>), k4::Cfg<16>::SMEM, k4::kThreads, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, false>), k4::Cfg<16>::SMEM, k4::kThreads, q);
+    } else if (tx == 32) {
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true>), k4::Cfg<32>::SMEM, k4::kThreads, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, false>), k4::Cfg<32>::SMEM, k4::kThreads, q);
+    } else {
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true>), k4::Cfg<64>::SMEM, k4::kThreads, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, false>), k4::Cfg<64>::SMEM, k4::kThreads, q);
+    }
   }
 #undef SVDQ_AWQ_LAUNCH
   return launch_status();

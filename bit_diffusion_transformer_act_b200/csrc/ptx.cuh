@@ -157,6 +157,13 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                : "memory");
 }
 
+// The same hint for any range: the 16-byte-aligned span inside [src, src + bytes), if any.
+__device__ __forceinline__ void bulk_prefetch_l2_any(const void* src, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src), e = a + bytes;
+  const uintptr_t a16 = (a + 15) & ~static_cast<uintptr_t>(15), e16 = e & ~static_cast<uintptr_t>(15);
+  if (e16 > a16) bulk_prefetch_l2(reinterpret_cast<const void*>(a16), static_cast<uint32_t>(e16 - a16));
+}
+
 // TMA tile store shared -> global (bulk async-group completion); rows or columns of
 // the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int x, int y) {
@@ -308,6 +315,18 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+// The 16-bit words of groups 4 kb .. 4 kb + 3 of a row of `gpr` per-group values (AWQ scales and
+// zero points), packed as two 32-bit words: one 8-byte load when every row starts 8-byte aligned
+// and holds a multiple of four groups (vec), else four 2-byte loads with the groups past the row's
+// end read as 0.
+__device__ __forceinline__ uint2 ld_groups4(const uint16_t* row, int kb, int gpr, bool vec) {
+  if (vec) return __ldg(reinterpret_cast<const uint2*>(row) + kb);
+  uint32_t h[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) h[j] = 4 * kb + j < gpr ? __ldg(row + 4 * kb + j) : 0u;
+  return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 }
 
 // ------------------------------------------------------------------ conversions

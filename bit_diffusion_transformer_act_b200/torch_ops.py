@@ -131,7 +131,8 @@ class SvdqLinear(nn.Module):
 
 class AwqLinear(nn.Module):
     """AWQ-style W4A16 int4 (group 64) linear layer, a drop-in for nn.Linear on bf16 inputs
-    of any leading shape with at most 64 rows after flattening."""
+    of any leading shape (built for the few rows of the adaptive normalisation; more than 64
+    rows after flattening run in 64-row tiles that each re-read the weights)."""
 
     def __init__(self, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
                  bias: Optional[torch.Tensor] = None):

@@ -90,7 +90,8 @@ size_t svdq_packed_weight_bytes(int N, int K, int rank);
  *   bias  bf16   [N] or NULL (then the bias is zero).
  *   smooth_inv bf16 [K]    the layer's 1/lambda; the same vector must be passed
  *                          to svdq_quantize_act_lowrank_down.
- *   N % 128 == 0, K % 64 == 0, N, K > 0, rank == 32.
+ *   N % 64 == 0, K % 64 == 0, N, K > 0, rank == 32 (the fused QKV and MLP calls and the int4 row
+ *   need N % 128 == 0).
  *   out   host buffer of out_bytes >= svdq_packed_weight_bytes(N, K, rank).
  *   w_global_scale  receives g_w = 2^ceil(log2(amax(R) / 2688)) (1 if R == 0).
  * The blob is device-private: copy it to the GPU as it is and pass that copy
@@ -144,8 +145,8 @@ int svdq_quantize_act_lowrank_down(const void* X, const void* smooth_inv,
  *   act_global_scale  the g_a given to kernel 1 (power of two)
  *   packed_w          device copy of the blob; w_global_scale its g_w
  *   Y                 device bf16 [M, N] out
- * N % 128 == 0, K % 64 == 0, rank == 32, M >= 0; all pointers 16-byte
- * aligned.  Asynchronous on `stream`. */
+ * N % 64 == 0 (when N % 128 == 64 the last output tile is 128 columns wide and ragged), K % 64 ==
+ * 0, rank == 32, M >= 0; all pointers 16-byte aligned.  Asynchronous on `stream`. */
 int svdq_w4a4_nvfp4_linear(const void* act_codes, const void* act_scales,
                            const void* lowrank_act, float act_global_scale,
                            const void* packed_w, float w_global_scale,
@@ -308,8 +309,10 @@ int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, v
 /* ---------------------------------------------------------------- AWQ W4A16 */
 
 /* y = X ((q - z) s)^T (+ b), weight-only int4 with group 64 along K.  M <= 8 runs the
- * mma.sync kernel (kernel 3), 9 <= M <= 64 the tcgen05 kernel (kernel 4, 16, 32 or 64
- * token columns).  Both form every product exactly and scale each group's fp32 sum by s
+ * mma.sync kernel (kernel 3), M >= 9 the tcgen05 kernel (kernel 4, 16, 32 or 64 token
+ * columns; past 64 tokens one row of CTAs per 64-token tile, each re-reading the weights from
+ * L2 -- correct at any M, but the layer is built for the small token counts of the adaptive
+ * normalisation).  Both form every product exactly and scale each group's fp32 sum by s
  * once; kernel 4 multiplies (q - z) x, kernel 3 forms s (sum (128 + q) x - (128 + z) sum x),
  * so the two differ only in fp32 rounding.
  *   X        device bf16 [M, K]
@@ -318,8 +321,9 @@ int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, v
  *   zeros    device bf16 [N, K/64], integer zero points 0..15
  *   bias     device bf16 [N] or NULL
  *   Y        device bf16 [M, N] out
- * 1 <= M <= 64 (or M == 0), N % 64 == 0, K % 256 == 0; pointers 16-byte
- * aligned.  Asynchronous on `stream`. */
+ * M >= 0 (M == 0 does nothing), N % 64 == 0, K % 64 == 0 (a K that is not a multiple of 256
+ * ends in a partial 256-K stage); X, qweight and Y 16-byte aligned, scales, zeros and bias
+ * 2-byte aligned.  Asynchronous on `stream`. */
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales,
                      const void* zeros, const void* bias, int M, int N, int K,
                      void* Y, void* stream);

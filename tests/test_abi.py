@@ -49,7 +49,8 @@ def test_status_strings_and_version():
 
 def test_sizes():
     assert P.svdq_packed_weight_bytes(3072, 3072) > 3072 * 1536
-    assert P.svdq_packed_weight_bytes(100, 3072) == 0          # N % 128
+    assert P.svdq_packed_weight_bytes(100, 3072) == 0          # N % 64
+    assert P.svdq_packed_weight_bytes(320, 3072) > 0           # N % 64 == 0 with N % 128 == 64
     assert P.svdq_packed_weight_bytes(128, 100) == 0           # K % 64
     assert P.svdq_packed_weight_bytes(128, 64, 16) == 0        # rank
     assert P.svdq_act_scale_bytes(1, 64) == 128 * 4
@@ -72,13 +73,15 @@ def test_gpu_entry_points_reject_bad_arguments_before_any_device_work():
     # unsupported shapes
     assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 96, 32, 1.0, FAKE, FAKE, FAKE, None) == 2
     assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, 4, 64, 16, 1.0, FAKE, FAKE, FAKE, None) == 2
-    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 192, 64, 32, FAKE, None) == 2
-    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 65, 64, 256, FAKE, None) == 2
-    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 320, FAKE, None) == 2
+    assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 96, 64, 32, FAKE, None) == 2
+    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 65, 96, 256, FAKE, None) == 2      # N % 64
+    assert L.awq_w4a16_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 64, 96, FAKE, None) == 2        # K % 64
     # misaligned pointers
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert L.svdq_quantize_act_lowrank_down(odd, FAKE, FAKE, 4, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
     assert L.svdq_w4a4_nvfp4_linear(FAKE, FAKE, FAKE, 1.0, FAKE, 1.0, 4, 128, 64, 32, odd, None) == 1
+    odd2 = ctypes.c_void_p((1 << 20) + 1)
+    assert L.awq_w4a16_linear(FAKE, FAKE, odd2, FAKE, None, 4, 64, 320, FAKE, None) == 1     # scales
     # negative sizes
     assert L.svdq_quantize_act_lowrank_down(FAKE, FAKE, FAKE, -1, 64, 32, 1.0, FAKE, FAKE, FAKE, None) == 1
     # an empty batch is valid even with null buffers, and needs no device
@@ -111,7 +114,7 @@ def test_gelu_quant_entry_point_rejects_bad_arguments_before_any_device_work():
     def call(M=4, N=256, K=64, g=1.0, gd=1.0, ws=FAKE, wsb=1 << 30, h=None, codes=FAKE, table=FAKE):
         return L.svdq_w4a4_nvfp4_linear_gelu_quant(FAKE, FAKE, FAKE, g, FAKE, 1.0, M, N, K, 32, FAKE, FAKE, gd,
                                                    codes, FAKE, FAKE, ws, wsb, table, h, None)
-    assert call(N=192) == 2                             # N % 128
+    assert call(N=96) == 2 and call(N=192) == 2         # N % 128 (the fused epilogue's tiles)
     assert call(K=96) == 2
     assert call(g=0.3) == 1 and call(gd=3.0) == 1       # scales must be powers of two
     assert call(ws=None) == 1 and call(codes=None) == 1 and call(table=None) == 1
@@ -162,7 +165,7 @@ def test_dynamic_scale_entry_points_reject_bad_arguments_before_any_device_work(
     assert L.svdq_quantize_act_lowrank_down_dyn(FAKE, FAKE, FAKE, 4, 96, 32, FAKE, FAKE, FAKE, FAKE, None) == 2
     assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, None, FAKE, 1.0, 4, 128, 64, 32, FAKE, None) == 1
     assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, FAKE, FAKE, 0.3, 4, 128, 64, 32, FAKE, None) == 1
-    assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, FAKE, FAKE, 1.0, 4, 192, 64, 32, FAKE, None) == 2
+    assert L.svdq_w4a4_nvfp4_linear_dyn(FAKE, FAKE, FAKE, FAKE, FAKE, 1.0, 4, 96, 64, 32, FAKE, None) == 2
     # an empty batch is valid and needs no device
     assert L.svdq_quantize_act_lowrank_down_dyn(None, None, None, 0, 64, 32, FAKE, None, None, None, None) == 0
     assert L.svdq_w4a4_nvfp4_linear_dyn(None, None, None, FAKE, None, 1.0, 0, 128, 64, 32, None, None) == 0

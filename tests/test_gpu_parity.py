@@ -100,8 +100,11 @@ def test_tiny_layer(P):
     assert P.svdq_device_status() == 0
 
 
+# N % 128 == 64 (64, 320, 704: a ragged 128-wide last tile) and N % 192 == 0 (576) next to the
+# 128- and 256-multiples
 @pytest.mark.parametrize("M,K,N", [(1, 64, 128), (63, 192, 256), (65, 320, 128), (127, 512, 384),
-                                   (129, 256, 640), (200, 1024, 256), (300, 448, 512)])
+                                   (129, 256, 640), (200, 1024, 256), (300, 448, 512),
+                                   (7, 128, 64), (130, 256, 320), (300, 512, 704), (257, 192, 576)])
 def test_edge_shapes_and_values(P, M, K, N):
     X, smooth, g_a = _edge_activations(M, K, seed=M * 7 + K)
     rng = np.random.default_rng(K + N)
@@ -388,12 +391,15 @@ def _run_awq(P, a, bias=None):
     return Y.float().cpu().numpy()
 
 
-# M <= 8: the mma.sync kernel; 9 <= M <= 64: the tcgen05 kernel with 16, 32 or 64 token columns
-# (K >= 1024 with an even stage count splits the K chain of kernel 3 between two CTAs)
+# M <= 8: the mma.sync kernel; M >= 9: the tcgen05 kernel with 16, 32 or 64 token columns (and,
+# past 64 tokens, one row of CTAs per 64-token tile, the last one ragged); K % 64 == 0 with a
+# partial last 256-K stage (K = 64, 320, 448, 832)
 @pytest.mark.parametrize("M,K,N", [(1, 256, 64), (3, 512, 128), (8, 768, 192), (2, 1024, 320), (7, 1536, 192),
                                    (9, 256, 64), (12, 512, 192),
                                    (16, 1024, 256), (24, 1024, 384), (33, 512, 320), (48, 768, 448),
-                                   (64, 256, 128), (64, 1536, 512)])
+                                   (64, 256, 128), (64, 1536, 512),
+                                   (1, 64, 64), (5, 320, 128), (8, 832, 192), (20, 448, 256), (64, 320, 128),
+                                   (65, 512, 128), (100, 320, 192), (200, 1024, 256), (129, 64, 64)])
 def test_awq_shapes(P, M, K, N):
     a = synth.awq_workload(M, K, N, seed=M + K)
     b = synth.to_bf16(np.random.default_rng(N).standard_normal(N) * 0.1) if M % 2 else None
@@ -401,7 +407,7 @@ def test_awq_shapes(P, M, K, N):
     check_output(Y, oawq.forward(a.X, a.q, a.scales, a.zeros, b))
 
 
-@pytest.mark.parametrize("M,K", [(5, 512), (40, 512), (6, 2048)])
+@pytest.mark.parametrize("M,K", [(5, 512), (40, 512), (6, 2048), (3, 320), (70, 448)])
 def test_awq_integer_case_is_exact(P, M, K):
     # s = 1, z = 8, small integer activations: every partial sum is an exact integer in fp32
     rng = np.random.default_rng(3)

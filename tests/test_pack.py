@@ -17,8 +17,9 @@ def _sections(blob, N, K, rank=32):
     codes = off; off = al(off + N * K // 2)
     scales = off; off = al(off + ((N + 127) // 128 * 128) * (K // 16))
     l2t = off; off = al(off + N * rank * 2)
-    bias = off; off = al(off + N * 2)
+    bias = off; off = al(off + (N + 255) // 256 * 256 * 2)       # zero-padded to 256 columns
     assert off == blob.size
+    assert not blob[bias + N * 2:off].any()
     return {
         "l1s": blob[l1s:l1s + 2 * rank * K * 2].view(np.uint16).reshape(2, rank, K),
         "codes": blob[codes:codes + N * K // 2].reshape(N, K // 2),
@@ -53,6 +54,18 @@ def _check_pack(R, L1, L2, b, smooth):
 def test_pack_synthetic_tiny_layer_is_bit_exact():
     w = synth.svdq_workload(256, 512, 512)
     _check_pack(w.R, w.L1, w.L2, w.bias, w.smooth_inv)
+
+
+def test_pack_ragged_width_is_bit_exact():
+    # N % 128 == 64: scale rows padded to 128 with zeros, bias padded to 256 columns
+    w = synth.svdq_workload(64, 256, 320)
+    blob = _check_pack(w.R, w.L1, w.L2, w.bias, w.smooth_inv)
+    s = _sections(blob, 320, 256)
+    assert not unswizzle_all_rows(s["scales"], 320, 256)[320:].any()
+
+
+def unswizzle_all_rows(scales, N, K):
+    return unswizzle(scales, (N + 127) // 128 * 128, K)
 
 
 def test_pack_attention_layer_is_bit_exact():
