@@ -147,6 +147,16 @@ bool set_smem_once(int bytes, int dev) {
   return true;
 }
 
+// Allows cluster sizes above 8 for one kernel, once per device.
+template <auto Kernel>
+bool allow_nonportable_cluster_once(int dev) {
+  static std::atomic<bool> done[kMaxDevices];
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) return false;
+  done[dev].store(true, std::memory_order_release);
+  return true;
+}
+
 // Number of SMs of a device (cached).
 int sm_count(int dev) {
   static std::atomic<int> count[kMaxDevices];
@@ -244,6 +254,9 @@ static int quantize_impl(const void* X, const void* smooth_inv, const void* pack
   }
   if (ks == 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   while (ks < 8 && kgroups % (2 * ks) == 0 && rowblocks * ks < 2 * sm_count(dev)) ks *= 2;
+  // few row blocks (small M): 16 slices (a non-portable cluster size) while the grid still fits
+  // one wave at two CTAs per SM -- shorter slices, each streamed in one round trip
+  if (ks == 8 && kgroups % 16 == 0 && rowblocks * 16 <= 2 * sm_count(dev)) ks = 16;
   p.kslices = ks;
 
   CUtensorMap tX, tL;
@@ -255,6 +268,9 @@ static int quantize_impl(const void* X, const void* smooth_inv, const void* pack
   const int smem = k1::kSmemBytes;
   if (!set_smem_once<k1::quant_act_lowrank_kernel<false>>(smem, dev) ||
       !set_smem_once<k1::quant_act_lowrank_kernel<true>>(smem, dev))
+    return SVDQ_ERR_CUDA;
+  if (ks > 8 && (!allow_nonportable_cluster_once<k1::quant_act_lowrank_kernel<false>>(dev) ||
+                 !allow_nonportable_cluster_once<k1::quant_act_lowrank_kernel<true>>(dev)))
     return SVDQ_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};

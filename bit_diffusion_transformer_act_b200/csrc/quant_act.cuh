@@ -8,7 +8,8 @@
 // U = X_hat L1 (rank 32) from the same smoothed activations.
 //
 // Design (sm_100a).  A CTA owns 128 rows and one K slice; the K slices of a row
-// block form a thread-block cluster (1..8 CTAs) so that the grid fills the SMs
+// block form a thread-block cluster (1..16 CTAs; 16, a non-portable size, only where the
+// grid then still fits one wave, i.e. for a few row blocks) so that the grid fills the SMs
 // (two CTAs per SM), and the slices' partial U are summed over distributed
 // shared memory -- no global scratch, no atomics.  Warp roles:
 //   warp 0     TMA producer: per 64-column chunk the X tile (128 rows, 128-byte
@@ -362,14 +363,20 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
     const int rr = static_cast<int>(crank) * rpc + i / 8;
     const int piece = i % 8;
     const float* src_addr = upart + rr * 32 + ((piece + rr) & 7) * 4;
-    float4 v[8];
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int s0 = 0; s0 < ks; s0 += 8) {           // up to 16 slices, eight loads in flight at a time
+      float4 v[8];
 #pragma unroll
-    for (int src = 0; src < 8; ++src)             // all loads in flight before the sum
-      if (src < ks) v[src] = ld_dsmem_f32x4(src_addr, static_cast<uint32_t>(src));
-    float4 sum = v[0];
+      for (int j = 0; j < 8; ++j)
+        if (s0 + j < ks) v[j] = ld_dsmem_f32x4(src_addr, static_cast<uint32_t>(s0 + j));
 #pragma unroll
-    for (int src = 1; src < 8; ++src)
-      if (src < ks) { sum.x += v[src].x; sum.y += v[src].y; sum.z += v[src].z; sum.w += v[src].w; }
+      for (int j = 0; j < 8; ++j)                  // in slice order: deterministic
+        if (s0 + j < ks) {
+          if (s0 + j == 0) sum = v[0];
+          else { sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w; }
+        }
+    }
     const int mm = m0 + rr;
     if (mm < p.M) {
       const float uu[4] = {sum.x * inv_g, sum.y * inv_g, sum.z * inv_g, sum.w * inv_g};  // exact
