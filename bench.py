@@ -726,13 +726,14 @@ def run_ours(args, world, rank, local):
     return result
 
 
-def e2e_ours(args, P, case, dev, world, chunks=4):
+def e2e_ours(args, P, case, dev, world, chunks=1):
     """The attention layer through the public API with the input in pinned host memory and
     the output read back to pinned host memory, every step inside the timed region.  The rows
-    go in `chunks` pieces through three streams -- host-to-device copies, the two kernels,
-    device-to-host copies -- so that both copy directions and the kernels overlap; consecutive
-    steps alternate between two sets of device buffers, so a step's copy-in waits only for the
-    kernels of the step before last.  The `e2e_steps` steps (copies, calls and their
+    go in `chunks` pieces (one by default: each copy node of a graph has a fixed cost, and the
+    overlap comes from consecutive steps) through three streams -- host-to-device copies, the
+    two kernels, device-to-host copies -- so that both copy directions and the kernels overlap;
+    consecutive steps alternate between two sets of device buffers, so a step's copy-in waits
+    only for the kernels of the step before last.  The `e2e_steps` steps (copies, calls and their
     cross-stream order) are captured once into a CUDA graph and replayed: eager, the ≈ 80 host
     calls per step take longer than the step's transfers on the GPU."""
     import torch
