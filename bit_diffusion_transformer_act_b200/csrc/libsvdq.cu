@@ -781,7 +781,7 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
   const dim3 grid((N + k3::kRows - 1) / k3::kRows, (M + tx - 1) / tx, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-#define SVDQ_AWQ_LAUNCH(KERNEL, SMEM_, THREADS_, PARAMS_)                                       \
+#define SVDQ_AWQ_LAUNCH(KERNEL, SMEM_, THREADS_, ...)                                           \
   do {                                                                                          \
     const int smem = SMEM_;                                                                     \
     if (!set_smem_once<KERNEL>(smem, dev)) return SVDQ_ERR_CUDA;                                \
@@ -795,15 +795,25 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     attr[0].val.programmaticStreamSerializationAllowed = 1;                                     \
     cfg.attrs = attr;                                                                           \
     cfg.numAttrs = 1;                                                                           \
-    if (cudaLaunchKernelEx(&cfg, KERNEL, tW, tX, PARAMS_) != cudaSuccess) {                     \
+    if (cudaLaunchKernelEx(&cfg, KERNEL, __VA_ARGS__) != cudaSuccess) {                         \
       (void)cudaGetLastError();                                                                 \
       return SVDQ_ERR_CUDA;                                                                     \
     }                                                                                           \
   } while (0)
 
   if (tx == 8) {
-    if (vec) SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<true>, k3::kSmem, k3::kThreads, p);
-    else SVDQ_AWQ_LAUNCH(k3::awq_gemm_kernel<false>, k3::kSmem, k3::kThreads, p);
+    // the CTA's scale and zero rows staged in shared memory by two copies (K / 64 groups of 128
+    // rows each; the copies want 16-byte rows and a 16-byte aligned base)
+    const int gpr = K / 64;
+    CUtensorMap tS = tW, tZ = tW;
+    const bool sz = K % 512 == 0 && gpr <= k3::kMaxSzGroups && aligned16(scales) && aligned16(zeros) &&
+                    make_tmap(&tS, scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                    make_tmap(&tZ, zeros, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (sz) SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<true, true>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
+    else if (vec) SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<true, false>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
+    else SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<false, false>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
   } else {
     namespace k4 = svdq::k4;
     k4::Params q;
@@ -815,14 +825,14 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     q.N = N;
     q.K = K;
     if (tx == 16) {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true>), k4::Cfg<16>::SMEM, k4::kThreads, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, false>), k4::Cfg<16>::SMEM, k4::kThreads, q);
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, false>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, q);
     } else if (tx == 32) {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true>), k4::Cfg<32>::SMEM, k4::kThreads, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, false>), k4::Cfg<32>::SMEM, k4::kThreads, q);
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, false>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, q);
     } else {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true>), k4::Cfg<64>::SMEM, k4::kThreads, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, false>), k4::Cfg<64>::SMEM, k4::kThreads, q);
+      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, false>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, q);
     }
   }
 #undef SVDQ_AWQ_LAUNCH

@@ -421,6 +421,29 @@ def test_awq_integer_case_is_exact(P, M, K):
     assert np.array_equal(Y, synth.to_bf16(ref.astype(np.float64)))
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 1024, 192), (8, 3072, 320), (5, 4096, 128), (4, 4608, 128)])
+def test_awq_scale_paths_agree(P, M, K, N):
+    # M <= 8 reads the scale and zero rows from shared memory when K % 512 == 0, K <= 4096 and both
+    # are 16-byte aligned, else from global memory (8-byte loads of four groups when 8-byte aligned,
+    # 2-byte loads otherwise): the same values in the same order, so the outputs are bit-identical
+    a = synth.awq_workload(M, K, N, seed=K + N)
+    X = _bf16_dev(a.X)
+    qw = torch.from_numpy(a.qweight).cuda()
+    outs = []
+    for off in (0, 4, 1):                          # elements: 16-, 8- and 2-byte aligned copies
+        sb = torch.zeros((a.scales.size + 8,), dtype=torch.bfloat16, device="cuda")
+        zb = torch.zeros_like(sb)
+        s = sb[off:off + a.scales.size].view(a.scales.shape)
+        z = zb[off:off + a.zeros.size].view(a.zeros.shape)
+        s.copy_(_bf16_dev(a.scales))
+        z.copy_(_bf16_dev(a.zeros))
+        outs.append(P.awq_w4a16_linear(X, qw, s, z))
+    torch.cuda.synchronize()
+    assert P.svdq_device_status() == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    check_output(outs[0].float().cpu().numpy(), oawq.forward(a.X, a.q, a.scales, a.zeros, None))
+
+
 @pytest.fixture(scope="module")
 def awq_full():
     a = synth.awq_workload(64, 3072, 18432)
