@@ -50,6 +50,8 @@ constexpr int kDeqWarps = 8;               // two per lane quarter (half a group
 constexpr int kEpiWarp0 = 2 + kDeqWarps;
 constexpr int kMmaWarp2 = kEpiWarp0 + 4;   // the second MMA-issuing warp (odd units)
 constexpr int kThreads = (kMmaWarp2 + 1) * 32;
+constexpr int kMaxSzGroups = 64;           // K <= 4096: the CTA's scale and zero rows held in shared memory
+constexpr int kPace = 3;                   // stage kb is requested once stage kb - kPace has landed
 
 template <int T>
 struct Cfg {
@@ -60,10 +62,11 @@ struct Cfg {
   // the accumulators take more tensor memory
   static constexpr int UG = T == 64 ? 2 : 4;
   static constexpr int STAGES = T == 64 ? 4 : (T == 32 ? 6 : 8);
-  static constexpr int OFF_BAR = STAGES * STAGE;
+  static constexpr int OFF_SZ = STAGES * STAGE;             // [scales, zeros][128 rows][K / 64 <= 64 groups] bf16
+  static constexpr int OFF_BAR = OFF_SZ + 2 * kRows * kMaxSzGroups * 2;
   static constexpr int DBUFS = T == 64 ? 4 : 8;             // accumulators in tensor memory (T columns each)
   static constexpr int DPAIRS = DBUFS / UG;                 // handed over a unit at a time
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * kABufs + 2 * DPAIRS + 1;   // + drain
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * kABufs + 2 * DPAIRS + 2;   // + drain, scale rows
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int A_COL0 = DBUFS * T;                  // tensor memory: accumulators, then the A units
@@ -123,10 +126,14 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
   }
 }
 
-// kVec: the scale and zero rows take 8-byte loads of four groups (K % 256 == 0, aligned rows)
-template <int T, bool kVec>
+// kSz: the CTA's scale and zero rows are copied into shared memory once, before the grid-dependency
+// wait (tmS / tmZ: [N, K/64] bf16, box K/64 x 128; K % 512 == 0, K <= 4096, 16-byte aligned);
+// otherwise they are read from global memory a stage ahead, with 8-byte loads of four groups when
+// kVec (K % 256 == 0, aligned rows).
+template <int T, bool kVec, bool kSz>
 __global__ void __launch_bounds__(kThreads, 1)
-awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, const Params p) {
+awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ, const Params p) {
   using C = Cfg<T>;
   constexpr int S = C::STAGES;
   static_assert(4 % C::UG == 0, "units divide a stage");
@@ -143,6 +150,7 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   auto dfull = [&](int d) { return bars + 8u * (2 * S + 2 * kABufs + d); };
   auto dfree = [&](int d) { return bars + 8u * (2 * S + 2 * kABufs + DP + d); };
   const uint32_t drain = bars + 8u * (2 * S + 2 * kABufs + 2 * DP);
+  const uint32_t sz_bar = drain + 8u;              // the scale and zero rows have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 4);
 
@@ -159,11 +167,16 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     for (int a = 0; a < kABufs; ++a) { mbar_init(afull(a), kDeqWarps); mbar_init(afree(a), 1); }
     for (int d = 0; d < DP; ++d) { mbar_init(dfull(d), 1); mbar_init(dfree(d), 4); }
     mbar_init(drain, 2);                           // both MMA-issuing warps
+    mbar_init(sz_bar, 1);
     *abort_flag = 0;
     abort_flag[1] = 0x43004300;                    // the dequantization constant, read back as a register
     fence_mbar_init();
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
+    if (kSz) {
+      prefetch_tmap(&tmS);
+      prefetch_tmap(&tmZ);
+    }
   }
   if (warp == 1) tmem_alloc<C::TMEM_COLS>(smem_addr(tmem_slot));
   tc_fence_before();
@@ -171,14 +184,20 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp == 0 && lane == 0) {
-    // The weights, scales and zeros never come from the previous kernel: start the first
-    // stages' tiles and this CTA's scale and zero rows toward L2 while it finishes (hints;
-    // L2 is coherent, so nothing stale can be read).
-    for (int kb = 0; kb < min(S, nkb); ++kb) tma_prefetch_l2_2d(&tmW, kb * (kChunk / 2), n0);
-    const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
-    const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
-    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
-    bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
+    // The weights, scales and zeros never come from the previous kernel: this CTA's scale and
+    // zero rows are copied into shared memory (or pulled toward L2) and the first stages' tiles
+    // toward L2 while it finishes (hints; L2 is coherent, so nothing stale can be read).
+    if (kSz) {
+      mbar_arrive_expect_tx(sz_bar, 2u * kRows * gpr * 2);
+      tma_load_2d(base + C::OFF_SZ, &tmS, 0, n0, sz_bar);
+      tma_load_2d(base + C::OFF_SZ + kRows * kMaxSzGroups * 2, &tmZ, 0, n0, sz_bar);
+    } else {
+      const size_t rb = static_cast<size_t>(n0) * (p.K / kGroup) * 2;
+      const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.N - n0) * (p.K / kGroup) * 2);
+      bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
+      bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
+    }
+    for (int kb = 0; kb < min(kPace, nkb); ++kb) tma_prefetch_l2_2d(&tmW, kb * (kChunk / 2), n0);
   }
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
@@ -189,6 +208,12 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       const int s = kb % S;
       const uint32_t ph = (kb / S) & 1u;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, 31))) break;
+      if (kb >= kPace) {
+        // paced: with every CTA's whole ring requested at once the memory system serves all of
+        // them interleaved and each CTA's first tile lands late
+        const int kp = kb - kPace;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(kp % S), (kp / S) & 1u, abort_flag, 41))) break;
+      }
       if (elect_one()) {
         const uint32_t sb = base + s * C::STAGE;
         mbar_arrive_expect_tx(full(s), C::STAGE);
@@ -239,12 +264,21 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     // groups past K (a partial last stage) read as zero points 0 and their codes as 0 (zero-filled
     // copies): their A columns are 0
     const uint16_t* zrow = reinterpret_cast<const uint16_t*>(p.zeros) + static_cast<size_t>(min(n0 + r, p.N - 1)) * gpr;
+    const uint8_t* zsm = gbase + C::OFF_SZ + kRows * kMaxSzGroups * 2 + static_cast<size_t>(r) * gpr * 2;
     constexpr bool vec = kVec;
-    uint2 zn = ld_groups4(zrow, 0, gpr, vec);      // zeros of the 4 groups of the next stage
-    for (int kb = 0; kb < nkb; ++kb) {
+    uint2 zn = make_uint2(0u, 0u);                 // zeros of the 4 groups of the next stage
+    bool sz_ok = true;
+    if constexpr (kSz) sz_ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(sz_bar, 0, abort_flag, 39));
+    else zn = ld_groups4(zrow, 0, gpr, vec);
+    for (int kb = 0; sz_ok && kb < nkb; ++kb) {
       const int s = kb % S;
-      const uint2 zc = zn;
-      if (kb + 1 < nkb) zn = ld_groups4(zrow, kb + 1, gpr, vec);
+      uint2 zc;
+      if constexpr (kSz) {
+        zc = *reinterpret_cast<const uint2*>(zsm + kb * 8);
+      } else {
+        zc = zn;
+        if (kb + 1 < nkb) zn = ld_groups4(zrow, kb + 1, gpr, vec);
+      }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full(s), (kb / S) & 1u, abort_flag, 35))) break;
       const uint8_t* wrow = gbase + s * C::STAGE + r * 128;
       bool ok = true;
@@ -299,12 +333,20 @@ awq_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     float tot[T];
 #pragma unroll
     for (int t = 0; t < T; ++t) tot[t] = 0.f;
-    uint2 sn = ld_groups4(srow, 0, gpr, vec), sc = sn;
-    for (int u = 0; u < nunits; ++u) {
+    const uint8_t* ssm = gbase + C::OFF_SZ + static_cast<size_t>(r) * gpr * 2;
+    uint2 sn = make_uint2(0u, 0u), sc = sn;
+    bool sz_ok = true;
+    if constexpr (kSz) sz_ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(sz_bar, 0, abort_flag, 40));
+    else sn = sc = ld_groups4(srow, 0, gpr, vec);
+    for (int u = 0; sz_ok && u < nunits; ++u) {
       const int dp = u % DP;
       if ((u * C::UG) % 4 == 0) {                   // first unit of a stage
-        sc = sn;
-        if (u * C::UG / 4 + 1 < nkb) sn = ld_groups4(srow, u * C::UG / 4 + 1, gpr, vec);
+        if constexpr (kSz) {
+          sc = *reinterpret_cast<const uint2*>(ssm + (u * C::UG / 4) * 8);
+        } else {
+          sc = sn;
+          if (u * C::UG / 4 + 1 < nkb) sn = ld_groups4(srow, u * C::UG / 4 + 1, gpr, vec);
+        }
       }
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(dfull(dp), (u / DP) & 1u, abort_flag, 37))) break;
       tc_fence_after();

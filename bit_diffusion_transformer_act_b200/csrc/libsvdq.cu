@@ -801,16 +801,17 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     }                                                                                           \
   } while (0)
 
+  // the CTA's scale and zero rows staged in shared memory by two copies (K / 64 groups of 128 rows
+  // each; the copies want 16-byte rows and a 16-byte aligned base)
+  const int gpr = K / 64;
+  CUtensorMap tS = tW, tZ = tW;
+  static_assert(k3::kMaxSzGroups == svdq::k4::kMaxSzGroups && k3::kRows == svdq::k4::kRows, "one staging rule");
+  const bool sz = K % 512 == 0 && gpr <= k3::kMaxSzGroups && aligned16(scales) && aligned16(zeros) &&
+                  make_tmap(&tS, scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_tmap(&tZ, zeros, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
   if (tx == 8) {
-    // the CTA's scale and zero rows staged in shared memory by two copies (K / 64 groups of 128
-    // rows each; the copies want 16-byte rows and a 16-byte aligned base)
-    const int gpr = K / 64;
-    CUtensorMap tS = tW, tZ = tW;
-    const bool sz = K % 512 == 0 && gpr <= k3::kMaxSzGroups && aligned16(scales) && aligned16(zeros) &&
-                    make_tmap(&tS, scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
-                              CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                    make_tmap(&tZ, zeros, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, gpr, gpr, k3::kRows,
-                              CU_TENSOR_MAP_SWIZZLE_NONE);
     if (sz) SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<true, true>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
     else if (vec) SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<true, false>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
     else SVDQ_AWQ_LAUNCH((k3::awq_gemm_kernel<false, false>), k3::kSmem, k3::kThreads, tW, tX, tS, tZ, p);
@@ -825,14 +826,17 @@ int awq_w4a16_linear(const void* X, const void* qweight, const void* scales, con
     q.N = N;
     q.K = K;
     if (tx == 16) {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, false>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, q);
+      if (sz) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true, true>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, true, false>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<16, false, false>), k4::Cfg<16>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
     } else if (tx == 32) {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, false>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, q);
+      if (sz) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true, true>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, true, false>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<32, false, false>), k4::Cfg<32>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
     } else {
-      if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, q);
-      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, false>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, q);
+      if (sz) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true, true>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else if (vec) SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, true, false>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
+      else SVDQ_AWQ_LAUNCH((k4::awq_umma_kernel<64, false, false>), k4::Cfg<64>::SMEM, k4::kThreads, tW, tX, tS, tZ, q);
     }
   }
 #undef SVDQ_AWQ_LAUNCH
