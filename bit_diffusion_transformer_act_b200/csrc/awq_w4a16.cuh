@@ -297,18 +297,21 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                        : "=r"(xv[grp][half][0]), "=r"(xv[grp][half][1]), "=r"(xv[grp][half][2]), "=r"(xv[grp][half][3])
                        : "r"(wst + kWBytes + grp * kXSub + (half ? xoff1 : xoff0)));
       }
-      float gp[4][2][4];
+      float gp[4][4];                              // per group: one chain of four MMAs
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int grp = 0; grp < 4; ++grp) {
           // nibbles (p, p + 4) -> K slot pairs; the activations were reordered to match
           const uint32_t wg = wq[grp][2 * half], wh = wq[grp][2 * half + 1];
           const uint32_t wg4 = wg >> 4, wh4 = wh >> 4;
           const uint32_t(&x)[4] = xv[grp][half];
-          mma16816_zero_c(gp[grp][half], nib04(wg, magic), nib04(wh, magic), nib04(wg4, magic), nib04(wh4, magic),
-                          x[0], x[1]);
-          mma16816(gp[grp][half], nib04(wg >> 8, magic), nib04(wh >> 8, magic), nib04(wg4 >> 8, magic),
+          if (half == 0)
+            mma16816_zero_c(gp[grp], nib04(wg, magic), nib04(wh, magic), nib04(wg4, magic), nib04(wh4, magic),
+                            x[0], x[1]);
+          else
+            mma16816(gp[grp], nib04(wg, magic), nib04(wh, magic), nib04(wg4, magic), nib04(wh4, magic), x[0], x[1]);
+          mma16816(gp[grp], nib04(wg >> 8, magic), nib04(wh >> 8, magic), nib04(wg4 >> 8, magic),
                    nib04(wh4 >> 8, magic), x[2], x[3]);
         }
       }
@@ -320,10 +323,8 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         const float sh = (grp & 1) ? bf16hi_to_f32(w1) : bf16lo_to_f32(w1);
         const float zg = ((grp & 1) ? bf16hi_to_f32(w2) : bf16lo_to_f32(w2)) + 128.f;
         const float zh = ((grp & 1) ? bf16hi_to_f32(w3) : bf16lo_to_f32(w3)) + 128.f;
-        // the group's exact integer-weighted sums (each half's fp32 sum of 32 exact products)
-        float ga[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ga[e] = gp[grp][0][e] + gp[grp][1][e];
+        // the group's integer-weighted sums (fp32 sums of 64 exact products)
+        const float(&ga)[4] = gp[grp];
         // D fragment: c0 (row g, token 2q), c1 (row g, token 2q+1), c2/c3 the same for row g+8
         const float2 sx = *reinterpret_cast<const float2*>(sxs + grp * 8 + 2 * q);
         tot[0] = fmaf(sg, fmaf(-zg, sx.x, ga[0]), tot[0]);
