@@ -421,11 +421,13 @@ def test_awq_integer_case_is_exact(P, M, K):
     assert np.array_equal(Y, synth.to_bf16(ref.astype(np.float64)))
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 1024, 192), (8, 3072, 320), (5, 4096, 128), (4, 4608, 128)])
+@pytest.mark.parametrize("M,K,N", [(1, 1024, 192), (8, 3072, 320), (5, 4096, 128), (4, 4608, 128),
+                                   (16, 1024, 192), (40, 3072, 128), (70, 2048, 64)])
 def test_awq_scale_paths_agree(P, M, K, N):
-    # M <= 8 reads the scale and zero rows from shared memory when K % 512 == 0, K <= 4096 and both
-    # are 16-byte aligned, else from global memory (8-byte loads of four groups when 8-byte aligned,
-    # 2-byte loads otherwise): the same values in the same order, so the outputs are bit-identical
+    # both AWQ kernels read the scale and zero rows from shared memory when K % 512 == 0, K <= 4096
+    # and both are 16-byte aligned, else from global memory (8-byte loads of four groups when 8-byte
+    # aligned, 2-byte loads otherwise): the same values in the same order, so the outputs are
+    # bit-identical
     a = synth.awq_workload(M, K, N, seed=K + N)
     X = _bf16_dev(a.X)
     qw = torch.from_numpy(a.qweight).cuda()
