@@ -140,9 +140,14 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
   const int npre = min(kPace, nkb);                // stages whose weight tiles load before the wait
   if (warp == kProducer && lane == 0) {
     // The weights, scales and zeros never come from the previous kernel: they are requested
-    // before the grid-dependency wait -- the CTA's scale and zero rows first (every stage needs
-    // them), copied into shared memory or pulled toward L2 (hints; L2 is coherent, so nothing
-    // stale can be read), then the first stages' weight tiles.
+    // before the grid-dependency wait -- the first weight tile, the CTA's scale and zero rows
+    // (every stage's epilogue needs them), copied into shared memory or pulled toward L2 (hints;
+    // L2 is coherent, so nothing stale can be read), then the next weight tiles.
+    auto load_w = [&](int kb) {
+      mbar_arrive_expect_tx(full(kb), kWBytes + 4 * kXSub);
+      tma_load_2d(base + kb * kStage, &tmW, kb * (kChunk / 2), n0, full(kb));
+    };
+    if (npre > 0) load_w(0);
     if (kSz) {
       const int gpr = p.K / kGroup;
       mbar_arrive_expect_tx(sz_bar, 2u * kRows * gpr * 2);
@@ -154,10 +159,7 @@ awq_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
       bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.scales) + rb, bytes);
       bulk_prefetch_l2_any(reinterpret_cast<const uint8_t*>(p.zeros) + rb, bytes);
     }
-    for (int kb = 0; kb < npre; ++kb) {
-      mbar_arrive_expect_tx(full(kb), kWBytes + 4 * kXSub);
-      tma_load_2d(base + kb * kStage, &tmW, kb * (kChunk / 2), n0, full(kb));
-    }
+    for (int kb = 1; kb < npre; ++kb) load_w(kb);
   }
   grid_dependency_wait();                          // X may belong to the previous kernel
   grid_launch_dependents();
