@@ -323,7 +323,9 @@ int svdq_act_amax_noalloc(const void* X, const void* smooth_inv, int M, int K, v
  *   Y        device bf16 [M, N] out
  * M >= 0 (M == 0 does nothing), N % 64 == 0, K % 64 == 0 (a K that is not a multiple of 256
  * ends in a partial 256-K stage); X, qweight and Y 16-byte aligned, scales, zeros and bias
- * 2-byte aligned.  Asynchronous on `stream`. */
+ * 2-byte aligned.  With K % 512 == 0, K <= 4096 and scales and zeros 16-byte aligned, both
+ * kernels copy each CTA's scale and zero rows into shared memory up front (the faster path;
+ * the results are bit-identical to those of the other alignments).  Asynchronous on `stream`. */
 int awq_w4a16_linear(const void* X, const void* qweight, const void* scales,
                      const void* zeros, const void* bias, int M, int N, int K,
                      void* Y, void* stream);
