@@ -14,9 +14,13 @@
 // accumulators in tensor memory too.  Keeping A out of shared memory matters: a bf16 A
 // written to and read back from shared memory costs four times the packed weight bytes
 // twice, more shared-memory bandwidth than the MMAs' own B reads.  480 threads:
-//   warp 0     TMA producer: per 256-K stage the 128 x 128-byte weight-code tile and
-//              the tokens' activations as four 64-column sub-tiles (128-byte swizzle,
-//              rows past M read as zeros) -- the MMA's B operand as they land.
+//   warp 0     TMA producer: before the grid-dependency wait the CTA's scale and zero rows
+//              into shared memory (when K % 512 == 0, K <= 4096 and both are 16-byte
+//              aligned; else the dequantizers and the epilogue read them from global memory a
+//              stage ahead); then per 256-K stage the 128 x 128-byte weight-code tile and the
+//              tokens' activations as four 64-column sub-tiles (128-byte swizzle, rows past
+//              M read as zeros) -- the MMA's B operand as they land -- paced: stage kb is
+//              requested once stage kb - 3 has landed.
 //   warps 2-9  dequantizers, two per tensor-memory lane quarter: a thread owns one weight
 //              row (its lane) and half of every group; it turns its 16 code bytes of a
 //              group into bf16 q - z (128 + q by bit placement, one packed subtraction of
