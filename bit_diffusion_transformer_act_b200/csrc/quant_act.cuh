@@ -245,6 +245,9 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
     }
   } else if (warp < kReadWarp0) {
     // ---------------------------------------------------------------- quantizers
+    // The first cluster barrier gates the sum of U over the slices; the quantizers publish
+    // nothing it reads, so they arrive now and the sum overlaps their last chunks.
+    cluster_arrive_relaxed();
     const int qt = tid - 64;                      // 0..255
     const int r = qt >> 1;                        // row of the chunk
     const int h = qt & 1;                         // columns [32 h, 32 h + 32) of the chunk
@@ -325,16 +328,24 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   }
 
   // ---------------------------------------------------------------- U = hi + lo, summed over the cluster
-  __syncthreads();                                 // every stage has been consumed: reuse them for U
-  float* upart = reinterpret_cast<float*>(gbase); // [128][32] fp32, 16-byte pieces rotated by the row
-  // Read out by warps 0, 1, 10 and 11 (lane quarters 0-3), which store nothing to global
-  // memory: their release arrival below does not wait for the quantizers' code stores.
+  // Read out by warps 0, 1, 10 and 11 (lane quarters 0-3) once the last MMA is done, while the
+  // quantizers may still be on their last chunks.  The partial goes to the ring slot after the
+  // last chunk's: free once its last chunk (nck - kStages) has been consumed, never used when
+  // nck < kStages.  Only these warps arrive at the first cluster barrier now (with release:
+  // their partials; none of them stores to global memory, so the arrival waits for nothing
+  // else); the quantizers arrived before their loop and wait on it after.
+  const int ks = p.kslices;
+  const int su = nck % kStages;
+  float* upart = reinterpret_cast<float*>(gbase + su * kStageBytes);   // [128][32] fp32, 16-byte pieces rotated by the row
   const bool reader = warp < 2 || warp >= kReadWarp0;
   if (reader) {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     float u[32];
-    if (__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full, 0, abort_flag, 14))) {
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full, 0, abort_flag, 14));
+    if (ok && nck >= kStages)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty(su), ((nck - kStages) / kStages) & 1u, abort_flag, 17));
+    if (ok) {
       tc_fence_after();
       uint32_t hi[32], lo[32];
       tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16), hi);
@@ -351,47 +362,48 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
     for (int j = 0; j < 8; ++j)
       *reinterpret_cast<float4*>(upart + row * 32 + ((j + row) & 7) * 4) =
           make_float4(u[j * 4], u[j * 4 + 1], u[j * 4 + 2], u[j * 4 + 3]);
-  }
-  const int ks = p.kslices;
-  tc_fence_before();
-  if (reader) cluster_arrive_release();            // partials of every slice in shared memory
-  else cluster_arrive_relaxed();
-  cluster_wait_acquire();
-  const uint32_t crank = cluster_ctarank();
-  const int rpc = kRows / ks;                      // rows finished by this CTA
-  for (int i = tid; i < rpc * 8; i += kThreads) {  // one 4-column piece of one row per thread
-    const int rr = static_cast<int>(crank) * rpc + i / 8;
-    const int piece = i % 8;
-    const float* src_addr = upart + rr * 32 + ((piece + rr) & 7) * 4;
-    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    tc_fence_before();
+    cluster_arrive_release();                      // this CTA's partial is in shared memory
+    cluster_wait_acquire();                        // ... and every other slice's
+    const uint32_t crank = cluster_ctarank();
+    const int rpc = kRows / ks;                    // rows finished by this CTA
+    const int rt = (warp < 2 ? warp : warp - kReadWarp0 + 2) * 32 + lane;   // 0..127
+    for (int i = rt; i < rpc * 8; i += 128) {      // one 4-column piece of one row per thread
+      const int rr = static_cast<int>(crank) * rpc + i / 8;
+      const int piece = i % 8;
+      const float* src_addr = upart + rr * 32 + ((piece + rr) & 7) * 4;
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-    for (int s0 = 0; s0 < ks; s0 += 8) {           // up to 16 slices, eight loads in flight at a time
-      float4 v[8];
+      for (int s0 = 0; s0 < ks; s0 += 8) {         // up to 16 slices, eight loads in flight at a time
+        float4 v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (s0 + j < ks) v[j] = ld_dsmem_f32x4(src_addr, static_cast<uint32_t>(s0 + j));
+        for (int j = 0; j < 8; ++j)
+          if (s0 + j < ks) v[j] = ld_dsmem_f32x4(src_addr, static_cast<uint32_t>(s0 + j));
 #pragma unroll
-      for (int j = 0; j < 8; ++j)                  // in slice order: deterministic
-        if (s0 + j < ks) {
-          if (s0 + j == 0) sum = v[0];
-          else { sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w; }
-        }
-    }
-    const int mm = m0 + rr;
-    if (mm < p.M) {
-      const float uu[4] = {sum.x * inv_g, sum.y * inv_g, sum.z * inv_g, sum.w * inv_g};  // exact
-      uint32_t hw[2], lw[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float h0 = __bfloat162float(__float2bfloat16_rn(uu[2 * j]));
-        const float h1 = __bfloat162float(__float2bfloat16_rn(uu[2 * j + 1]));
-        hw[j] = pack_bf16x2(h0, h1);
-        lw[j] = pack_bf16x2(uu[2 * j] - h0, uu[2 * j + 1] - h1);
+        for (int j = 0; j < 8; ++j)                // in slice order: deterministic
+          if (s0 + j < ks) {
+            if (s0 + j == 0) sum = v[0];
+            else { sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w; }
+          }
       }
-      __nv_bfloat16* dst = p.ucat + static_cast<size_t>(mm) * (2 * kRank) + piece * 4;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(hw[0], hw[1]);
-      *reinterpret_cast<uint2*>(dst + kRank) = make_uint2(lw[0], lw[1]);
+      const int mm = m0 + rr;
+      if (mm < p.M) {
+        const float uu[4] = {sum.x * inv_g, sum.y * inv_g, sum.z * inv_g, sum.w * inv_g};  // exact
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float h0 = __bfloat162float(__float2bfloat16_rn(uu[2 * j]));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(uu[2 * j + 1]));
+          hw[j] = pack_bf16x2(h0, h1);
+          lw[j] = pack_bf16x2(uu[2 * j] - h0, uu[2 * j + 1] - h1);
+        }
+        __nv_bfloat16* dst = p.ucat + static_cast<size_t>(mm) * (2 * kRank) + piece * 4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2*>(dst + kRank) = make_uint2(lw[0], lw[1]);
+      }
     }
+  } else {
+    cluster_wait_acquire();                        // the quantizers' arrival came before their loop
   }
   if (*abort_flag) {
     // a wait ran out: let the MMAs and copies already issued finish before the memory goes away
@@ -407,6 +419,7 @@ quant_act_lowrank_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_c
   }
   // the other CTAs are done reading this CTA's partials (their loads have returned: nothing
   // to order, so a relaxed arrival)
+  __syncwarp();
   cluster_arrive_relaxed();
   cluster_wait_acquire();
   if (warp == 1) {
