@@ -27,13 +27,14 @@
 // A stage is free again when the eight quantizer warps have read it and the MMAs
 // that read it have completed (tcgen05.commit).  At the end, warps 0, 1, 10 and 11
 // (one per tensor-memory lane quarter; none of them stores to global memory) read
-// U = hi + lo into shared memory, the cluster sums the slices, and U / g_a is written
-// split into bf16 hi + lo, the operand layout of the GEMM's low-rank MMA.  Only those
-// four warps arrive at the cluster barrier with release semantics (the quantizers'
-// pending code stores need not complete first), and the barrier that keeps shared
-// memory alive until the peers have read it is relaxed.  Every mbarrier wait is
-// bounded; a wait that runs out records SVDQ_ERR_TIMEOUT in the device status word
-// and the CTA winds down.
+// U = hi + lo into a ring slot that is already free as soon as the last MMA is done, the
+// cluster sums the slices, and U / g_a is written split into bf16 hi + lo, the operand
+// layout of the GEMM's low-rank MMA.  Only those four warps gate the first cluster
+// barrier (with release semantics): the quantizers arrive at it before their loop, so the
+// sum over the slices overlaps their last chunks; the barrier that keeps shared memory
+// alive until the peers have read it is relaxed.  Every mbarrier wait is bounded; a wait
+// that runs out records SVDQ_ERR_TIMEOUT in the device status word and the CTA winds
+// down.
 //
 // Rounding.  amax/6 is formed by a Markstein-corrected multiplication by the
 // rounded reciprocal of 6 (P. Markstein's correction: with y = RN(1/b) and
