@@ -10,8 +10,9 @@
 // Design (sm_100a, memory-bound).  Used for M <= 8 tokens (9..64 go to the tcgen05
 // kernel, awq_umma.cuh).  A CTA (one per SM) owns 128 output rows and all tokens and
 // streams its 128 x K/2 bytes of packed weights exactly once.  Warp 16 is the TMA producer:
-// first the CTA's scale and zero rows into shared memory (when K % 512 == 0 and K <= 4096;
-// else the consumers read them from global memory), then per 256-K stage one 128-row x
+// after the first weight tile, the CTA's scale and zero rows into shared memory (when
+// K % 512 == 0 and K <= 4096; else the consumers read them from global memory), then per
+// 256-K stage one 128-row x
 // 128-byte weight tile (128-byte swizzle) and the tokens' activations as four 64-column
 // sub-tiles (128-byte swizzle, rows past M read as zeros; the activations are shared by every
 // CTA and come from L2), paced: stage kb is requested once stage kb - 3 has landed (with every
