@@ -1,4 +1,7 @@
-"""GPU parity of the three kernels against the float64 oracle, through the C ABI.
+"""GPU parity of every kernel against the float64 oracle, through the C ABI: the SVDQ
+activation pass and GEMM (NVFP4 and int4 / group 64, static and dynamic activation scale),
+the fused QKV (RMSNorm + RoPE) and MLP-up (GELU + re-quantization) epilogues, and both AWQ
+W4A16 kernels.
 
 Bars: packed activation codes and scales bit-exact; the low-rank activations
 within fp32 accumulation error of the exact product; layer outputs within
