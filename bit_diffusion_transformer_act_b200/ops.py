@@ -471,7 +471,11 @@ def svdq_w4a4_nvfp4_linear_dyn(act_codes, act_scales, lowrank_act, act_amax, pac
 
 
 def awq_w4a16_linear(X, qweight, scales, zeros, bias=None, Y=None):
-    """X bf16 [M, K]; qweight uint8 [N, K/2]; scales, zeros bf16 [N, K/64]; bias bf16 [N] or None."""
+    """X bf16 [M, K]; qweight uint8 [N, K/2]; scales, zeros bf16 [N, K/64]; bias bf16 [N] or None.
+
+    With K % 512 == 0, K <= 4096 and scales / zeros 16-byte aligned (tensors of their own are)
+    the kernels stage the scale and zero rows in shared memory: the faster path, with results
+    bit-identical to those of any other alignment."""
     M, K = X.shape
     N = qweight.shape[0]
     _require(X, torch.bfloat16, (M, K), "X")
